@@ -1,0 +1,178 @@
+"""fp64 CPU oracle of the gated delta rule -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import this
+package.  The product path (``linear_attention_10_b200``) never imports, links or runs it, and this
+package imports nothing from the product path: the two share no code.
+
+What is computed and why (each function cites its source):
+
+* ``recurrence``  -- the gated delta rule token by token (``gdn_oracle.c``), the definition.
+* ``rows``        -- the same recurrence restricted to chosen rows of the state, for sampled checks
+                     of full-size workloads.
+* ``chunked``     -- the chunkwise WY/UT evaluation of the recurrence in fp64 for any chunk size
+                     (Ferrite project page, Design section 03 "Chunked Gated DeltaNet": chunks of
+                     32 rows, WY/UT form).
+* ``brute_force`` -- explicit d x d matrix products of the unrolled recurrence, numpy, for T <= 8.
+
+The recurrence (published gated delta rule, Yang, Kautz and Hatamizadeh, "Gated Delta Networks"):
+``S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T``, ``o_t = S_t q_t / sqrt(dk)``.
+Layouts: q, k ``[T, H, dk]``; v, o ``[T, H, dv]``; g, beta ``[T, H]``; state ``[N, H, dv, dk]``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libgdn_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``gdn_oracle.c`` into ``libgdn_oracle.so`` with gcc (fp64, no contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        dp = ctypes.POINTER(ctypes.c_double)
+        lp = ctypes.POINTER(ctypes.c_int64)
+        i64 = ctypes.c_int64
+        lib.gdn_oracle_recurrence.argtypes = [dp, dp, dp, dp, dp, lp, i64, dp, dp, dp, i64, i64, i64]
+        lib.gdn_oracle_rows.argtypes = [dp, dp, dp, dp, dp, lp, i64, dp, i64, i64, i64, i64,
+                                        lp, lp, lp, dp, dp]
+        lib.gdn_oracle_chunked.argtypes = [dp, dp, dp, dp, dp, lp, i64, dp, dp, dp, i64, i64, i64, i64]
+        for f in (lib.gdn_oracle_recurrence, lib.gdn_oracle_rows, lib.gdn_oracle_chunked):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _d(a):
+    """Contiguous fp64 copy (widening is exact for bf16 / fp32 inputs)."""
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a, typ=ctypes.c_double):
+    return None if a is None else a.ctypes.data_as(ctypes.POINTER(typ))
+
+
+def _cu(cu_seqlens, T):
+    if cu_seqlens is None:
+        return np.array([0, T], dtype=np.int64)
+    return np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+
+
+def _prep(q, k, v, g, beta, cu_seqlens, state_in):
+    q, k, v, g, beta = (_d(x) for x in (q, k, v, g, beta))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    cu = _cu(cu_seqlens, T)
+    assert k.shape == (T, H, dk) and v.shape[:2] == (T, H) and g.shape == (T, H) == beta.shape
+    assert cu[-1] == T
+    N = len(cu) - 1
+    s0 = None
+    if state_in is not None:
+        s0 = _d(state_in)
+        assert s0.shape == (N, H, dv, dk)
+    return q, k, v, g, beta, cu, s0, T, H, dk, dv, N
+
+
+def recurrence(q, k, v, g, beta, cu_seqlens=None, state_in=None):
+    """Token-by-token gated delta rule in fp64.  Returns ``(o [T,H,dv], state [N,H,dv,dk])``."""
+    q, k, v, g, beta, cu, s0, T, H, dk, dv, N = _prep(q, k, v, g, beta, cu_seqlens, state_in)
+    out = np.zeros((T, H, dv))
+    st = np.zeros((N, H, dv, dk))
+    rc = _load().gdn_oracle_recurrence(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                       _ptr(cu, ctypes.c_int64), N, _ptr(s0), _ptr(out), _ptr(st),
+                                       H, dk, dv)
+    if rc != 0:
+        raise ValueError("gdn_oracle_recurrence failed: %d" % rc)
+    return out, st
+
+
+def rows(q, k, v, g, beta, samples, cu_seqlens=None, state_in=None):
+    """Recurrence for sampled state rows.
+
+    ``samples`` is an int array ``[n, 3]`` of (sequence, head, row).  Returns ``(o_rows, s_rows)``:
+    ``o_rows[i, t]`` = o_t[h, r] for t in that sequence (NaN elsewhere), ``s_rows[i]`` = final
+    state row ``S[n, h, r, :]``.
+    """
+    q, k, v, g, beta, cu, s0, T, H, dk, dv, N = _prep(q, k, v, g, beta, cu_seqlens, state_in)
+    smp = np.ascontiguousarray(np.asarray(samples, dtype=np.int64).reshape(-1, 3))
+    n = smp.shape[0]
+    si, hi, ri = (np.ascontiguousarray(smp[:, j]) for j in range(3))
+    o_rows = np.full((n, T), np.nan)
+    s_rows = np.zeros((n, dk))
+    rc = _load().gdn_oracle_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                 _ptr(cu, ctypes.c_int64), N, _ptr(s0), H, dk, dv, n,
+                                 _ptr(si, ctypes.c_int64), _ptr(hi, ctypes.c_int64),
+                                 _ptr(ri, ctypes.c_int64), _ptr(o_rows), _ptr(s_rows))
+    if rc != 0:
+        raise ValueError("gdn_oracle_rows failed: %d" % rc)
+    return o_rows, s_rows
+
+
+def chunked(q, k, v, g, beta, chunk, cu_seqlens=None, state_in=None):
+    """Chunkwise WY/UT evaluation in fp64 with chunk size ``chunk``.  Same returns as ``recurrence``."""
+    q, k, v, g, beta, cu, s0, T, H, dk, dv, N = _prep(q, k, v, g, beta, cu_seqlens, state_in)
+    out = np.zeros((T, H, dv))
+    st = np.zeros((N, H, dv, dk))
+    rc = _load().gdn_oracle_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                    _ptr(cu, ctypes.c_int64), N, _ptr(s0), _ptr(out), _ptr(st),
+                                    H, dk, dv, int(chunk))
+    if rc != 0:
+        raise ValueError("gdn_oracle_chunked failed: %d" % rc)
+    return out, st
+
+
+def decode_step(q, k, v, g, beta, state):
+    """One recurrent step for B independent sequences: inputs ``[B, H, d]`` / ``[B, H]``, state
+    ``[B, H, dv, dk]``.  This is the recurrence over B sequences of length one."""
+    B = np.asarray(q).shape[0]
+    return recurrence(q, k, v, g, beta, cu_seqlens=np.arange(B + 1), state_in=state)
+
+
+def brute_force(q, k, v, g, beta, state_in=None):
+    """Unrolled recurrence with explicit matrices, one sequence, T <= 8 (numpy, fp64).
+
+    With A_t = exp(g_t) (I - beta_t k_t k_t^T) and B_t = beta_t v_t k_t^T:
+    ``S_t = S_0 A_1 ... A_t + sum_{j<=t} B_j A_{j+1} ... A_t``.  Each partial product is formed
+    explicitly as a d x d matrix; nothing is shared with the loop in ``gdn_oracle.c``.
+    """
+    q, k, v, g, beta = (_d(x) for x in (q, k, v, g, beta))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    assert T <= 8, "brute force is for tiny cases only"
+    out = np.zeros((T, H, dv))
+    st = np.zeros((H, dv, dk))
+    eye = np.eye(dk)
+    for h in range(H):
+        S0 = np.zeros((dv, dk)) if state_in is None else _d(state_in)[0, h]
+        A = [np.exp(g[t, h]) * (eye - beta[t, h] * np.outer(k[t, h], k[t, h])) for t in range(T)]
+        Bm = [beta[t, h] * np.outer(v[t, h], k[t, h]) for t in range(T)]
+        for t in range(T):
+            prod = eye.copy()
+            for s in range(t + 1):
+                prod = prod @ A[s]
+            St = S0 @ prod
+            for j in range(t + 1):
+                tail = eye.copy()
+                for s in range(j + 1, t + 1):
+                    tail = tail @ A[s]
+                St = St + Bm[j] @ tail
+            out[t, h] = St @ q[t, h] / np.sqrt(dk)
+            if t == T - 1:
+                st[h] = St
+    return out, st[None]
