@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark of the gated-delta-rule prefill (and decode step) on B200.
+
+``python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]``
+
+One step = one ``gdn_chunk_prefill`` call over the 4096-token workload (B=1, T=4096, H=32,
+dk=dv=128, bf16 q/k/v, fp32 g/beta, C=32, zero initial state, final state written).  Under torchrun
+every rank runs its own independent prefill (weak scaling, no data-path collective).  The line also
+carries the recurrent decode step (B=64, H=32, d=128, 1000 chained steps) as ``decode``.
+
+Timing: CUDA events on the launching stream, W warm-up steps, barrier + synchronize around the K
+timed steps, max over ranks.  L2: every step reads one of three rotating input sets (about 300 MB
+of q/k/v in total, above the 126 MB L2), so no step finds its inputs in L2.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "gated-delta-rule prefill tokens/s per layer (H=32,d=128); % of roofline"
+UNIT = "tokens/s"
+C = 32
+H, D, T_PREFILL = 32, 128, 4096
+WORKLOAD = "prefill_4k"
+WORKLOAD_DESC = ("B=1, T=4096, H=32, dk=dv=128, bf16 q/k/v (q,k L2-normalised), fp32 g=-softplus(N(0,1))*0.1 "
+                 "and beta=sigmoid(N(0,1)), zero initial state, C=32, fp32 final state")
+
+# Algorithmic work per (token, head), chunk size C, head size d (dk = dv = d):
+#   whole method      6 d^2 + 10 C d       (K K^T, Q K^T, W/U', intra-chunk P U, S-products, carry)
+#   chunk-parallel    8 C d                (K K^T 2Cd, Q K^T 2Cd, W and U' 4Cd)
+#   state-dependent   6 d^2 + 2 C d        (W S^T and Q S^T 4 d^2, P U 2 C d, carry 2 d^2)
+def flops_whole(d=D):
+    return 6 * d * d + 10 * C * d
+
+
+def flops_scan(d=D):
+    return 6 * d * d + 2 * C * d
+
+
+def flops_prep(d=D):
+    return 8 * C * d
+
+
+# Per-kernel roofline model.  "alu": fp32 CUDA-core FMAs, 1x the algorithmic flops, against the fp32
+# FMA peak derived from unit counts (148 SMs x 128 lanes x 2 flop x max SM clock).  "tensor": TF32
+# tensor cores with the 3xTF32 split, 3x the algorithmic flops, against the TF32 peak (measured
+# bf16 GEMM peak x nominal TF32/bf16 ratio 1.1/2.25).  "hbm": algorithmic bytes against the measured
+# copy bandwidth.
+KERNELS = {
+    "gdn_scan_kernel": dict(bound="alu", flops_per_token_head=flops_scan(), split=1),
+    "gdn_prep_kernel": dict(bound="alu", flops_per_token_head=flops_prep(), split=1),
+    "gdn_plan_kernel": dict(bound="latency"),
+    "gdn_decode_step_kernel": dict(bound="hbm"),
+}
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from the last ncu capture of that kernel
+# on the bench workload (None until captured, and reset whenever the kernel changes).
+TRAFFIC = {}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        j = json.load(open(p))
+        return dict(hbm_gbs=float(j["hbm_gbs"]), bf16_tflops=float(j["bf16_tflops"]),
+                    bf16_tflops_sustained=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                    sm_max_mhz=float(j.get("sm_max_mhz", 1965.0)), source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, sm_max_mhz=1965.0,
+                    source="fallback")
+
+
+def peak_for(bound, peaks):
+    if bound == "tensor":
+        return peaks["bf16_tflops"] * (1.1 / 2.25), "TFLOP/s", "%s bf16 GEMM x 1.1/2.25 (TF32)" % peaks["source"]
+    if bound == "alu":
+        return 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12, "TFLOP/s", "fp32 FMA: 148 SM x 128 x 2 x max clock"
+    if bound == "hbm":
+        return peaks["hbm_gbs"], "GB/s", "%s copy bandwidth" % peaks["source"]
+    return None, None, None
+
+
+# ---------------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id):
+        self.bus_id = (bus_id or "").lower()
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="gdn_clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            if self.bus_id and not self.bus_id.endswith(f[0].lower()[-len(self.bus_id):]) and \
+                    f[0].lower()[-12:] != self.bus_id[-12:]:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), util=float(f[4]),
+                                 reasons=[n for n, v in zip(("hw_slowdown", "hw_thermal_slowdown",
+                                                             "sw_thermal_slowdown", "sw_power_cap"), f[5:9])
+                                          if v.lower() == "active"]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        busy = [r for r in rows if r["util"] > 0] or rows
+        reasons = sorted({x for r in busy for x in r["reasons"]})
+        return dict(sm_mhz=statistics.median(r["sm"] for r in busy), sm_max_mhz=max(r["smax"] for r in rows),
+                    reasons=reasons, samples=len(busy))
+
+
+# ---------------------------------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and the reference arm)
+# ---------------------------------------------------------------------------------------------------
+def oracle_layer_rate(inp, budget_s=15.0, max_heads=None, tokens=None):
+    """Time the fp64 single-thread oracle over whole heads of the workload until ``budget_s`` is
+    spent; returns (tokens/s for the full layer of H heads, seconds, heads, tokens)."""
+    import numpy as np
+    import oracle
+    q, k, v, g, b = (inp[n].float().cpu().numpy().astype(np.float64) for n in ("q", "k", "v", "g", "beta"))
+    Tt = q.shape[0] if tokens is None else min(tokens, q.shape[0])
+    Hh = q.shape[1]
+    heads, spent = 0, 0.0
+    for h in range(Hh if max_heads is None else min(max_heads, Hh)):
+        sl = slice(h, h + 1)
+        t0 = time.perf_counter()
+        oracle.recurrence(q[:Tt, sl], k[:Tt, sl], v[:Tt, sl], g[:Tt, sl], b[:Tt, sl])
+        spent += time.perf_counter() - t0
+        heads += 1
+        if spent >= budget_s:
+            break
+    per_layer_s = spent / heads * Hh
+    return Tt / per_layer_s, spent, heads, Tt
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the fp64 CPU oracle, timed on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    import torch
+    from linear_attention_10_b200.workloads import workload_inputs
+    inp = workload_inputs(WORKLOAD, device="cpu")
+    q, k, v, g, b = (inp[n].float().numpy().astype(np.float64) for n in ("q", "k", "v", "g", "beta"))
+    # calibrate the cost of one token of one head, then size each step to keep the run short
+    t0 = time.perf_counter()
+    oracle.recurrence(q[:256, :1], k[:256, :1], v[:256, :1], g[:256, :1], b[:256, :1])
+    per_tok = (time.perf_counter() - t0) / 256
+    budget = 150.0
+    L = int(max(64, min(T_PREFILL, budget / max(args.steps + args.warmup, 1) / per_tok)))
+    times = []
+    for i in range(args.warmup + args.steps):
+        h = i % H
+        sl = slice(h, h + 1)
+        t0 = time.perf_counter()
+        oracle.recurrence(q[:L, sl], k[:L, sl], v[:L, sl], g[:L, sl], b[:L, sl])
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    per_step = sum(times) / len(times)           # seconds for L tokens of one head
+    value = L / (per_step * H)                   # tokens/s of a whole layer (H heads)
+    sample = "fp64 oracle recurrence, 1 head x %d tokens of the %s workload per step (layer rate = tokens / (step time x %d heads))" % (L, WORKLOAD, H)
+    line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
+                ms_per_step=per_step * 1e3, higher_is_better=True, scaling="weak", vs_baseline=None,
+                dtype="f64", data="synthetic", impl="reference",
+                config=dict(workload="%s: %s" % (WORKLOAD, WORKLOAD_DESC), global_batch=1, seq_len=T_PREFILL,
+                            parallelism="host CPU, 1 thread"),
+                cpu_baseline=dict(value=value, unit=UNIT, cores=1, kind="oracle", sample=sample),
+                e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from linear_attention_10_b200 import gdn
+    from linear_attention_10_b200.workloads import WORKLOADS, make_decode_inputs, workload_inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    gdn.lib()
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    # three rotating input sets (q/k/v of all three ~ 300 MB > L2)
+    sets = [workload_inputs(WORKLOAD, device=dev, seed=1000 * rank + i) for i in range(3)]
+    N = 1
+    ws = torch.empty(gdn.workspace_bytes(T_PREFILL, N, H, D, D), dtype=torch.uint8, device=dev)
+    out = torch.empty((T_PREFILL, H, D), dtype=torch.bfloat16, device=dev)
+    st_out = torch.empty((N, H, D, D), dtype=torch.float32, device=dev)
+
+    def step(i):
+        s = sets[i % 3]
+        gdn.gdn_chunk_prefill(s["q"], s["k"], s["v"], s["g"], s["beta"], cu_seqlens=s["cu_seqlens"],
+                              out=out, state_out=st_out, workspace=ws)
+
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    if gdn.gdn_get_device_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    bus = None
+    try:
+        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+    except Exception:
+        try:
+            p = torch.cuda.get_device_properties(dev)
+            bus = "%08x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+        except Exception:
+            bus = None
+    clocks = ClockSampler(bus if isinstance(bus, str) else None)
+    clocks.start()
+    time.sleep(0.3)
+
+    # ---- timed region: K prefill steps ----
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    gdn.gdn_profile_start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    prof = gdn.gdn_profile_stop()
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if gdn.gdn_get_device_status() != 0:
+        raise RuntimeError("device status error in the timed region")
+    ms_per_step = ms / args.steps
+    value = T_PREFILL * world * args.steps / (ms / 1e3)
+
+    # ---- e2e: host (pinned) inputs -> device -> prefill -> host outputs, every step ----
+    host = {n: sets[0][n].cpu().pin_memory() for n in ("q", "k", "v", "g", "beta", "cu_seqlens")}
+    dbuf = {n: torch.empty_like(sets[0][n]) for n in host}
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_st = torch.empty(st_out.shape, dtype=st_out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = h_out.numel() * h_out.element_size() + h_st.numel() * h_st.element_size()
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        for n in host:
+            dbuf[n].copy_(host[n], non_blocking=True)
+        gdn.gdn_chunk_prefill(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], cu_seqlens=dbuf["cu_seqlens"],
+                              out=out, state_out=st_out, workspace=ws)
+        h_out.copy_(out, non_blocking=True)
+        h_st.copy_(st_out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = T_PREFILL * world * e2e_steps / (e2e_ms / 1e3)
+
+    # ---- decode step: B=64, 1000 chained steps ----
+    decode = None
+    if not args.no_decode:
+        w = WORKLOADS["decode_b64"]
+        dd = make_decode_inputs(w.decode_batch, w.H, w.dk, w.dv, w.decode_steps, dtype=w.dtype, gate=w.gate,
+                                seed=w.seed + rank, state_std=w.state_std, device=dev)
+        S = dd["state"].clone()
+        dout = torch.empty((w.decode_batch, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+        for s in range(3):
+            gdn.gdn_decode_step(dd["q"][s], dd["k"][s], dd["v"][s], dd["g"][s], dd["beta"][s], S, out=dout)
+        S.copy_(dd["state"])
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        gdn.gdn_profile_start()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for s in range(w.decode_steps):
+            gdn.gdn_decode_step(dd["q"][s], dd["k"][s], dd["v"][s], dd["g"][s], dd["beta"][s], S, out=dout)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dprof = gdn.gdn_profile_stop()
+        dms = d0.elapsed_time(d1)
+        if world > 1:
+            t = torch.tensor([dms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            dms = float(t.item())
+        name = "gdn_decode_step_kernel"
+        kms, kl = dprof.get(name, (dms, w.decode_steps))
+        B_, H_, d_ = w.decode_batch, w.H, w.dk
+        bytes_per_launch = 2 * B_ * H_ * d_ * d_ * 4 + B_ * H_ * (3 * d_) * 2 + B_ * H_ * 2 * 4 + B_ * H_ * d_ * 2
+        ach = bytes_per_launch / (kms / kl / 1e3) / 1e9
+        pk, pu, pdesc = peak_for("hbm", peaks)
+        decode = dict(workload="decode_b64: B=64, H=32, dk=dv=128, bf16 q/k/v, fp32 state [64,32,128,128] in place, "
+                               "%d chained steps, fresh inputs per step" % w.decode_steps,
+                      value=B_ * world * w.decode_steps / (dms / 1e3), unit="tokens/s",
+                      us_per_step=dms / w.decode_steps * 1e3,
+                      roofline=dict(kernel=name, bound="hbm", achieved=ach, peak=pk, unit=pu, frac=ach / pk,
+                                    peak_source=pdesc, bytes_per_launch=bytes_per_launch,
+                                    traffic=TRAFFIC.get(name)))
+        del dd, S
+
+    clk = clocks.stop()
+
+    # ---- roofline of the dominant prefill kernel ----
+    dom = max((n for n in prof if n in KERNELS), key=lambda n: prof[n][0])
+    kms, kl = prof[dom]
+    spec = KERNELS[dom]
+    units = T_PREFILL * H                             # (token, head) pairs per launch
+    flops = spec["flops_per_token_head"] * spec["split"] * units
+    ach = flops / (kms / kl / 1e3) / 1e12
+    pk, pu, pdesc = peak_for(spec["bound"], peaks)
+    total_prof_ms = sum(v[0] for v in prof.values())
+    roofline = dict(kernel=dom, bound=spec["bound"], achieved=ach, peak=pk, unit=pu, frac=ach / pk,
+                    peak_source=pdesc, flops_per_launch=flops, avg_launch_us=kms / kl * 1e3,
+                    traffic=TRAFFIC.get(dom),
+                    kernels={n: dict(avg_us=v[0] / v[1] * 1e3, launches=v[1], share=v[0] / total_prof_ms)
+                             for n, v in prof.items()})
+    # whole-call roofline of the method (TF32 3x split vs HBM), as the metric defines "% of roofline"
+    tf32, _, _ = peak_for("tensor", peaks)
+    t_flop = 3 * flops_whole() * T_PREFILL * H / (tf32 * 1e12)
+    alg_bytes = 3 * T_PREFILL * H * D * 2 + 2 * T_PREFILL * H * 4 + T_PREFILL * H * D * 2 + N * H * D * D * 4
+    t_byte = alg_bytes / (peaks["hbm_gbs"] * 1e9)
+    roof_s = max(t_flop, t_byte)
+    method_roofline = dict(bound="tensor(TF32 x3)" if t_flop >= t_byte else "hbm", roofline_us=roof_s * 1e6,
+                           achieved_us=ms_per_step * 1e3, frac=roof_s / (ms_per_step / 1e3),
+                           tf32_peak_tflops=tf32, hbm_peak_gbs=peaks["hbm_gbs"])
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        rate, spent, heads, toks = oracle_layer_rate(sets[0], budget_s=args.cpu_seconds)
+        cpu = dict(value=rate, unit=UNIT, cores=1, kind="oracle",
+                   sample="fp64 single-thread oracle recurrence over %d of %d heads x %d tokens of the %s workload "
+                          "(%.1f s), scaled to a full layer" % (heads, H, toks, WORKLOAD, spent))
+
+    launches = sum(v[1] for v in prof.values())
+    line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
+                ms_per_step=ms_per_step, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f32",
+                data="synthetic",
+                config=dict(workload="%s: %s" % (WORKLOAD, WORKLOAD_DESC), global_batch=world, seq_len=T_PREFILL,
+                            parallelism="one independent prefill per GPU" if world > 1 else "1 GPU",
+                            l2="3 rotating input sets, ~300 MB of q/k/v > 126 MB L2"),
+                roofline=roofline, method_roofline=method_roofline, cpu_baseline=cpu,
+                e2e=dict(value=e2e_value, unit=UNIT, h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
+                         steps=e2e_steps),
+                gpu_launches=launches, clocks=clk, decode=decode)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,143 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) gated-delta-rule library, libgdn.so.
+ *
+ * The operation.  Ferrite project page (bhcc2025.github.io/ferrite), Design section 03 "Chunked
+ * Gated DeltaNet": a linear-attention layer keeps one recurrent state per request; prompt rows go
+ * through it in chunks of 32 using the chunkwise WY/UT form of the delta rule on TF32 tensor cores
+ * with a 3xTF32 split for fp32 accuracy, and the state is written back for decoding.  The state
+ * recurrence is the gated delta rule (Yang, Kautz and Hatamizadeh, "Gated Delta Networks"), per
+ * sequence and head:
+ *
+ *     S_t = exp(g_t) * S_{t-1} * (I - beta_t k_t k_t^T) + beta_t v_t k_t^T      (S is dv x dk)
+ *     o_t = S_t q_t / sqrt(dk)
+ *
+ * q_t and k_t must already be L2-normalised; the library does not normalise them.  g_t is the
+ * log-gate (alpha_t = exp(g_t); g <= 0 is the intended range but is not enforced); beta_t is used
+ * as given (intended range (0, 1), not enforced).
+ *
+ * Layouts (all row-major, contiguous, innermost index last):
+ *     q, k        [T_total, H, dk]     dtype GDN_F32 or GDN_BF16
+ *     v, out      [T_total, H, dv]     same dtype as q (out is written in that dtype)
+ *     g, beta     [T_total, H]         fp32
+ *     state       [N, H, dv, dk]       fp32 (dk contiguous: one row of S per dv index)
+ *     cu_seqlens  int32 [N + 1]        cu[0] = 0, non-decreasing, cu[N] = T_total
+ *
+ * Conventions shared by every entry point.
+ *   - Pointers named "device" must be device memory of the current CUDA device (or managed
+ *     memory); every such pointer must be 16-byte aligned (GDN_ERR_MISALIGNED otherwise).
+ *   - The caller owns every buffer; the library never allocates device memory in these calls.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  All work is
+ *     enqueued on it; no call synchronises the host except gdn_get_device_status.
+ *   - Return value: GDN_OK (0) when the work was enqueued, a negative GDN_ERR_* otherwise (nothing
+ *     is enqueued then).  Errors the host cannot see (bad cu_seqlens contents, an expired bounded
+ *     wait) are recorded by the kernels in a per-device status word; read it with
+ *     gdn_get_device_status.  Kernels never trap.
+ *   - Supported head sizes: dk, dv in {64, 128}.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Storage type of q, k, v and out. */
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
+
+/* Status codes. */
+enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = -1,  /* null required pointer, H < 1, N < 1, T < 0, bad dtype         */
+    GDN_ERR_UNSUPPORTED = -2,  /* dk or dv not in {64, 128}                                     */
+    GDN_ERR_MISALIGNED = -3,   /* a pointer is not 16-byte aligned                              */
+    GDN_ERR_LAUNCH = -4,       /* a kernel launch failed (the CUDA error is left pending)        */
+    GDN_ERR_WORKSPACE = -5,    /* workspace missing, misaligned (256 B) or smaller than needed   */
+    GDN_ERR_BAD_SEQLENS = -6,  /* device-detected: cu_seqlens not 0..T_total non-decreasing     */
+    GDN_ERR_TIMEOUT = -7,      /* device-detected: a bounded wait inside a kernel expired        */
+    GDN_ERR_CUDA = -8          /* a CUDA runtime call made by the library failed                */
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* gdn_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int gdn_version(void);
+
+/*
+ * Bytes of device workspace that gdn_chunk_prefill needs for this problem size.  Depends only on
+ * total_tokens, num_seqs, H and dk (chunk tables, the per-chunk WY/UT operator and gate data).
+ * Returns 0 for arguments that gdn_chunk_prefill would reject.
+ */
+size_t gdn_chunk_prefill_workspace_bytes(int64_t total_tokens, int num_seqs, int H, int dk, int dv);
+
+/*
+ * Chunked prefill (Ferrite project page, Design section 03): runs the gated delta rule over every
+ * token of N packed sequences, chunk size C = 32 with chunk boundaries relative to each sequence's
+ * start, and writes every output o_t and each sequence's final state.
+ *
+ *   q, k, v       device, layouts above, dtype `dtype`
+ *   g, beta       device fp32 [T_total, H]
+ *   cu_seqlens    device int32 [num_seqs + 1]; NULL means num_seqs sequences of equal length
+ *                 total_tokens / num_seqs (GDN_ERR_INVALID_ARG when that does not divide)
+ *   num_seqs      N >= 1
+ *   total_tokens  T_total >= 0, must equal cu_seqlens[N] (checked on the device)
+ *   state_in      device fp32 [N, H, dv, dk] initial states, or NULL for zero states
+ *   out           device [T_total, H, dv], dtype `dtype`; must not overlap any input
+ *   state_out     device fp32 [N, H, dv, dk] final states, or NULL (not written).  May equal
+ *                 state_in (in-place resume); must not overlap any other buffer otherwise.
+ *   workspace     device scratch of at least gdn_chunk_prefill_workspace_bytes(...) bytes,
+ *                 256-byte aligned; its contents on entry do not matter and are clobbered.  The
+ *                 workspace must not be used by another call that runs concurrently.
+ *
+ * Device-detected errors (GDN_ERR_BAD_SEQLENS) leave out and state_out unwritten.
+ */
+int gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* g,
+                      const float* beta, const int32_t* cu_seqlens, int num_seqs,
+                      int64_t total_tokens, const float* state_in, void* out, float* state_out,
+                      int H, int dk, int dv, int dtype, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/*
+ * Recurrent decode step (the consumer of the written-back state, Design section 03): one token for
+ * each of B sequences, state updated in place.
+ *
+ *   q, k          device [B, H, dk], dtype `dtype`
+ *   v             device [B, H, dv], dtype `dtype`
+ *   g, beta       device fp32 [B, H]
+ *   state_inout   device fp32 [B, H, dv, dk]; read once and overwritten with S_t
+ *   out           device [B, H, dv] in dtype `dtype`, or NULL (outputs not written)
+ */
+int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
+                    const float* beta, float* state_inout, void* out, int B, int H, int dk, int dv,
+                    int dtype, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of the current device:
+ * GDN_OK, or the first device-detected error (GDN_ERR_BAD_SEQLENS, GDN_ERR_TIMEOUT) recorded since
+ * the last read.  Returns GDN_ERR_CUDA when the synchronisation itself fails.
+ */
+int gdn_get_device_status(void* stream);
+
+/*
+ * Measurement aid (no counterpart on the pages): per-kernel device time of the library's own
+ * launches.  After gdn_profile_start, every kernel the library launches (from any host thread) is
+ * bracketed by a pair of CUDA events recorded on the launch's stream.  gdn_profile_stop
+ * synchronises those events, stops recording and aggregates by kernel name.
+ *
+ *   gdn_profile_start  GDN_OK, GDN_ERR_INVALID_ARG when already started, GDN_ERR_CUDA on failure.
+ *   gdn_profile_stop   returns the number of distinct kernels seen (>= 0) or a negative status;
+ *                      fills min(that, max_kernels) entries: names (host char[max_kernels][64],
+ *                      NUL-terminated, may be NULL), total_ms (host double[max_kernels], may be
+ *                      NULL; summed event time) and launches (host int[max_kernels], may be NULL).
+ */
+int gdn_profile_start(void);
+int gdn_profile_stop(int max_kernels, char* names, double* total_ms, int* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

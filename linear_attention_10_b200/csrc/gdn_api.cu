@@ -1,0 +1,311 @@
+// gdn_api.cu -- C ABI of libgdn.so: argument checks, workspace layout and kernel launches.
+//
+// Every entry point declared in include/gdn.h is defined here.  The kernels live in the .cuh files
+// included below, so the whole library is one translation unit and the per-device status word is
+// one symbol.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "gdn_common.cuh"
+#include "gdn_decode.cuh"
+#include "gdn_plan.cuh"
+#include "gdn_prefill_simt.cuh"
+
+namespace gdn {
+
+// First device-detected error since the last gdn_get_device_status (one per device).
+__device__ int g_status;
+
+static int* status_ptr()
+{
+    static std::mutex mu;
+    static int* cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+        cache[dev] = static_cast<int*>(p);
+    }
+    return cache[dev];
+}
+
+// ---- optional per-kernel event timing (gdn_profile_start / gdn_profile_stop) ----------------------
+struct ProfRec {
+    const char* name;
+    cudaEvent_t a, b;
+};
+static std::mutex g_prof_mu;
+static bool g_prof_on = false;
+static std::vector<ProfRec> g_prof_recs;
+static std::vector<cudaEvent_t> g_prof_pool;
+
+static cudaEvent_t prof_event()
+{
+    if (!g_prof_pool.empty()) {
+        cudaEvent_t e = g_prof_pool.back();
+        g_prof_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// Records an event pair around one launch when profiling is on.
+struct ProfScope {
+    ProfRec rec{nullptr, nullptr, nullptr};
+    cudaStream_t st;
+    ProfScope(const char* name, cudaStream_t s) : st(s)
+    {
+        std::lock_guard<std::mutex> lock(g_prof_mu);
+        if (!g_prof_on) return;
+        rec.name = name;
+        rec.a = prof_event();
+        rec.b = prof_event();
+        cudaEventRecord(rec.a, st);
+    }
+    ~ProfScope()
+    {
+        if (!rec.name) return;
+        cudaEventRecord(rec.b, st);
+        std::lock_guard<std::mutex> lock(g_prof_mu);
+        g_prof_recs.push_back(rec);
+    }
+};
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool head_ok(int d) { return d == 64 || d == 128; }
+
+template <typename T, int DK, int DV>
+static int launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                         float* state, void* out, int B, int H, cudaStream_t st)
+{
+    ProfScope prof("gdn_decode_step_kernel", st);
+    decode_step_kernel<T, DK, DV><<<(unsigned)B * H, 256, 0, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g, beta, state,
+        static_cast<T*>(out), H);
+    return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
+}
+
+template <typename T>
+static int dispatch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                           float* state, void* out, int B, int H, int dk, int dv, cudaStream_t st)
+{
+    if (dk == 128 && dv == 128) return launch_decode<T, 128, 128>(q, k, v, g, beta, state, out, B, H, st);
+    if (dk == 128 && dv == 64) return launch_decode<T, 128, 64>(q, k, v, g, beta, state, out, B, H, st);
+    if (dk == 64 && dv == 128) return launch_decode<T, 64, 128>(q, k, v, g, beta, state, out, B, H, st);
+    return launch_decode<T, 64, 64>(q, k, v, g, beta, state, out, B, H, st);
+}
+
+template <typename T, int DK, int DV>
+static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, const void* k, const void* v,
+                          const float* g, const float* beta, const int32_t* cu, int N, int64_t T_total,
+                          int fixed_len, const float* state_in, void* out, float* state_out, int H,
+                          cudaStream_t st)
+{
+    int* status = status_ptr();
+    if (!status) return GDN_ERR_CUDA;
+    int* meta = reinterpret_cast<int*>(ws + lay.off_meta);
+    int* chunk_off = reinterpret_cast<int*>(ws + lay.off_chunk_off);
+    int4* chunk_tab = reinterpret_cast<int4*>(ws + lay.off_chunk_tab);
+    float* op = reinterpret_cast<float*>(ws + lay.off_op);
+    float* aux = reinterpret_cast<float*>(ws + lay.off_aux);
+
+    {
+        ProfScope prof("gdn_plan_kernel", st);
+        plan_kernel<<<1, 1024, 0, st>>>(cu, N, T_total, fixed_len, meta, chunk_off, chunk_tab, status);
+    }
+    if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
+
+    constexpr int C = kChunk;
+    if (lay.nc_max > 0 && T_total > 0) {
+        const size_t smem1 = sizeof(float) * (3 * C * (DK + 1) + 3 * C * (C + 1) + 2 * C);
+        auto k1 = prep_simt_kernel<T, DK>;
+        if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) != cudaSuccess)
+            return GDN_ERR_LAUNCH;
+        ProfScope prof("gdn_prep_kernel", st);
+        k1<<<dim3((unsigned)lay.nc_max, H), 256, smem1, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                                              g, beta, meta, chunk_tab, op, aux, H);
+        if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
+    }
+    const size_t smem2 = sizeof(float) * (64 * (C + DK + 1) + C * (DK + 1) + 16 * (DK + 1) + 2 * C * 16);
+    auto k2 = scan_simt_kernel<T, DK, DV>;
+    if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) != cudaSuccess)
+        return GDN_ERR_LAUNCH;
+    {
+        ProfScope prof("gdn_scan_kernel", st);
+        k2<<<dim3((unsigned)N, H, DV / 16), 256, smem2, st>>>(static_cast<const T*>(k), static_cast<const T*>(v),
+                                                              meta, chunk_off, chunk_tab, op, aux, state_in,
+                                                              static_cast<T*>(out), state_out, H);
+    }
+    return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
+}
+
+template <typename T>
+static int dispatch_prefill(int dk, int dv, const PrefillLayout& lay, char* ws, const void* q, const void* k,
+                            const void* v, const float* g, const float* beta, const int32_t* cu, int N,
+                            int64_t T_total, int fixed_len, const float* state_in, void* out,
+                            float* state_out, int H, cudaStream_t st)
+{
+#define GDN_PF(DK_, DV_)                                                                                   \
+    if (dk == DK_ && dv == DV_)                                                                            \
+        return launch_prefill<T, DK_, DV_>(lay, ws, q, k, v, g, beta, cu, N, T_total, fixed_len, state_in, \
+                                           out, state_out, H, st);
+    GDN_PF(128, 128)
+    GDN_PF(128, 64)
+    GDN_PF(64, 128)
+    GDN_PF(64, 64)
+#undef GDN_PF
+    return GDN_ERR_UNSUPPORTED;
+}
+
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+const char* gdn_status_string(int s)
+{
+    switch (s) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: invalid argument";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: dk and dv must be 64 or 128";
+    case GDN_ERR_MISALIGNED: return "GDN_ERR_MISALIGNED: pointers must be 16-byte aligned";
+    case GDN_ERR_LAUNCH: return "GDN_ERR_LAUNCH: kernel launch failed";
+    case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case GDN_ERR_BAD_SEQLENS: return "GDN_ERR_BAD_SEQLENS: cu_seqlens is not 0..T_total non-decreasing";
+    case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT: a bounded wait inside a kernel expired";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA: a CUDA runtime call failed";
+    default: return "unknown gdn status";
+    }
+}
+
+int gdn_version(void) { return 100; }
+
+size_t gdn_chunk_prefill_workspace_bytes(int64_t total_tokens, int num_seqs, int H, int dk, int dv)
+{
+    if (total_tokens < 0 || num_seqs < 1 || H < 1 || !head_ok(dk) || !head_ok(dv)) return 0;
+    return PrefillLayout(total_tokens, num_seqs, H, dk).total;
+}
+
+int gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                      const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens, const float* state_in,
+                      void* out, float* state_out, int H, int dk, int dv, int dtype, void* workspace,
+                      size_t workspace_bytes, void* stream)
+{
+    if (num_seqs < 1 || H < 1 || total_tokens < 0 || total_tokens > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!head_ok(dk) || !head_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return GDN_ERR_INVALID_ARG;
+    int fixed_len = 0;
+    if (!cu_seqlens) {
+        if (total_tokens % num_seqs != 0) return GDN_ERR_INVALID_ARG;
+        fixed_len = (int)(total_tokens / num_seqs);
+    }
+    const void* ptrs[] = {q, k, v, g, beta, cu_seqlens, state_in, out, state_out};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    PrefillLayout lay(total_tokens, num_seqs, H, dk);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < lay.total)
+        return GDN_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    if (dtype == GDN_F32)
+        return dispatch_prefill<float>(dk, dv, lay, ws, q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
+                                       fixed_len, state_in, out, state_out, H, st);
+    return dispatch_prefill<__nv_bfloat16>(dk, dv, lay, ws, q, k, v, g, beta, cu_seqlens, num_seqs,
+                                           total_tokens, fixed_len, state_in, out, state_out, H, st);
+}
+
+int gdn_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                    float* state_inout, void* out, int B, int H, int dk, int dv, int dtype, void* stream)
+{
+    if (B < 0 || H < 1) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!head_ok(dk) || !head_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    if (B == 0) return GDN_OK;
+    if (!q || !k || !v || !g || !beta || !state_inout) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, beta, state_inout, out};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    if ((int64_t)B * H > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == GDN_F32) return dispatch_decode<float>(q, k, v, g, beta, state_inout, out, B, H, dk, dv, st);
+    return dispatch_decode<__nv_bfloat16>(q, k, v, g, beta, state_inout, out, B, H, dk, dv, st);
+}
+
+int gdn_get_device_status(void* stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDN_ERR_CUDA;
+    int* p = status_ptr();
+    if (!p) return GDN_ERR_CUDA;
+    int v = 0, zero = 0;
+    if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return GDN_ERR_CUDA;
+    return v;
+}
+
+int gdn_profile_start(void)
+{
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    if (g_prof_on) return GDN_ERR_INVALID_ARG;
+    for (int i = 0; i < 256; ++i) {
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreate(&e) != cudaSuccess) return GDN_ERR_CUDA;
+        g_prof_pool.push_back(e);
+    }
+    g_prof_recs.clear();
+    g_prof_on = true;
+    return GDN_OK;
+}
+
+int gdn_profile_stop(int max_kernels, char* names, double* total_ms, int* launches)
+{
+    std::vector<ProfRec> recs;
+    {
+        std::lock_guard<std::mutex> lock(g_prof_mu);
+        if (!g_prof_on) return GDN_ERR_INVALID_ARG;
+        g_prof_on = false;
+        recs.swap(g_prof_recs);
+    }
+    std::vector<std::string> uniq;
+    std::vector<double> tot;
+    std::vector<int> cnt;
+    int rc = GDN_OK;
+    for (const ProfRec& r : recs) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+            rc = GDN_ERR_CUDA;
+        size_t i = 0;
+        while (i < uniq.size() && uniq[i] != r.name) ++i;
+        if (i == uniq.size()) { uniq.push_back(r.name); tot.push_back(0.0); cnt.push_back(0); }
+        tot[i] += ms;
+        cnt[i] += 1;
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    {
+        std::lock_guard<std::mutex> lock(g_prof_mu);
+        for (cudaEvent_t e : g_prof_pool) cudaEventDestroy(e);
+        g_prof_pool.clear();
+    }
+    if (rc != GDN_OK) return rc;
+    const int n = (int)uniq.size();
+    for (int i = 0; i < n && i < max_kernels; ++i) {
+        if (names) {
+            snprintf(names + 64 * i, 64, "%s", uniq[i].c_str());
+        }
+        if (total_ms) total_ms[i] = tot[i];
+        if (launches) launches[i] = cnt[i];
+    }
+    return n;
+}
+
+}  // extern "C"

@@ -1,0 +1,112 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every entry point that
+include/gdn.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_10_b200 import build as gdn_build
+from linear_attention_10_b200 import gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    gdn_build.build()
+    return gdn.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]*?\b(gdn_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for n in ("gdn_chunk_prefill", "gdn_decode_step", "gdn_get_device_status", "gdn_status_string",
+              "gdn_chunk_prefill_workspace_bytes", "gdn_version"):
+        assert n in names
+    assert set(names) == set(gdn.EXPORTS), names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_status_strings(L):
+    for code in range(0, -9, -1):
+        s = gdn.status_string(code)
+        assert s and "unknown" not in s
+    assert "unknown" in gdn.status_string(-99)
+    assert L.gdn_version() >= 100
+
+
+def test_workspace_bytes(L):
+    w = gdn.workspace_bytes
+    assert w(4096, 1, 32, 128, 128) > 0
+    assert w(0, 1, 32, 128, 128) > 0
+    assert w(4096, 1, 32, 96, 128) == 0          # unsupported head size
+    assert w(-1, 1, 32, 128, 128) == 0
+    assert w(4096, 0, 32, 128, 128) == 0
+    assert w(8192, 1, 32, 128, 128) >= w(4096, 1, 32, 128, 128)
+    assert w(4096, 1, 32, 128, 128) % 256 == 0
+
+
+FAKE = 1 << 20   # 16-byte aligned non-null address; never dereferenced on these paths
+
+
+def prefill(L, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu=FAKE, N=1, T=64, s_in=None, out=FAKE,
+             s_out=FAKE, H=2, dk=64, dv=64, dtype=1, ws=FAKE, ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return L.gdn_chunk_prefill(a["q"], a["k"], a["v"], a["g"], a["beta"], a["cu"], a["N"], a["T"], a["s_in"],
+                               a["out"], a["s_out"], a["H"], a["dk"], a["dv"], a["dtype"], a["ws"],
+                               a["ws_bytes"], a["stream"])
+
+
+def test_prefill_rejects_bad_arguments(L):
+    assert prefill(L, q=None) == -1
+    assert prefill(L, out=None) == -1
+    assert prefill(L, N=0) == -1
+    assert prefill(L, H=0) == -1
+    assert prefill(L, T=-1) == -1
+    assert prefill(L, dtype=7) == -1
+    assert prefill(L, cu=None, N=3, T=64) == -1        # 64 tokens do not split into 3 equal sequences
+    assert prefill(L, dk=96) == -2
+    assert prefill(L, dv=32) == -2
+    assert prefill(L, k=FAKE + 4) == -3
+    assert prefill(L, s_out=FAKE + 8) == -3
+    assert prefill(L, ws=None) == -5
+    assert prefill(L, ws=FAKE + 16) == -5              # workspace must be 256-byte aligned
+    assert prefill(L, ws_bytes=16) == -5
+
+
+def decode(L, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, s=FAKE, out=FAKE, B=4, H=2, dk=128, dv=128, dtype=1,
+             stream=None)
+    a.update(kw)
+    return L.gdn_decode_step(a["q"], a["k"], a["v"], a["g"], a["beta"], a["s"], a["out"], a["B"], a["H"],
+                             a["dk"], a["dv"], a["dtype"], a["stream"])
+
+
+def test_decode_rejects_bad_arguments(L):
+    assert decode(L, s=None) == -1
+    assert decode(L, H=0) == -1
+    assert decode(L, B=-1) == -1
+    assert decode(L, dtype=3) == -1
+    assert decode(L, dk=32) == -2
+    assert decode(L, v=FAKE + 2) == -3
+    assert decode(L, B=0) == 0                          # nothing to do, nothing enqueued
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(gdn, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(gdn, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        gdn.lib()
