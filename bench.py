@@ -56,8 +56,8 @@ def flops_prep(d=D):
 # bf16 GEMM peak x nominal TF32/bf16 ratio 1.1/2.25).  "hbm": algorithmic bytes against the measured
 # copy bandwidth.
 KERNELS = {
-    "gdn_scan_kernel": dict(bound="alu", flops_per_token_head=flops_scan(), split=1),
-    "gdn_prep_kernel": dict(bound="alu", flops_per_token_head=flops_prep(), split=1),
+    "gdn_scan_simt_kernel": dict(bound="alu", flops_per_token_head=flops_scan(), split=1),
+    "gdn_prep_simt_kernel": dict(bound="alu", flops_per_token_head=flops_prep(), split=1),
     "gdn_plan_kernel": dict(bound="latency"),
     "gdn_decode_step_kernel": dict(bound="hbm"),
 }

@@ -24,7 +24,8 @@
  *
  * Conventions shared by every entry point.
  *   - Pointers named "device" must be device memory of the current CUDA device (or managed
- *     memory); every such pointer must be 16-byte aligned (GDN_ERR_MISALIGNED otherwise).
+ *     memory).  q, k, v, out and state pointers must be 16-byte aligned, g, beta and cu_seqlens
+ *     4-byte aligned (GDN_ERR_MISALIGNED otherwise).
  *   - The caller owns every buffer; the library never allocates device memory in these calls.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  All work is
  *     enqueued on it; no call synchronises the host except gdn_get_device_status.
@@ -52,7 +53,7 @@ enum {
     GDN_OK = 0,
     GDN_ERR_INVALID_ARG = -1,  /* null required pointer, H < 1, N < 1, T < 0, bad dtype         */
     GDN_ERR_UNSUPPORTED = -2,  /* dk or dv not in {64, 128}                                     */
-    GDN_ERR_MISALIGNED = -3,   /* a pointer is not 16-byte aligned                              */
+    GDN_ERR_MISALIGNED = -3,   /* a pointer breaks the alignment rule above                     */
     GDN_ERR_LAUNCH = -4,       /* a kernel launch failed (the CUDA error is left pending)        */
     GDN_ERR_WORKSPACE = -5,    /* workspace missing, misaligned (256 B) or smaller than needed   */
     GDN_ERR_BAD_SEQLENS = -6,  /* device-detected: cu_seqlens not 0..T_total non-decreasing     */

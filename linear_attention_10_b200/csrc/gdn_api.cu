@@ -80,6 +80,7 @@ struct ProfScope {
 };
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 static bool head_ok(int d) { return d == 64 || d == 128; }
 
 template <typename T, int DK, int DV>
@@ -87,7 +88,7 @@ static int launch_decode(const void* q, const void* k, const void* v, const floa
                          float* state, void* out, int B, int H, cudaStream_t st)
 {
     ProfScope prof("gdn_decode_step_kernel", st);
-    decode_step_kernel<T, DK, DV><<<(unsigned)B * H, 256, 0, st>>>(
+    gdn_decode_step_kernel<T, DK, DV><<<(unsigned)B * H, 256, 0, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g, beta, state,
         static_cast<T*>(out), H);
     return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
@@ -119,27 +120,27 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
 
     {
         ProfScope prof("gdn_plan_kernel", st);
-        plan_kernel<<<1, 1024, 0, st>>>(cu, N, T_total, fixed_len, meta, chunk_off, chunk_tab, status);
+        gdn_plan_kernel<<<1, 1024, 0, st>>>(cu, N, T_total, fixed_len, meta, chunk_off, chunk_tab, status);
     }
     if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
 
     constexpr int C = kChunk;
     if (lay.nc_max > 0 && T_total > 0) {
         const size_t smem1 = sizeof(float) * (3 * C * (DK + 1) + 3 * C * (C + 1) + 2 * C);
-        auto k1 = prep_simt_kernel<T, DK>;
+        auto k1 = gdn_prep_simt_kernel<T, DK>;
         if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) != cudaSuccess)
             return GDN_ERR_LAUNCH;
-        ProfScope prof("gdn_prep_kernel", st);
+        ProfScope prof("gdn_prep_simt_kernel", st);
         k1<<<dim3((unsigned)lay.nc_max, H), 256, smem1, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
                                                               g, beta, meta, chunk_tab, op, aux, H);
         if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
     }
     const size_t smem2 = sizeof(float) * (64 * (C + DK + 1) + C * (DK + 1) + 16 * (DK + 1) + 2 * C * 16);
-    auto k2 = scan_simt_kernel<T, DK, DV>;
+    auto k2 = gdn_scan_simt_kernel<T, DK, DV>;
     if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) != cudaSuccess)
         return GDN_ERR_LAUNCH;
     {
-        ProfScope prof("gdn_scan_kernel", st);
+        ProfScope prof("gdn_scan_simt_kernel", st);
         k2<<<dim3((unsigned)N, H, DV / 16), 256, smem2, st>>>(static_cast<const T*>(k), static_cast<const T*>(v),
                                                               meta, chunk_off, chunk_tab, op, aux, state_in,
                                                               static_cast<T*>(out), state_out, H);
@@ -177,7 +178,7 @@ const char* gdn_status_string(int s)
     case GDN_OK: return "GDN_OK";
     case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: invalid argument";
     case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: dk and dv must be 64 or 128";
-    case GDN_ERR_MISALIGNED: return "GDN_ERR_MISALIGNED: pointers must be 16-byte aligned";
+    case GDN_ERR_MISALIGNED: return "GDN_ERR_MISALIGNED: q/k/v/out/state need 16-byte, g/beta/cu_seqlens 4-byte alignment";
     case GDN_ERR_LAUNCH: return "GDN_ERR_LAUNCH: kernel launch failed";
     case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace missing, misaligned or too small";
     case GDN_ERR_BAD_SEQLENS: return "GDN_ERR_BAD_SEQLENS: cu_seqlens is not 0..T_total non-decreasing";
@@ -209,9 +210,12 @@ int gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* 
         if (total_tokens % num_seqs != 0) return GDN_ERR_INVALID_ARG;
         fixed_len = (int)(total_tokens / num_seqs);
     }
-    const void* ptrs[] = {q, k, v, g, beta, cu_seqlens, state_in, out, state_out};
+    const void* ptrs[] = {q, k, v, state_in, out, state_out};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    const void* small[] = {g, beta, cu_seqlens};
+    for (const void* p : small)
+        if (p && !aligned4(p)) return GDN_ERR_MISALIGNED;
     PrefillLayout lay(total_tokens, num_seqs, H, dk);
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < lay.total)
         return GDN_ERR_WORKSPACE;
@@ -232,9 +236,10 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
     if (!head_ok(dk) || !head_ok(dv)) return GDN_ERR_UNSUPPORTED;
     if (B == 0) return GDN_OK;
     if (!q || !k || !v || !g || !beta || !state_inout) return GDN_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, g, beta, state_inout, out};
+    const void* ptrs[] = {q, k, v, state_inout, out};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    if (!aligned4(g) || !aligned4(beta)) return GDN_ERR_MISALIGNED;
     if ((int64_t)B * H > INT32_MAX) return GDN_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dtype == GDN_F32) return dispatch_decode<float>(q, k, v, g, beta, state_inout, out, B, H, dk, dv, st);

@@ -21,7 +21,7 @@
 namespace gdn {
 
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(256) decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(256) gdn_decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                           const T* __restrict__ v, const float* __restrict__ g,
                                                           const float* __restrict__ beta, float* state,
                                                           T* __restrict__ out, int H)

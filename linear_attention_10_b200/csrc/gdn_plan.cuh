@@ -64,7 +64,7 @@ __device__ __forceinline__ int block_inclusive_scan_1024(int x, int* warp_tot)
 }
 
 // <<<1, 1024>>>.  cu_seqlens may be null: N sequences of equal length `fixed_len`.
-__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ cu, int N, int64_t T,
+__global__ void __launch_bounds__(1024) gdn_plan_kernel(const int32_t* __restrict__ cu, int N, int64_t T,
                                                     int fixed_len, int* meta, int* chunk_off,
                                                     int4* chunk_tab, int* status)
 {

@@ -34,7 +34,7 @@ namespace gdn {
 // Kernel 1: per (chunk, head) operator M and exp(gamma_31).  grid (nc_max, H), 256 threads.
 // ------------------------------------------------------------------------------------------------
 template <typename T, int DK>
-__global__ void __launch_bounds__(256) prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(256) gdn_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                         const float* __restrict__ g,
                                                         const float* __restrict__ beta,
                                                         const int* __restrict__ meta,
@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(256) prep_simt_kernel(const T* __restrict__ q,
 // Each CTA owns 16 rows of one head's state (rows of S evolve independently).
 // ------------------------------------------------------------------------------------------------
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(256) scan_simt_kernel(const T* __restrict__ k, const T* __restrict__ v,
+__global__ void __launch_bounds__(256) gdn_scan_simt_kernel(const T* __restrict__ k, const T* __restrict__ v,
                                                         const int* __restrict__ meta,
                                                         const int* __restrict__ chunk_off,
                                                         const int4* __restrict__ chunk_tab,

@@ -82,6 +82,8 @@ def test_prefill_rejects_bad_arguments(L):
     assert prefill(L, dv=32) == -2
     assert prefill(L, k=FAKE + 4) == -3
     assert prefill(L, s_out=FAKE + 8) == -3
+    assert prefill(L, beta=FAKE + 2) == -3
+    assert prefill(L, cu=FAKE + 1) == -3
     assert prefill(L, ws=None) == -5
     assert prefill(L, ws=FAKE + 16) == -5              # workspace must be 256-byte aligned
     assert prefill(L, ws_bytes=16) == -5
@@ -102,6 +104,7 @@ def test_decode_rejects_bad_arguments(L):
     assert decode(L, dtype=3) == -1
     assert decode(L, dk=32) == -2
     assert decode(L, v=FAKE + 2) == -3
+    assert decode(L, g=FAKE + 2) == -3
     assert decode(L, B=0) == 0                          # nothing to do, nothing enqueued
 
 
