@@ -56,8 +56,8 @@ def flops_prep(d=D):
 # bf16 GEMM peak x nominal TF32/bf16 ratio 1.1/2.25).  "hbm": algorithmic bytes against the measured
 # copy bandwidth.
 KERNELS = {
-    "gdn_scan_simt_kernel": dict(bound="alu", flops_per_token_head=flops_scan(), split=1),
-    "gdn_prep_simt_kernel": dict(bound="alu", flops_per_token_head=flops_prep(), split=1),
+    "gdn_scan_tc_kernel": dict(bound="tensor", flops_per_token_head=flops_scan(), split=3),
+    "gdn_prep_kernel": dict(bound="tensor", flops_per_token_head=flops_prep(), split=3),
     "gdn_plan_kernel": dict(bound="latency"),
     "gdn_decode_step_kernel": dict(bound="hbm"),
 }
@@ -86,6 +86,25 @@ def peak_for(bound, peaks):
     if bound == "hbm":
         return peaks["hbm_gbs"], "GB/s", "%s copy bandwidth" % peaks["source"]
     return None, None, None
+
+
+# ---------------------------------------------------------------------------------------------------
+# multi-rank timing: every rank times its own independent work; the job is as slow as its slowest rank
+# ---------------------------------------------------------------------------------------------------
+def max_over_ranks(x, world, device=None):
+    """Maximum of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step, steps, world, max_ms):
+    """Whole-job units per second: all ranks' units over the slowest rank's time."""
+    return units_per_rank_step * world * steps / (max_ms / 1e3)
 
 
 # ---------------------------------------------------------------------------------------------------
@@ -266,15 +285,11 @@ def run_ours(args, rank, world, local_rank):
     prof = gdn.gdn_profile_stop()
     if world > 1:
         dist.barrier()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     if gdn.gdn_get_device_status() != 0:
         raise RuntimeError("device status error in the timed region")
     ms_per_step = ms / args.steps
-    value = T_PREFILL * world * args.steps / (ms / 1e3)
+    value = job_throughput(T_PREFILL, args.steps, world, ms)
 
     # ---- e2e: host (pinned) inputs -> device -> prefill -> host outputs, every step ----
     host = {n: sets[0][n].cpu().pin_memory() for n in ("q", "k", "v", "g", "beta", "cu_seqlens")}
@@ -304,12 +319,8 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = T_PREFILL * world * e2e_steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = job_throughput(T_PREFILL, e2e_steps, world, e2e_ms)
 
     # ---- decode step: B=64, 1000 chained steps ----
     decode = None
@@ -333,11 +344,7 @@ def run_ours(args, rank, world, local_rank):
         d1.record(stream)
         torch.cuda.synchronize()
         dprof = gdn.gdn_profile_stop()
-        dms = d0.elapsed_time(d1)
-        if world > 1:
-            t = torch.tensor([dms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            dms = float(t.item())
+        dms = max_over_ranks(d0.elapsed_time(d1), world, dev)
         name = "gdn_decode_step_kernel"
         kms, kl = dprof.get(name, (dms, w.decode_steps))
         B_, H_, d_ = w.decode_batch, w.H, w.dk
@@ -346,7 +353,7 @@ def run_ours(args, rank, world, local_rank):
         pk, pu, pdesc = peak_for("hbm", peaks)
         decode = dict(workload="decode_b64: B=64, H=32, dk=dv=128, bf16 q/k/v, fp32 state [64,32,128,128] in place, "
                                "%d chained steps, fresh inputs per step" % w.decode_steps,
-                      value=B_ * world * w.decode_steps / (dms / 1e3), unit="tokens/s",
+                      value=job_throughput(B_, w.decode_steps, world, dms), unit="tokens/s",
                       us_per_step=dms / w.decode_steps * 1e3,
                       roofline=dict(kernel=name, bound="hbm", achieved=ach, peak=pk, unit=pu, frac=ach / pk,
                                     peak_source=pdesc, bytes_per_launch=bytes_per_launch,
@@ -356,7 +363,7 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
 
     # ---- roofline of the dominant prefill kernel ----
-    dom = max((n for n in prof if n in KERNELS), key=lambda n: prof[n][0])
+    dom = max((n for n in prof if "flops_per_token_head" in KERNELS.get(n, {})), key=lambda n: prof[n][0])
     kms, kl = prof[dom]
     spec = KERNELS[dom]
     units = T_PREFILL * H                             # (token, head) pairs per launch
@@ -388,7 +395,7 @@ def run_ours(args, rank, world, local_rank):
 
     launches = sum(v[1] for v in prof.values())
     line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
-                ms_per_step=ms_per_step, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f32",
+                ms_per_step=ms_per_step, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="tf32x3",
                 data="synthetic",
                 config=dict(workload="%s: %s" % (WORKLOAD, WORKLOAD_DESC), global_batch=world, seq_len=T_PREFILL,
                             parallelism="one independent prefill per GPU" if world > 1 else "1 GPU",

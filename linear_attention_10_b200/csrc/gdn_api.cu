@@ -13,7 +13,7 @@
 #include "gdn_common.cuh"
 #include "gdn_decode.cuh"
 #include "gdn_plan.cuh"
-#include "gdn_prefill_simt.cuh"
+#include "gdn_prefill_tc.cuh"
 
 namespace gdn {
 
@@ -104,6 +104,8 @@ static int dispatch_decode(const void* q, const void* k, const void* v, const fl
     return launch_decode<T, 64, 64>(q, k, v, g, beta, state, out, B, H, st);
 }
 
+static int g_num_sms = 0;
+
 template <typename T, int DK, int DV>
 static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, const void* k, const void* v,
                           const float* g, const float* beta, const int32_t* cu, int N, int64_t T_total,
@@ -116,7 +118,11 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
     int* chunk_off = reinterpret_cast<int*>(ws + lay.off_chunk_off);
     int4* chunk_tab = reinterpret_cast<int4*>(ws + lay.off_chunk_tab);
     float* op = reinterpret_cast<float*>(ws + lay.off_op);
-    float* aux = reinterpret_cast<float*>(ws + lay.off_aux);
+    if (g_num_sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) g_num_sms = 148;
+    }
 
     {
         ProfScope prof("gdn_plan_kernel", st);
@@ -124,26 +130,32 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
     }
     if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
 
-    constexpr int C = kChunk;
     if (lay.nc_max > 0 && T_total > 0) {
-        const size_t smem1 = sizeof(float) * (3 * C * (DK + 1) + 3 * C * (C + 1) + 2 * C);
-        auto k1 = gdn_prep_simt_kernel<T, DK>;
-        if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) != cudaSuccess)
+        using PL = PrepSmem<T, DK>;
+        auto k1 = gdn_prep_kernel<T, DK>;
+        if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PL::kBytes) != cudaSuccess)
             return GDN_ERR_LAUNCH;
-        ProfScope prof("gdn_prep_simt_kernel", st);
-        k1<<<dim3((unsigned)lay.nc_max, H), 256, smem1, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
-                                                              g, beta, meta, chunk_tab, op, aux, H);
+        const int64_t items = lay.nc_max * (int64_t)H;
+        const int64_t cap = (int64_t)g_num_sms * 4;
+        const unsigned grid = (unsigned)(items < cap ? items : cap);
+        ProfScope prof("gdn_prep_kernel", st);
+        k1<<<grid, 128, PL::kBytes, st>>>(static_cast<const T*>(q), static_cast<const T*>(k), g, beta, meta,
+                                          chunk_tab, op, H, status);
         if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
     }
-    const size_t smem2 = sizeof(float) * (64 * (C + DK + 1) + C * (DK + 1) + 16 * (DK + 1) + 2 * C * 16);
-    auto k2 = gdn_scan_simt_kernel<T, DK, DV>;
-    if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) != cudaSuccess)
+    constexpr int MS = 32;
+    using S2 = ScanSmem<T, DK, MS, 2>;
+    constexpr int STAGES = (S2::kBytes <= 227 * 1024) ? 2 : 1;
+    using SL = ScanSmem<T, DK, MS, STAGES>;
+    static_assert(SL::kBytes <= 227 * 1024, "scan kernel shared memory");
+    auto k2 = gdn_scan_tc_kernel<T, DK, DV, MS, STAGES>;
+    if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SL::kBytes) != cudaSuccess)
         return GDN_ERR_LAUNCH;
     {
-        ProfScope prof("gdn_scan_simt_kernel", st);
-        k2<<<dim3((unsigned)N, H, DV / 16), 256, smem2, st>>>(static_cast<const T*>(k), static_cast<const T*>(v),
-                                                              meta, chunk_off, chunk_tab, op, aux, state_in,
-                                                              static_cast<T*>(out), state_out, H);
+        ProfScope prof("gdn_scan_tc_kernel", st);
+        k2<<<dim3((unsigned)N, H, DV / MS), 256, SL::kBytes, st>>>(
+            static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), meta, chunk_off,
+            chunk_tab, op, state_in, static_cast<T*>(out), state_out, H, status);
     }
     return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
 }

@@ -1,0 +1,664 @@
+// gdn_prefill_tc.cuh -- chunkwise WY/UT prefill of the gated delta rule on tcgen05 tensor cores.
+//
+// Ferrite project page, Design section 03 "Chunked Gated DeltaNet": prompt rows go through the
+// recurrent state in chunks of 32 using the chunkwise WY/UT form of the delta rule on TF32 tensor
+// cores with a 3xTF32 split for fp32 accuracy; the final state is written back for decoding.
+//
+// Notation for one chunk of L <= 32 rows (rows L..31 are padding: q = k = v = 0, g = 0, beta = 0);
+// S is the dv x dk state entering the chunk, s = 1/sqrt(dk):
+//
+//   gamma_i = g_0 + ... + g_i (chunk-local),  Gamma_i = exp(gamma_i),  delta_i = exp(gamma_31 - gamma_i)
+//   A  = strictly-lower( diag(beta) (D o K K^T) ),  D_ij = exp(gamma_i - gamma_j)
+//   T  = (I + A)^-1 (unit lower triangular),  T'' = T diag(beta)
+//   P  = lower-including-diagonal( D o Q K^T )
+//
+// With X = K S^T and Z = Q S^T, the delta-rule writes of the chunk solve (I + A) U = diag(beta)
+// (V - diag(Gamma) X), so U = T'' Y with Y = V - diag(Gamma) X, and
+//
+//   O  = s ( diag(Gamma) Z + P U )                 (inter-chunk part + intra-chunk attention)
+//   S' = Gamma_31 S + (diag(delta) U)^T K          (inter-chunk state carry)
+//
+// Kernel 1 (gdn_prep_kernel, every (chunk, head) in parallel) builds the state-independent pieces:
+// the Gram matrices [K; Q] K^T on the tensor cores, then A, P, the forward substitution for T,
+// T'' and P T''.  It writes the 64 x 32 operator [T''; P T''] and the gate vectors per (chunk, head).
+//
+// Kernel 2 (gdn_scan_tc_kernel, one CTA per (sequence, head, slice of MS state rows)) walks the
+// chunks in order.  Rows of S evolve independently (right multiplication), so a head's dv rows are
+// split over dv/MS CTAs.  Per chunk, three dependent tensor-core products:
+//
+//   MMA_a  [X ; Z]     = [K ; Q] S^T            M=64, N=MS, K=dk
+//   MMA_b  [U ; P U]   = [T'' ; P T''] Y        M=64, N=MS, K=32
+//   MMA_c  (dS)^T      = K^T (diag(delta) U)    M=dk, N=MS, K=32
+//
+// with the elementwise steps between them done by the epilogue warps on tensor-memory rows.  Every
+// product uses the 3xTF32 split (hi*hi + hi*lo + lo*hi); the lo terms of an operand that is
+// exactly representable in TF32 (bf16 q/k) are zero and are skipped.  Producer warps stage the
+// next chunk's operands into a second buffer while the current chunk runs.
+#pragma once
+
+#include "gdn_common.cuh"
+#include "gdn_sm100.cuh"
+
+namespace gdn {
+
+constexpr int kOpStride = 64 * 32 + 128;   // floats per (chunk, head) in the operator workspace
+constexpr int kGateOff = 64 * 32;          // gates: Gamma[32], delta[32], Gamma_31, pad
+
+template <typename T>
+struct ExactTF32 { static constexpr bool value = false; };
+template <>
+struct ExactTF32<__nv_bfloat16> { static constexpr bool value = true; };
+
+// Loads 8 consecutive elements as fp32 (16-byte aligned for bf16, two 16-byte loads for fp32).
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&x)[8]);
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float (&x)[8])
+{
+    float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&x)[8])
+{
+    uint4 raw = __ldg(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(h[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+}
+
+__device__ __forceinline__ void st_shared_f4(uint32_t addr, float a, float b, float c, float d)
+{
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float a)
+{
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(a) : "memory");
+}
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr)
+{
+    float a;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(a) : "r"(addr) : "memory");
+    return a;
+}
+
+// Stores 8 consecutive K-elements (k0 % 8 == 0) of row r of a K-major SW128 tile of R rows, as hi
+// (and lo when SPLIT) parts.
+template <bool SPLIT>
+__device__ __forceinline__ void put8(uint32_t hi_base, uint32_t lo_base, int r, int k0, int R, const float (&x)[8])
+{
+    using namespace sm100;
+    const uint32_t o0 = sw128_off(r, k0, R), o1 = sw128_off(r, k0 + 4, R);
+    if constexpr (SPLIT) {
+        float h[8], l[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) tf32_split(x[i], h[i], l[i]);
+        st_shared_f4(hi_base + o0, h[0], h[1], h[2], h[3]);
+        st_shared_f4(hi_base + o1, h[4], h[5], h[6], h[7]);
+        st_shared_f4(lo_base + o0, l[0], l[1], l[2], l[3]);
+        st_shared_f4(lo_base + o1, l[4], l[5], l[6], l[7]);
+    } else {
+        st_shared_f4(hi_base + o0, x[0], x[1], x[2], x[3]);
+        st_shared_f4(hi_base + o1, x[4], x[5], x[6], x[7]);
+    }
+}
+
+// Abort path shared by the tensor-core kernels: record the timeout once, tell the other warps.
+__device__ __forceinline__ void tc_abort(int* status, volatile int* abort_flag)
+{
+    if (!*abort_flag) {
+        *abort_flag = 1;
+        report(status, GDN_ERR_TIMEOUT);
+    }
+}
+
+// Synchronisation rule of both kernels: exactly one thread performs each bounded mbarrier wait and
+// records a timeout in the shared abort flag; a CTA-wide (or role-wide) barrier follows, after
+// which every thread reads the abort flag.  So a timeout is seen by all threads at the same point,
+// no thread is ever left waiting at a hardware barrier, and all of them reach the final barrier
+// before the tensor memory is released.
+
+// =================================================================================================
+// Kernel 1: per (chunk, head) operator.  Persistent, 128 threads, work item = (global chunk, head).
+// =================================================================================================
+template <typename T, int DK>
+struct PrepSmem {
+    static constexpr bool EXACT = ExactTF32<T>::value;
+    static constexpr uint32_t kTile = 64 * DK * 4;                    // [K;Q] SW128, 64 rows
+    static constexpr uint32_t kTileHi = 0;
+    static constexpr uint32_t kTileLo = kTile;                        // fp32 inputs only
+    static constexpr uint32_t kF32 = kTile * (EXACT ? 1 : 2);         // start of plain fp32 scratch
+    static constexpr int LD = 33;
+    static constexpr uint32_t kG = kF32;                              // [32][33] K K^T -> A
+    static constexpr uint32_t kP = kG + 32 * LD * 4;                  // [32][33] Q K^T -> P
+    static constexpr uint32_t kT = kP + 32 * LD * 4;                  // [32][33] T''
+    static constexpr uint32_t kGam = kT + 32 * LD * 4;                // [32] gamma
+    static constexpr uint32_t kBet = kGam + 128;                      // [32] beta
+    static constexpr uint32_t kBar = kBet + 128;                      // mbarriers: MMA, drain
+    static constexpr uint32_t kTmem = kBar + 16;                      // tmem base (4 B)
+    static constexpr uint32_t kAbort = kTmem + 4;                     // abort flag (4 B)
+    static constexpr uint32_t kTotal = kAbort + 4;
+    static constexpr uint32_t kBytes = kTotal + 1024;                 // + alignment slack
+};
+
+template <typename T, int DK>
+__global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                       const float* __restrict__ g, const float* __restrict__ beta,
+                                                       const int* __restrict__ meta,
+                                                       const int4* __restrict__ chunk_tab, float* __restrict__ op,
+                                                       int H, int* status)
+{
+    using namespace sm100;
+    using L = PrepSmem<T, DK>;
+    constexpr bool EXACT = L::EXACT;
+    constexpr int C = kChunk;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    float* G = reinterpret_cast<float*>(sm + L::kG);
+    float* P = reinterpret_cast<float*>(sm + L::kP);
+    float* Tm = reinterpret_cast<float*>(sm + L::kT);
+    float* gam = reinterpret_cast<float*>(sm + L::kGam);
+    float* bet = reinterpret_cast<float*>(sm + L::kBet);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBar);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::kTmem);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kAbort);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init(bar + 1, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tslot, 32);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    const int nitems = meta[0] * H;
+    constexpr uint32_t idesc = idesc_tf32(64, 32);
+    uint32_t iter = 0;
+
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++iter) {
+        const int gc = item / H, h = item % H;
+        const int4 ct = chunk_tab[gc];
+        const int64_t t0 = ct.y;
+        const int Lr = ct.z;
+
+        // [K; Q] tile as fp32 (split for fp32 inputs), 64 rows x DK
+        for (int idx = tid; idx < 64 * (DK / 8); idx += 128) {
+            const int r = idx / (DK / 8), kg = idx % (DK / 8);
+            const int row = r & 31;
+            float x[8];
+            if (row < Lr) {
+                const T* src = (r < 32 ? k : q) + ((size_t)(t0 + row) * H + h) * DK + kg * 8;
+                load8<T>(src, x);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[i] = 0.f;
+            }
+            put8<!EXACT>(sbase + L::kTileHi, sbase + L::kTileLo, r, kg * 8, 64, x);
+        }
+        if (tid < 32) {
+            const bool ok = tid < Lr;
+            float gv = ok ? __ldg(g + (size_t)(t0 + tid) * H + h) : 0.f;
+            bet[tid] = ok ? __ldg(beta + (size_t)(t0 + tid) * H + h) : 0.f;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                float y = __shfl_up_sync(0xffffffffu, gv, o);
+                if (tid >= o) gv += y;
+            }
+            gam[tid] = gv;
+        }
+        fence_async_smem();
+        __syncthreads();
+
+        // Gram matrices on the tensor cores: D[r][n] = [K;Q]_r . K_n  (M=64, N=32, K=DK)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int ks = 0; ks < DK / 8; ++ks) {
+                const uint64_t a_hi = sw128_desc(sbase + L::kTileHi, ks, 64);
+                mma_tf32(tmem, a_hi, a_hi, idesc, ks > 0);
+                if constexpr (!EXACT) {
+                    const uint64_t a_lo = sw128_desc(sbase + L::kTileLo, ks, 64);
+                    mma_tf32(tmem, a_hi, a_lo, idesc, 1);
+                    mma_tf32(tmem, a_lo, a_hi, idesc, 1);
+                }
+            }
+            mma_commit(bar);
+            if (!mbar_wait(bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
+        }
+        __syncthreads();
+        if (*abort_flag) break;
+        tc_fence_after();
+        {
+            float d[32];
+            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), d);
+            tmem_ld_wait();
+            if (lane < 16) {
+                const int r = warp * 16 + lane;             // M=64 accumulator: row 16w+t in lane 32w+t
+                float* dst = (r < 32) ? (G + r * L::LD) : (P + (r - 32) * L::LD);
+#pragma unroll
+                for (int n = 0; n < 32; ++n) dst[n] = d[n];
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+
+        // gates: A (strictly lower) and P (lower incl. diagonal)
+        for (int idx = tid; idx < C * C; idx += 128) {
+            const int i = idx >> 5, j = idx & 31;
+            const float dd = (j <= i) ? expf(gam[i] - gam[j]) : 0.f;
+            G[i * L::LD + j] = (j < i) ? bet[i] * dd * G[i * L::LD + j] : 0.f;
+            P[i * L::LD + j] = dd * P[i * L::LD + j];
+        }
+        __syncthreads();
+        // T = (I + A)^-1, one lane per column j with the column in registers (entries above the
+        // diagonal are zero, so every lane runs the same unrolled recurrence); T'' = T diag(beta).
+        if (warp == 0) {
+            const int j = lane;
+            float t[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < i; ++m) acc = fmaf(G[i * L::LD + m], t[m], acc);
+                t[i] = (i == j) ? 1.f : ((i < j) ? 0.f : -acc);
+            }
+            const float bj = bet[j];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) Tm[i * L::LD + j] = t[i] * bj;
+        }
+        __syncthreads();
+        // operator rows [T''; P T''] and the gates
+        float* dst = op + ((size_t)gc * H + h) * kOpStride;
+        for (int idx = tid; idx < 64 * 32; idx += 128) {
+            const int i = idx >> 5, j = idx & 31;
+            float val;
+            if (i < 32) {
+                val = Tm[i * L::LD + j];
+            } else {
+                const int ii = i - 32;
+                float acc = 0.f;
+                for (int m = j; m <= ii; ++m) acc = fmaf(P[ii * L::LD + m], Tm[m * L::LD + j], acc);
+                val = acc;
+            }
+            dst[idx] = val;
+        }
+        if (tid < 32) {
+            const float gl = gam[31];
+            dst[kGateOff + tid] = expf(gam[tid]);
+            dst[kGateOff + 32 + tid] = expf(gl - gam[tid]);
+            if (tid == 0) dst[kGateOff + 64] = expf(gl);
+        }
+        __syncthreads();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *abort_flag) {
+        // after a timeout, give an MMA still in flight a bounded time to finish
+        mma_commit(bar + 1);
+        volatile int never = 0;
+        mbar_wait(bar + 1, 0, &never, 100000000ull);
+    }
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 32);
+}
+
+// =================================================================================================
+// Kernel 2: chunk-sequential scan on the tensor cores.
+// grid (N, H, DV / MS), 256 threads: warps 0-3 consumers (tensor-memory epilogues; thread 0 issues
+// the MMAs), warps 4-7 producers (operand staging for the next chunks, STAGES buffers).
+// =================================================================================================
+template <typename T, int DK, int MS, int STAGES>
+struct ScanSmem {
+    static constexpr bool EXACT = ExactTF32<T>::value;
+    static constexpr uint32_t kAKQ = 64 * DK * 4;                     // [K;Q], 64 x DK
+    static constexpr uint32_t kAKT = DK * 32 * 4;                     // K^T, DK x 32
+    static constexpr uint32_t kAB = 64 * 32 * 4;                      // [T'';PT''], 64 x 32
+    static constexpr uint32_t kB32 = ((MS * 32 * 4) + 1023) & ~1023u; // MS x 32 B-operand tile
+    // one stage
+    static constexpr uint32_t oAKQh = 0;
+    static constexpr uint32_t oAKQl = oAKQh + kAKQ;
+    static constexpr uint32_t oAKTh = oAKQl + (EXACT ? 0 : kAKQ);
+    static constexpr uint32_t oAKTl = oAKTh + kAKT;
+    static constexpr uint32_t oABh = oAKTl + (EXACT ? 0 : kAKT);
+    static constexpr uint32_t oABl = oABh + kAB;
+    static constexpr uint32_t oV = oABl + kAB;                        // fp32 [32][MS]
+    static constexpr uint32_t oGate = oV + 32 * MS * 4;               // fp32 [80]
+    static constexpr uint32_t kStage = ((oGate + 80 * 4) + 1023) & ~1023u;
+    // shared by all stages
+    static constexpr uint32_t oBSh = STAGES * kStage;                 // S as B operand: MS x DK
+    static constexpr uint32_t oBSl = oBSh + MS * DK * 4;
+    static constexpr uint32_t oBYh = oBSl + MS * DK * 4;              // Y as B: MS x 32
+    static constexpr uint32_t oBYl = oBYh + kB32;
+    static constexpr uint32_t oBUh = oBYl + kB32;                     // U~ as B: MS x 32
+    static constexpr uint32_t oBUl = oBUh + kB32;
+    static constexpr uint32_t oBar = oBUl + kB32;                     // full[S], empty[S], a, b, c
+    static constexpr uint32_t oTmem = oBar + 8 * (2 * STAGES + 4);   // + drain barrier
+    static constexpr uint32_t oAbort = oTmem + 4;
+    static constexpr uint32_t kTotal = oAbort + 4;
+    static constexpr uint32_t kBytes = kTotal + 1024;
+};
+
+template <typename T, int DK, int DV, int MS, int STAGES>
+__global__ void __launch_bounds__(256, 1) gdn_scan_tc_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                             const T* __restrict__ v,
+                                                             const int* __restrict__ meta,
+                                                             const int* __restrict__ chunk_off,
+                                                             const int4* __restrict__ chunk_tab,
+                                                             const float* __restrict__ op,
+                                                             const float* state_in, T* __restrict__ out,
+                                                             float* state_out, int H, int* status)
+{
+    using namespace sm100;
+    using L = ScanSmem<T, DK, MS, STAGES>;
+    constexpr bool EXACT = L::EXACT;
+    static_assert(MS == 16 || MS == 32, "MS");
+    static_assert(DK == 64 || DK == 128, "DK");
+    static_assert(DV % MS == 0, "DV");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::oBar);
+    uint64_t* empty = full + STAGES;
+    uint64_t* bar_a = empty + STAGES;
+    uint64_t* bar_b = bar_a + 1;
+    uint64_t* bar_c = bar_a + 2;
+    uint64_t* bar_drain = bar_a + 3;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::oTmem);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::oAbort);
+
+    if (meta[1]) return;   // bad cu_seqlens: nothing is written
+    const int n = blockIdx.x, h = blockIdx.y, r0 = blockIdx.z * MS;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c_begin = chunk_off[n], c_end = chunk_off[n + 1];
+    const int nch = c_end - c_begin;
+
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 128);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(bar_a, 1);
+        mbar_init(bar_b, 1);
+        mbar_init(bar_c, 1);
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tslot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    const uint32_t tD1 = tmem, tD2 = tmem + 32, tD3 = tmem + 64;   // accumulator columns
+
+    if (warp >= 4) {
+        // ------------------------------------------------------------------ producers
+        const int ptid = tid - 128;
+        for (int cl = 0; cl < nch; ++cl) {
+            const int s = cl % STAGES;
+            if (cl >= STAGES) {
+                if (ptid == 0 && !mbar_wait(&empty[s], (uint32_t)((cl / STAGES) - 1) & 1u, abort_flag))
+                    tc_abort(status, abort_flag);
+                named_bar(1, 128);
+                if (*abort_flag) break;
+            }
+            const uint32_t st = sbase + s * L::kStage;
+            float* stf = reinterpret_cast<float*>(sm + s * L::kStage);
+            const int gc = c_begin + cl;
+            const int4 ct = chunk_tab[gc];
+            const int64_t t0 = ct.y;
+            const int Lr = ct.z;
+            // K and Q in blocks of 4 tokens x 8 features; K goes to [K;Q] rows and to K^T
+            for (int idx = ptid; idx < 2 * 8 * (DK / 8); idx += 128) {
+                const int isq = idx >= 8 * (DK / 8);
+                const int b = isq ? idx - 8 * (DK / 8) : idx;
+                const int jg = b & 7, kg = b >> 3;
+                float x[4][8];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = 4 * jg + u;
+                    if (j < Lr) {
+                        load8<T>((isq ? q : k) + ((size_t)(t0 + j) * H + h) * DK + kg * 8, x[u]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) x[u][e] = 0.f;
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) put8<!EXACT>(st + L::oAKQh, st + L::oAKQl, (isq ? 32 : 0) + 4 * jg + u, kg * 8, 64, x[u]);
+                if (!isq) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const uint32_t o = sw128_off(kg * 8 + e, 4 * jg, DK);
+                        if constexpr (EXACT) {
+                            st_shared_f4(st + L::oAKTh + o, x[0][e], x[1][e], x[2][e], x[3][e]);
+                        } else {
+                            float hi[4], lo[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) tf32_split(x[u][e], hi[u], lo[u]);
+                            st_shared_f4(st + L::oAKTh + o, hi[0], hi[1], hi[2], hi[3]);
+                            st_shared_f4(st + L::oAKTl + o, lo[0], lo[1], lo[2], lo[3]);
+                        }
+                    }
+                }
+            }
+            // [T''; P T''] operator, split
+            const float* opc = op + ((size_t)gc * H + h) * kOpStride;
+            for (int idx = ptid; idx < 64 * 4; idx += 128) {
+                const int r = idx >> 2, kg = idx & 3;
+                float x[8];
+                const float4 a = __ldg(reinterpret_cast<const float4*>(opc + r * 32 + kg * 8));
+                const float4 b = __ldg(reinterpret_cast<const float4*>(opc + r * 32 + kg * 8 + 4));
+                x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+                put8<true>(st + L::oABh, st + L::oABl, r, kg * 8, 64, x);
+            }
+            // V slice [32][MS] fp32 and the gates
+            float* Vs = stf + L::oV / 4;
+            for (int idx = ptid; idx < 32 * MS; idx += 128) {
+                const int j = idx / MS, c = idx % MS;
+                Vs[idx] = (j < Lr) ? Elem<T>::ld(v + ((size_t)(t0 + j) * H + h) * DV + r0 + c) : 0.f;
+            }
+            float* gate = stf + L::oGate / 4;
+            if (ptid < 80) gate[ptid] = (ptid < 65) ? __ldg(opc + kGateOff + ptid) : 0.f;
+            fence_async_smem();
+            mbar_arrive(&full[s]);
+        }
+    } else {
+        // ------------------------------------------------------------------ consumers
+        // thread (warp, lane) owns column c of the state slice: S[0..MS)[c]
+        const int c_own = (DK == 128) ? (warp * 32 + lane) : (warp * 16 + lane);
+        const bool owns = (DK == 128) || (lane < 16);
+        float S[MS];
+#pragma unroll
+        for (int i = 0; i < MS; ++i)
+            S[i] = (state_in && owns) ? state_in[(((size_t)n * H + h) * DV + r0 + i) * DK + c_own] : 0.f;
+
+        const float scale = rsqrtf((float)DK);
+        constexpr uint32_t idA = idesc_tf32(64, MS);
+        constexpr uint32_t idB = idesc_tf32(64, MS);
+        constexpr uint32_t idC = idesc_tf32(DK, MS);
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int row16 = warp * 16 + lane;          // accumulator row of an M=64 product in this lane
+        const int tok = (warp < 2) ? row16 : (row16 - 32);
+        bool aborted = false;
+
+        for (int cl = 0; cl <= nch; ++cl) {
+            // S (initial, or after the previous chunk's carry) -> B operand of MMA_a
+            if (owns) {
+#pragma unroll
+                for (int i = 0; i < MS; ++i) {
+                    float hi, lo;
+                    tf32_split(S[i], hi, lo);
+                    const uint32_t o = sw128_off(i, c_own, MS);
+                    st_shared_f32(sbase + L::oBSh + o, hi);
+                    st_shared_f32(sbase + L::oBSl + o, lo);
+                }
+            }
+            if (cl == nch) break;
+            fence_async_smem();
+            tc_fence_before();
+            named_bar(2, 128);      // every column of S written before MMA_a reads it
+            const int s = cl % STAGES;
+            const uint32_t st = sbase + s * L::kStage;
+            const float* stf = reinterpret_cast<const float*>(sm + s * L::kStage);
+
+            // ---- MMA_a: [X; Z] = [K; Q] S^T
+            if (tid == 0) {
+                if (!mbar_wait(&full[s], (uint32_t)(cl / STAGES) & 1u, abort_flag)) {
+                    tc_abort(status, abort_flag);
+                } else {
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int ks = 0; ks < DK / 8; ++ks) {
+                        const uint64_t a = sw128_desc(st + L::oAKQh, ks, 64);
+                        mma_tf32(tD1, a, sw128_desc(sbase + L::oBSh, ks, MS), idA, ks > 0);
+                        mma_tf32(tD1, a, sw128_desc(sbase + L::oBSl, ks, MS), idA, 1);
+                        if constexpr (!EXACT)
+                            mma_tf32(tD1, sw128_desc(st + L::oAKQl, ks, 64), sw128_desc(sbase + L::oBSh, ks, MS),
+                                     idA, 1);
+                    }
+                    mma_commit(bar_a);
+                    if (!mbar_wait(bar_a, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
+                }
+            }
+            named_bar(2, 128);
+            if (*abort_flag) { aborted = true; break; }
+            tc_fence_after();
+            const int4 ct = chunk_tab[c_begin + cl];
+            const int64_t t0 = ct.y;
+            const int Lr = ct.z;
+            const float* gate = stf + L::oGate / 4;
+            const float* Vs = stf + L::oV / 4;
+            const float Gam = (lane < 16) ? gate[tok] : 0.f;
+            const float del = (lane < 16 && warp < 2) ? gate[32 + tok] : 0.f;
+            const float GamC = gate[64];
+            float za[MS];
+            if (warp < 2) {
+                // Y = V - diag(Gamma) X  ->  B operand of MMA_b (row i of S, K index = token)
+                float x[MS];
+                tmem_ld<MS>(tD1 + lane_base, x);
+                tmem_ld_wait();
+                if (lane < 16) {
+#pragma unroll
+                    for (int i = 0; i < MS; ++i) {
+                        float hi, lo;
+                        tf32_split(Vs[tok * MS + i] - Gam * x[i], hi, lo);
+                        const uint32_t o = sw128_off(i, tok, MS);
+                        st_shared_f32(sbase + L::oBYh + o, hi);
+                        st_shared_f32(sbase + L::oBYl + o, lo);
+                    }
+                }
+                fence_async_smem();
+            } else {
+                tmem_ld<MS>(tD1 + lane_base, za);    // Z rows, token i = row16 - 32
+                tmem_ld_wait();
+            }
+            tc_fence_before();
+            named_bar(2, 128);
+            // ---- MMA_b: [U; PU] = [T''; PT''] Y
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t ah = sw128_desc(st + L::oABh, ks, 64);
+                    const uint64_t bh = sw128_desc(sbase + L::oBYh, ks, MS);
+                    mma_tf32(tD2, ah, bh, idB, ks > 0);
+                    mma_tf32(tD2, ah, sw128_desc(sbase + L::oBYl, ks, MS), idB, 1);
+                    mma_tf32(tD2, sw128_desc(st + L::oABl, ks, 64), bh, idB, 1);
+                }
+                mma_commit(bar_b);
+                if (!mbar_wait(bar_b, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
+            }
+            named_bar(2, 128);
+            if (*abort_flag) { aborted = true; break; }
+            tc_fence_after();
+            {
+                float u[MS];
+                tmem_ld<MS>(tD2 + lane_base, u);
+                tmem_ld_wait();
+                if (warp < 2) {
+                    // U~ = diag(delta) U  ->  B operand of MMA_c
+                    if (lane < 16) {
+#pragma unroll
+                        for (int i = 0; i < MS; ++i) {
+                            float hi, lo;
+                            tf32_split(del * u[i], hi, lo);
+                            const uint32_t o = sw128_off(i, tok, MS);
+                            st_shared_f32(sbase + L::oBUh + o, hi);
+                            st_shared_f32(sbase + L::oBUl + o, lo);
+                        }
+                    }
+                    fence_async_smem();
+                } else if (lane < 16 && tok < Lr) {
+                    // O = s (diag(Gamma) Z + P U)
+                    T* dst = out + ((size_t)(t0 + tok) * H + h) * DV + r0;
+#pragma unroll
+                    for (int i = 0; i < MS; ++i) Elem<T>::st(dst + i, scale * fmaf(Gam, za[i], u[i]));
+                }
+            }
+            tc_fence_before();
+            named_bar(2, 128);
+            // ---- MMA_c: dS^T = K^T U~   (its completion also frees the stage buffer)
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t ah = sw128_desc(st + L::oAKTh, ks, DK);
+                    const uint64_t bh = sw128_desc(sbase + L::oBUh, ks, MS);
+                    mma_tf32(tD3, ah, bh, idC, ks > 0);
+                    mma_tf32(tD3, ah, sw128_desc(sbase + L::oBUl, ks, MS), idC, 1);
+                    if constexpr (!EXACT) mma_tf32(tD3, sw128_desc(st + L::oAKTl, ks, DK), bh, idC, 1);
+                }
+                mma_commit(bar_c);
+                mma_commit(&empty[s]);
+                if (!mbar_wait(bar_c, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
+            }
+            named_bar(2, 128);
+            if (*abort_flag) { aborted = true; break; }
+            tc_fence_after();
+            {
+                // S' = Gamma_31 S + dS   (row c_own of dS^T; for dk = 64 the M=64 layout puts row
+                // 16w+t in lane 32w+t, which is c_own of that lane)
+                float ds[MS];
+                tmem_ld<MS>(tD3 + lane_base, ds);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < MS; ++i) S[i] = fmaf(GamC, S[i], ds[i]);
+            }
+            tc_fence_before();
+        }
+        if (state_out && owns && !aborted) {
+#pragma unroll
+            for (int i = 0; i < MS; ++i) state_out[(((size_t)n * H + h) * DV + r0 + i) * DK + c_own] = S[i];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *abort_flag) {
+        // after a timeout, give MMAs still in flight a bounded time to finish before the tensor
+        // memory they write is released
+        mma_commit(bar_drain);
+        volatile int never = 0;
+        mbar_wait(bar_drain, 0, &never, 100000000ull);
+    }
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+}  // namespace gdn
