@@ -104,6 +104,13 @@ static int dispatch_decode(const void* q, const void* k, const void* v, const fl
     return launch_decode<T, 64, 64>(q, k, v, g, beta, state, out, B, H, st);
 }
 
+#ifndef GDN_SCAN_MS
+#define GDN_SCAN_MS 32
+#endif
+#ifndef GDN_SCAN_MINB
+#define GDN_SCAN_MINB 1
+#endif
+
 static int g_num_sms = 0;
 
 template <typename T, int DK, int DV>
@@ -143,12 +150,15 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
                                           chunk_tab, op, H, status);
         if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
     }
-    constexpr int MS = 32;
+    // state rows per CTA and CTAs per SM of the scan (compile-time tuning knobs)
+    constexpr int MS = GDN_SCAN_MS;
+    using S1 = ScanSmem<T, DK, MS, 1>;
     using S2 = ScanSmem<T, DK, MS, 2>;
-    constexpr int STAGES = (S2::kBytes <= 227 * 1024) ? 2 : 1;
+    constexpr int MINB = ((S1::kBytes + 1024) * GDN_SCAN_MINB <= 228 * 1024) ? GDN_SCAN_MINB : 1;
+    constexpr int STAGES = ((S2::kBytes + 1024) * MINB <= 228 * 1024) ? 2 : 1;
     using SL = ScanSmem<T, DK, MS, STAGES>;
-    static_assert(SL::kBytes <= 227 * 1024, "scan kernel shared memory");
-    auto k2 = gdn_scan_tc_kernel<T, DK, DV, MS, STAGES>;
+    static_assert((SL::kBytes + 1024) * MINB <= 228 * 1024, "scan kernel shared memory");
+    auto k2 = gdn_scan_tc_kernel<T, DK, DV, MS, STAGES, MINB>;
     if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SL::kBytes) != cudaSuccess)
         return GDN_ERR_LAUNCH;
     {

@@ -351,8 +351,8 @@ struct ScanSmem {
     static constexpr uint32_t kBytes = kTotal + 1024;
 };
 
-template <typename T, int DK, int DV, int MS, int STAGES>
-__global__ void __launch_bounds__(256, 1) gdn_scan_tc_kernel(const T* __restrict__ q, const T* __restrict__ k,
+template <typename T, int DK, int DV, int MS, int STAGES, int MINB>
+__global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                              const T* __restrict__ v,
                                                              const int* __restrict__ meta,
                                                              const int* __restrict__ chunk_off,
