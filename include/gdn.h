@@ -102,6 +102,30 @@ int gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* 
                       void* stream);
 
 /*
+ * gdn_chunk_prefill without a caller-provided workspace.  The pages have no counterpart to this
+ * call; it exists for callers that cannot allocate device memory when they run a prefill -- for
+ * example an engine that plans every byte of GPU memory at start-up and forbids cudaMalloc later,
+ * or code on a latency-critical path where cudaMalloc/cudaFree could block or synchronise the
+ * device.  The call allocates nothing: its scratch is a fixed 64 MiB array inside this library,
+ * one per GPU that loads the library, held until the process exits.
+ *
+ *   Arguments, layouts and results are those of gdn_chunk_prefill minus workspace/workspace_bytes.
+ *   Limit: the problem must satisfy gdn_chunk_prefill_workspace_bytes(total_tokens, num_seqs, H,
+ *   dk, dv) <= 64 MiB (for H = 32, d = 128: about 7,600 tokens in one sequence); larger problems
+ *   return GDN_ERR_WORKSPACE and enqueue nothing.
+ *   Set-up: the first call on a device looks up that device's copy of the scratch array (a CUDA
+ *   runtime query, no allocation).  Make that first call before any stream capture on the device.
+ *   Sharing: every call on a device uses the same scratch array and leaves its contents behind
+ *   (nothing in it needs to start at zero).  Calls whose execution overlaps on the GPU -- on
+ *   different streams, or from different threads -- race on the scratch and give wrong results;
+ *   order them (one stream, or events).
+ */
+int gdn_chunk_prefill_noalloc(const void* q, const void* k, const void* v, const float* g,
+                              const float* beta, const int32_t* cu_seqlens, int num_seqs,
+                              int64_t total_tokens, const float* state_in, void* out,
+                              float* state_out, int H, int dk, int dv, int dtype, void* stream);
+
+/*
  * Recurrent decode step (the consumer of the written-back state, Design section 03): one token for
  * each of B sequences, state updated in place.
  *

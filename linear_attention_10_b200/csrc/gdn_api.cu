@@ -188,6 +188,29 @@ static int dispatch_prefill(int dk, int dv, const PrefillLayout& lay, char* ws, 
     return GDN_ERR_UNSUPPORTED;
 }
 
+// ---- scratch for the allocation-free prefill entry point -----------------------------------------
+// A fixed 64 MiB block of device memory per GPU, part of this library's module: it exists on every
+// device that loads the library, from module load until the process exits.  Host code must not use
+// the symbol itself as an address; noalloc_scratch_ptr() asks the runtime for the device address.
+constexpr size_t kNoallocScratchBytes = size_t(64) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device, looked up once per device.
+static void* noalloc_scratch_ptr()
+{
+    static std::mutex mu;
+    static void* cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        cache[dev] = p;
+    }
+    return cache[dev];
+}
+
 }  // namespace gdn
 
 using namespace gdn;
@@ -248,6 +271,21 @@ int gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* 
                                        fixed_len, state_in, out, state_out, H, st);
     return dispatch_prefill<__nv_bfloat16>(dk, dv, lay, ws, q, k, v, g, beta, cu_seqlens, num_seqs,
                                            total_tokens, fixed_len, state_in, out, state_out, H, st);
+}
+
+int gdn_chunk_prefill_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                              const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens,
+                              const float* state_in, void* out, float* state_out, int H, int dk, int dv,
+                              int dtype, void* stream)
+{
+    // the scratch must hold the whole workspace of this call; refuse before touching the device
+    const size_t need = gdn_chunk_prefill_workspace_bytes(total_tokens, num_seqs, H, dk, dv);
+    if (need > kNoallocScratchBytes) return GDN_ERR_WORKSPACE;
+    void* scratch = noalloc_scratch_ptr();
+    if (!scratch) return GDN_ERR_CUDA;
+    // nothing in the scratch has to start at zero: the kernels write every part they read
+    return gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, state_in, out, state_out, H,
+                             dk, dv, dtype, scratch, kNoallocScratchBytes, stream);
 }
 
 int gdn_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,

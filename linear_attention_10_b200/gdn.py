@@ -25,6 +25,7 @@ EXPORTS = (
     "gdn_version",
     "gdn_chunk_prefill_workspace_bytes",
     "gdn_chunk_prefill",
+    "gdn_chunk_prefill_noalloc",
     "gdn_decode_step",
     "gdn_get_device_status",
     "gdn_profile_start",
@@ -59,6 +60,8 @@ def lib() -> ctypes.CDLL:
     L.gdn_chunk_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, i32, i32,
                                     vp, sz, vp]
     L.gdn_chunk_prefill.restype = i32
+    L.gdn_chunk_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, i32, i32, vp]
+    L.gdn_chunk_prefill_noalloc.restype = i32
     L.gdn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
     L.gdn_decode_step.restype = i32
     L.gdn_get_device_status.argtypes = [vp]
