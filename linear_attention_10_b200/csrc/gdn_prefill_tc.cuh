@@ -108,6 +108,64 @@ __device__ __forceinline__ void put8(uint32_t hi_base, uint32_t lo_base, int r, 
     }
 }
 
+// Eight consecutive elements as loaded from global memory, not yet converted.  Producers keep the
+// next chunk's data in this form while they convert and store the current chunk, so the global
+// load latency of chunk c+1 overlaps the shared-memory work of chunk c.
+template <typename T>
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+    uint4 u;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
+    __device__ __forceinline__ void zero() { u = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void get(float (&x)[8]) const
+    {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(h[i]);
+            x[2 * i] = f.x;
+            x[2 * i + 1] = f.y;
+        }
+    }
+};
+template <>
+struct Raw8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p)
+    {
+        a = __ldg(reinterpret_cast<const float4*>(p));
+        b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    }
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ void get(float (&x)[8]) const
+    {
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+};
+
+// Stores N consecutive outputs with 16-byte stores (dst 16-byte aligned, N % 8 == 0).
+template <typename T, int N>
+__device__ __forceinline__ void store_row(T* dst, const float (&x)[N]);
+template <int N>
+__device__ __forceinline__ void store_row(__nv_bfloat16* dst, const float (&x)[N])
+{
+#pragma unroll
+    for (int i = 0; i < N; i += 8) {
+        uint4 u;
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(x[i + 2 * e], x[i + 2 * e + 1]);
+        *reinterpret_cast<uint4*>(dst + i) = u;
+    }
+}
+template <int N>
+__device__ __forceinline__ void store_row(float* dst, const float (&x)[N])
+{
+#pragma unroll
+    for (int i = 0; i < N; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+}
+
 // Abort path shared by the tensor-core kernels: record the timeout once, tell the other warps.
 __device__ __forceinline__ void tc_abort(int* status, volatile int* abort_flag)
 {
@@ -116,6 +174,11 @@ __device__ __forceinline__ void tc_abort(int* status, volatile int* abort_flag)
         report(status, GDN_ERR_TIMEOUT);
     }
 }
+
+// Optional phase-timing hook of the scan kernel (compiled out unless a build defines it).
+#ifndef GDN_SCAN_TRACE
+#define GDN_SCAN_TRACE(chunk, slot)
+#endif
 
 // Synchronisation rule of both kernels: exactly one thread performs each bounded mbarrier wait and
 // records a timeout in the shared abort flag; a CTA-wide (or role-wide) barrier follows, after
@@ -188,30 +251,51 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, 
     constexpr uint32_t idesc = idesc_tf32(64, 32);
     uint32_t iter = 0;
 
-    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++iter) {
-        const int gc = item / H, h = item % H;
-        const int4 ct = chunk_tab[gc];
+    // The next item's global loads are issued before the current item is processed, so their
+    // latency overlaps the tensor-core product and the triangular solve.
+    constexpr int NG = 64 * (DK / 8) / 128;          // 8-element groups of [K; Q] per thread
+    struct Pre {
+        Raw8<T> x[NG];
+        float gv, bv;
+        int gc, h, Lr;
+    };
+    auto load_item = [&](Pre& p, int item) {
+        p.gc = item / H;
+        p.h = item % H;
+        const int4 ct = chunk_tab[p.gc];
         const int64_t t0 = ct.y;
-        const int Lr = ct.z;
-
-        // [K; Q] tile as fp32 (split for fp32 inputs), 64 rows x DK
-        for (int idx = tid; idx < 64 * (DK / 8); idx += 128) {
+        p.Lr = ct.z;
+#pragma unroll
+        for (int u = 0; u < NG; ++u) {
+            const int idx = tid + 128 * u;
             const int r = idx / (DK / 8), kg = idx % (DK / 8);
             const int row = r & 31;
-            float x[8];
-            if (row < Lr) {
-                const T* src = (r < 32 ? k : q) + ((size_t)(t0 + row) * H + h) * DK + kg * 8;
-                load8<T>(src, x);
-            } else {
+            if (row < p.Lr) p.x[u].load((r < 32 ? k : q) + ((size_t)(t0 + row) * H + p.h) * DK + kg * 8);
+            else p.x[u].zero();
+        }
+        const bool ok = tid < p.Lr;
+        p.gv = ok ? __ldg(g + (size_t)(t0 + tid) * H + p.h) : 0.f;
+        p.bv = ok ? __ldg(beta + (size_t)(t0 + tid) * H + p.h) : 0.f;
+    };
+    Pre cur, nxt;
+    if ((int)blockIdx.x < nitems) load_item(cur, blockIdx.x);
+
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++iter) {
+        if (item + (int)gridDim.x < nitems) load_item(nxt, item + gridDim.x);
+        const int gc = cur.gc, h = cur.h;
+
+        // [K; Q] tile as fp32 (split for fp32 inputs), 64 rows x DK
 #pragma unroll
-                for (int i = 0; i < 8; ++i) x[i] = 0.f;
-            }
+        for (int u = 0; u < NG; ++u) {
+            const int idx = tid + 128 * u;
+            const int r = idx / (DK / 8), kg = idx % (DK / 8);
+            float x[8];
+            cur.x[u].get(x);
             put8<!EXACT>(sbase + L::kTileHi, sbase + L::kTileLo, r, kg * 8, 64, x);
         }
         if (tid < 32) {
-            const bool ok = tid < Lr;
-            float gv = ok ? __ldg(g + (size_t)(t0 + tid) * H + h) : 0.f;
-            bet[tid] = ok ? __ldg(beta + (size_t)(t0 + tid) * H + h) : 0.f;
+            float gv = cur.gv;
+            bet[tid] = cur.bv;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 float y = __shfl_up_sync(0xffffffffu, gv, o);
@@ -225,14 +309,14 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, 
         // Gram matrices on the tensor cores: D[r][n] = [K;Q]_r . K_n  (M=64, N=32, K=DK)
         if (tid == 0) {
             tc_fence_after();
-#pragma unroll 1
+            const uint64_t dh = sw128_desc(sbase + L::kTileHi, 0, 64), dl = sw128_desc(sbase + L::kTileLo, 0, 64);
+#pragma unroll
             for (int ks = 0; ks < DK / 8; ++ks) {
-                const uint64_t a_hi = sw128_desc(sbase + L::kTileHi, ks, 64);
-                mma_tf32(tmem, a_hi, a_hi, idesc, ks > 0);
+                const uint64_t o = sw128_ks_off(ks, 64);
+                mma_tf32(tmem, dh + o, dh + o, idesc, ks > 0);
                 if constexpr (!EXACT) {
-                    const uint64_t a_lo = sw128_desc(sbase + L::kTileLo, ks, 64);
-                    mma_tf32(tmem, a_hi, a_lo, idesc, 1);
-                    mma_tf32(tmem, a_lo, a_hi, idesc, 1);
+                    mma_tf32(tmem, dh + o, dl + o, idesc, 1);
+                    mma_tf32(tmem, dl + o, dh + o, idesc, 1);
                 }
             }
             mma_commit(bar);
@@ -302,6 +386,7 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, 
             if (tid == 0) dst[kGateOff + 64] = expf(gl);
         }
         __syncthreads();
+        cur = nxt;
     }
     tc_fence_before();
     __syncthreads();
@@ -334,8 +419,8 @@ struct ScanSmem {
     static constexpr uint32_t oAKTl = oAKTh + kAKT;
     static constexpr uint32_t oABh = oAKTl + (EXACT ? 0 : kAKT);
     static constexpr uint32_t oABl = oABh + kAB;
-    static constexpr uint32_t oV = oABl + kAB;                        // fp32 [32][MS]
-    static constexpr uint32_t oGate = oV + 32 * MS * 4;               // fp32 [80]
+    static constexpr uint32_t oV = oABl + kAB;                        // fp32 [MS][33] (V^T, padded)
+    static constexpr uint32_t oGate = oV + 33 * MS * 4;               // fp32 [80]
     static constexpr uint32_t kStage = ((oGate + 80 * 4) + 1023) & ~1023u;
     // shared by all stages
     static constexpr uint32_t oBSh = STAGES * kStage;                 // S as B operand: MS x DK
@@ -384,6 +469,13 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c_begin = chunk_off[n], c_end = chunk_off[n + 1];
     const int nch = c_end - c_begin;
+    // chunks of a sequence are consecutive 32-row blocks from its first token
+    int64_t seq_t0 = 0, seq_end = 0;
+    if (nch > 0) {
+        const int4 first = chunk_tab[c_begin], last = chunk_tab[c_end - 1];
+        seq_t0 = first.y;
+        seq_end = (int64_t)last.y + last.z;
+    }
 
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -409,40 +501,64 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
 
     if (warp >= 4) {
         // ------------------------------------------------------------------ producers
+        // Per chunk and thread: DK/64 blocks of 4 tokens x 8 features of K or Q, two 8-float
+        // groups of the [T''; P T''] operator, one 8-element group of the V slice, one gate value.
         const int ptid = tid - 128;
-        for (int cl = 0; cl < nch; ++cl) {
-            const int s = cl % STAGES;
-            if (cl >= STAGES) {
-                if (ptid == 0 && !mbar_wait(&empty[s], (uint32_t)((cl / STAGES) - 1) & 1u, abort_flag))
-                    tc_abort(status, abort_flag);
-                named_bar(1, 128);
-                if (*abort_flag) break;
+        constexpr int NB = DK / 64;
+        constexpr int NVG = 4 * MS;                    // 8-element groups in the V slice
+        struct Pre {
+            Raw8<T> kq[NB][4];
+            Raw8<float> ab[2];
+            Raw8<T> vv;
+            float gt;
+        };
+        auto load_chunk = [&](Pre& p, int cl) {
+            const int gc = c_begin + cl;
+            const int64_t t0 = seq_t0 + (int64_t)cl * kChunk;
+            const int Lr = (int)((seq_end - t0) < kChunk ? (seq_end - t0) : kChunk);
+#pragma unroll
+            for (int u = 0; u < NB; ++u) {
+                const int b = ptid + 128 * u;
+                const bool isq = b >= DK;
+                const int bb = isq ? b - DK : b;
+                const int jg = bb & 7, kg = bb >> 3;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int j = 4 * jg + r;
+                    if (j < Lr) p.kq[u][r].load((isq ? q : k) + ((size_t)(t0 + j) * H + h) * DK + kg * 8);
+                    else p.kq[u][r].zero();
+                }
             }
+            const float* opc = op + ((size_t)gc * H + h) * kOpStride;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int idx = ptid + 128 * u;
+                p.ab[u].load(opc + (idx >> 2) * 32 + (idx & 3) * 8);
+            }
+            if (ptid < NVG) {
+                const int j = ptid / (MS / 8), cg = ptid % (MS / 8);
+                if (j < Lr) p.vv.load(v + ((size_t)(t0 + j) * H + h) * DV + r0 + cg * 8);
+                else p.vv.zero();
+            }
+            p.gt = (ptid < 65) ? __ldg(opc + kGateOff + ptid) : 0.f;
+        };
+        auto store_chunk = [&](const Pre& p, int s) {
             const uint32_t st = sbase + s * L::kStage;
             float* stf = reinterpret_cast<float*>(sm + s * L::kStage);
-            const int gc = c_begin + cl;
-            const int4 ct = chunk_tab[gc];
-            const int64_t t0 = ct.y;
-            const int Lr = ct.z;
-            // K and Q in blocks of 4 tokens x 8 features; K goes to [K;Q] rows and to K^T
-            for (int idx = ptid; idx < 2 * 8 * (DK / 8); idx += 128) {
-                const int isq = idx >= 8 * (DK / 8);
-                const int b = isq ? idx - 8 * (DK / 8) : idx;
-                const int jg = b & 7, kg = b >> 3;
+#pragma unroll
+            for (int u = 0; u < NB; ++u) {
+                const int b = ptid + 128 * u;
+                const bool isq = b >= DK;
+                const int bb = isq ? b - DK : b;
+                const int jg = bb & 7, kg = bb >> 3;
                 float x[4][8];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int j = 4 * jg + u;
-                    if (j < Lr) {
-                        load8<T>((isq ? q : k) + ((size_t)(t0 + j) * H + h) * DK + kg * 8, x[u]);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) x[u][e] = 0.f;
-                    }
+                for (int r = 0; r < 4; ++r) {
+                    p.kq[u][r].get(x[r]);
+                    put8<!EXACT>(st + L::oAKQh, st + L::oAKQl, (isq ? 32 : 0) + 4 * jg + r, kg * 8, 64, x[r]);
                 }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) put8<!EXACT>(st + L::oAKQh, st + L::oAKQl, (isq ? 32 : 0) + 4 * jg + u, kg * 8, 64, x[u]);
                 if (!isq) {
+                    // K^T: feature rows, 4 consecutive tokens per 16-byte store
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const uint32_t o = sw128_off(kg * 8 + e, 4 * jg, DK);
@@ -451,33 +567,49 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                         } else {
                             float hi[4], lo[4];
 #pragma unroll
-                            for (int u = 0; u < 4; ++u) tf32_split(x[u][e], hi[u], lo[u]);
+                            for (int r = 0; r < 4; ++r) tf32_split(x[r][e], hi[r], lo[r]);
                             st_shared_f4(st + L::oAKTh + o, hi[0], hi[1], hi[2], hi[3]);
                             st_shared_f4(st + L::oAKTl + o, lo[0], lo[1], lo[2], lo[3]);
                         }
                     }
                 }
             }
-            // [T''; P T''] operator, split
-            const float* opc = op + ((size_t)gc * H + h) * kOpStride;
-            for (int idx = ptid; idx < 64 * 4; idx += 128) {
-                const int r = idx >> 2, kg = idx & 3;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int idx = ptid + 128 * u;
                 float x[8];
-                const float4 a = __ldg(reinterpret_cast<const float4*>(opc + r * 32 + kg * 8));
-                const float4 b = __ldg(reinterpret_cast<const float4*>(opc + r * 32 + kg * 8 + 4));
-                x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-                put8<true>(st + L::oABh, st + L::oABl, r, kg * 8, 64, x);
+                p.ab[u].get(x);
+                put8<true>(st + L::oABh, st + L::oABl, idx >> 2, (idx & 3) * 8, 64, x);
             }
-            // V slice [32][MS] fp32 and the gates
-            float* Vs = stf + L::oV / 4;
-            for (int idx = ptid; idx < 32 * MS; idx += 128) {
-                const int j = idx / MS, c = idx % MS;
-                Vs[idx] = (j < Lr) ? Elem<T>::ld(v + ((size_t)(t0 + j) * H + h) * DV + r0 + c) : 0.f;
+            if (ptid < NVG) {
+                const int j = ptid / (MS / 8), cg = ptid % (MS / 8);
+                float x[8];
+                p.vv.get(x);
+                float* Vt = stf + L::oV / 4;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) Vt[(cg * 8 + e) * 33 + j] = x[e];
             }
-            float* gate = stf + L::oGate / 4;
-            if (ptid < 80) gate[ptid] = (ptid < 65) ? __ldg(opc + kGateOff + ptid) : 0.f;
+            if (ptid < 80) stf[L::oGate / 4 + ptid] = p.gt;
+        };
+
+        Pre cur, nxt;
+        if (nch > 0) load_chunk(cur, 0);
+        for (int cl = 0; cl < nch; ++cl) {
+            const int s = cl % STAGES;
+            if (cl + 1 < nch) load_chunk(nxt, cl + 1);     // in flight while chunk cl is stored
+            GDN_SCAN_TRACE(cl, 10);
+            if (cl >= STAGES) {
+                if (ptid == 0 && !mbar_wait(&empty[s], (uint32_t)((cl / STAGES) - 1) & 1u, abort_flag))
+                    tc_abort(status, abort_flag);
+                named_bar(1, 128);
+                if (*abort_flag) break;
+            }
+            GDN_SCAN_TRACE(cl, 11);
+            store_chunk(cur, s);
             fence_async_smem();
             mbar_arrive(&full[s]);
+            GDN_SCAN_TRACE(cl, 12);
+            cur = nxt;
         }
     } else {
         // ------------------------------------------------------------------ consumers
@@ -499,6 +631,7 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
         bool aborted = false;
 
         for (int cl = 0; cl <= nch; ++cl) {
+            GDN_SCAN_TRACE(cl, 0);
             // S (initial, or after the previous chunk's carry) -> B operand of MMA_a
             if (owns) {
 #pragma unroll
@@ -514,6 +647,7 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
             fence_async_smem();
             tc_fence_before();
             named_bar(2, 128);      // every column of S written before MMA_a reads it
+            GDN_SCAN_TRACE(cl, 1);
             const int s = cl % STAGES;
             const uint32_t st = sbase + s * L::kStage;
             const float* stf = reinterpret_cast<const float*>(sm + s * L::kStage);
@@ -523,26 +657,28 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                 if (!mbar_wait(&full[s], (uint32_t)(cl / STAGES) & 1u, abort_flag)) {
                     tc_abort(status, abort_flag);
                 } else {
+                    GDN_SCAN_TRACE(cl, 2);
                     tc_fence_after();
-#pragma unroll 1
+                    const uint64_t ah = sw128_desc(st + L::oAKQh, 0, 64), al = sw128_desc(st + L::oAKQl, 0, 64);
+                    const uint64_t bh = sw128_desc(sbase + L::oBSh, 0, MS), bl = sw128_desc(sbase + L::oBSl, 0, MS);
+#pragma unroll
                     for (int ks = 0; ks < DK / 8; ++ks) {
-                        const uint64_t a = sw128_desc(st + L::oAKQh, ks, 64);
-                        mma_tf32(tD1, a, sw128_desc(sbase + L::oBSh, ks, MS), idA, ks > 0);
-                        mma_tf32(tD1, a, sw128_desc(sbase + L::oBSl, ks, MS), idA, 1);
-                        if constexpr (!EXACT)
-                            mma_tf32(tD1, sw128_desc(st + L::oAKQl, ks, 64), sw128_desc(sbase + L::oBSh, ks, MS),
-                                     idA, 1);
+                        const uint64_t oa = sw128_ks_off(ks, 64), ob = sw128_ks_off(ks, MS);
+                        mma_tf32(tD1, ah + oa, bh + ob, idA, ks > 0);
+                        mma_tf32(tD1, ah + oa, bl + ob, idA, 1);
+                        if constexpr (!EXACT) mma_tf32(tD1, al + oa, bh + ob, idA, 1);
                     }
                     mma_commit(bar_a);
+                    GDN_SCAN_TRACE(cl, 3);
                     if (!mbar_wait(bar_a, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
+                    GDN_SCAN_TRACE(cl, 4);
                 }
             }
             named_bar(2, 128);
             if (*abort_flag) { aborted = true; break; }
             tc_fence_after();
-            const int4 ct = chunk_tab[c_begin + cl];
-            const int64_t t0 = ct.y;
-            const int Lr = ct.z;
+            const int64_t t0 = seq_t0 + (int64_t)cl * kChunk;
+            const int Lr = (int)((seq_end - t0) < kChunk ? (seq_end - t0) : kChunk);
             const float* gate = stf + L::oGate / 4;
             const float* Vs = stf + L::oV / 4;
             const float Gam = (lane < 16) ? gate[tok] : 0.f;
@@ -558,7 +694,7 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
 #pragma unroll
                     for (int i = 0; i < MS; ++i) {
                         float hi, lo;
-                        tf32_split(Vs[tok * MS + i] - Gam * x[i], hi, lo);
+                        tf32_split(Vs[i * 33 + tok] - Gam * x[i], hi, lo);
                         const uint32_t o = sw128_off(i, tok, MS);
                         st_shared_f32(sbase + L::oBYh + o, hi);
                         st_shared_f32(sbase + L::oBYl + o, lo);
@@ -573,17 +709,20 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
             named_bar(2, 128);
             // ---- MMA_b: [U; PU] = [T''; PT''] Y
             if (tid == 0) {
+                GDN_SCAN_TRACE(cl, 5);
                 tc_fence_after();
-#pragma unroll 1
+                const uint64_t ah = sw128_desc(st + L::oABh, 0, 64), al = sw128_desc(st + L::oABl, 0, 64);
+                const uint64_t bh = sw128_desc(sbase + L::oBYh, 0, MS), bl = sw128_desc(sbase + L::oBYl, 0, MS);
+#pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t ah = sw128_desc(st + L::oABh, ks, 64);
-                    const uint64_t bh = sw128_desc(sbase + L::oBYh, ks, MS);
-                    mma_tf32(tD2, ah, bh, idB, ks > 0);
-                    mma_tf32(tD2, ah, sw128_desc(sbase + L::oBYl, ks, MS), idB, 1);
-                    mma_tf32(tD2, sw128_desc(st + L::oABl, ks, 64), bh, idB, 1);
+                    const uint64_t oa = sw128_ks_off(ks, 64), ob = sw128_ks_off(ks, MS);
+                    mma_tf32(tD2, ah + oa, bh + ob, idB, ks > 0);
+                    mma_tf32(tD2, ah + oa, bl + ob, idB, 1);
+                    mma_tf32(tD2, al + oa, bh + ob, idB, 1);
                 }
                 mma_commit(bar_b);
                 if (!mbar_wait(bar_b, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
+                GDN_SCAN_TRACE(cl, 6);
             }
             named_bar(2, 128);
             if (*abort_flag) { aborted = true; break; }
@@ -607,27 +746,31 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                     fence_async_smem();
                 } else if (lane < 16 && tok < Lr) {
                     // O = s (diag(Gamma) Z + P U)
-                    T* dst = out + ((size_t)(t0 + tok) * H + h) * DV + r0;
+                    float o[MS];
 #pragma unroll
-                    for (int i = 0; i < MS; ++i) Elem<T>::st(dst + i, scale * fmaf(Gam, za[i], u[i]));
+                    for (int i = 0; i < MS; ++i) o[i] = scale * fmaf(Gam, za[i], u[i]);
+                    store_row<MS>(out + ((size_t)(t0 + tok) * H + h) * DV + r0, o);
                 }
             }
             tc_fence_before();
             named_bar(2, 128);
             // ---- MMA_c: dS^T = K^T U~   (its completion also frees the stage buffer)
             if (tid == 0) {
+                GDN_SCAN_TRACE(cl, 7);
                 tc_fence_after();
-#pragma unroll 1
+                const uint64_t ah = sw128_desc(st + L::oAKTh, 0, DK), al = sw128_desc(st + L::oAKTl, 0, DK);
+                const uint64_t bh = sw128_desc(sbase + L::oBUh, 0, MS), bl = sw128_desc(sbase + L::oBUl, 0, MS);
+#pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t ah = sw128_desc(st + L::oAKTh, ks, DK);
-                    const uint64_t bh = sw128_desc(sbase + L::oBUh, ks, MS);
-                    mma_tf32(tD3, ah, bh, idC, ks > 0);
-                    mma_tf32(tD3, ah, sw128_desc(sbase + L::oBUl, ks, MS), idC, 1);
-                    if constexpr (!EXACT) mma_tf32(tD3, sw128_desc(st + L::oAKTl, ks, DK), bh, idC, 1);
+                    const uint64_t oa = sw128_ks_off(ks, DK), ob = sw128_ks_off(ks, MS);
+                    mma_tf32(tD3, ah + oa, bh + ob, idC, ks > 0);
+                    mma_tf32(tD3, ah + oa, bl + ob, idC, 1);
+                    if constexpr (!EXACT) mma_tf32(tD3, al + oa, bh + ob, idC, 1);
                 }
                 mma_commit(bar_c);
                 mma_commit(&empty[s]);
                 if (!mbar_wait(bar_c, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
+                GDN_SCAN_TRACE(cl, 8);
             }
             named_bar(2, 128);
             if (*abort_flag) { aborted = true; break; }
@@ -641,6 +784,7 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
 #pragma unroll
                 for (int i = 0; i < MS; ++i) S[i] = fmaf(GamC, S[i], ds[i]);
             }
+            GDN_SCAN_TRACE(cl, 9);
             tc_fence_before();
         }
         if (state_out && owns && !aborted) {

@@ -175,25 +175,28 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t base, int ks, int R)
     return d;
 }
 
+// Offset, in the descriptor's 16-byte start-address units, of K-slice `ks` relative to slice 0 of
+// a tile of R rows: adding it to the slice-0 descriptor gives the slice-ks descriptor (the start
+// address field cannot overflow for tiles inside the 227 KB of shared memory).
+__host__ __device__ constexpr uint64_t sw128_ks_off(int ks, int R)
+{
+    return (uint64_t)((ks >> 2) * (R * 8) + (ks & 3) * 2);
+}
+
 // Instruction descriptor: kind::tf32, fp32 accumulator, both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N)
 {
     return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// TF32 split x = hi + lo: hi keeps the 10 explicit mantissa bits (round to nearest), lo is the
-// exact fp32 remainder rounded the same way.  hi*hi + hi*lo + lo*hi recovers an fp32-accurate
-// product on TF32 tensor cores.
-__device__ __forceinline__ float tf32_round(float x)
-{
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
-}
+// TF32 split x = hi + lo: hi keeps the sign, exponent and the 10 leading mantissa bits of x (the
+// bits a TF32 operand carries), lo = x - hi is exact in fp32 and the tensor core reads its leading
+// 11 significant bits.  hi*hi + hi*lo + lo*hi then recovers an fp32-accurate product; the dropped
+// lo*lo term and the unread tail of lo are both below 2^-21 relative.
 __device__ __forceinline__ void tf32_split(float x, float& hi, float& lo)
 {
-    hi = tf32_round(x);
-    lo = tf32_round(x - hi);
+    hi = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
+    lo = x - hi;
 }
 
 }  // namespace sm100
