@@ -3,10 +3,12 @@
 // Every entry point declared in include/gdn.h is defined here.  The kernels live in the .cuh files
 // included below, so the whole library is one translation unit and the per-device status word is
 // one symbol.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
 #include <mutex>
+#include <type_traits>
 #include <string>
 #include <vector>
 
@@ -14,6 +16,7 @@
 #include "gdn_decode.cuh"
 #include "gdn_plan.cuh"
 #include "gdn_prefill_tc.cuh"
+#include "gdn_scan_bf16.cuh"
 
 namespace gdn {
 
@@ -104,6 +107,43 @@ static int dispatch_decode(const void* q, const void* k, const void* v, const fl
     return launch_decode<T, 64, 64>(q, k, v, g, beta, state, out, B, H, st);
 }
 
+// ---- tensor maps (2-D tiled views of q/k/v) -------------------------------------------------------
+// cuTensorMapEncodeTiled is taken from the driver through the runtime's entry-point query, so the
+// library does not link libcuda directly.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled()
+{
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [rows, inner] bf16 matrix with row stride `row_elems`, tiles of box_rows x box_inner elements;
+// rows past the end read as zeros.
+static bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_elems,
+                           uint32_t box_inner, uint32_t box_rows, bool swizzle128)
+{
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {row_elems * 2};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 #ifndef GDN_SCAN_MS
 #define GDN_SCAN_MS 32
 #endif
@@ -149,6 +189,31 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         k1<<<grid, 128, PL::kBytes, st>>>(static_cast<const T*>(q), static_cast<const T*>(k), g, beta, meta,
                                           chunk_tab, op, H, status);
         if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
+    }
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        // bf16 inputs: operands staged by tensor maps, bf16 tensor-core products for K and Q
+        constexpr int MSB = 32;
+        using SB2 = ScanBf16Smem<DK, MSB, 2>;
+        using SB3 = ScanBf16Smem<DK, MSB, 3>;
+        constexpr int ST = (SB3::kBytes + 1024 <= 228 * 1024) ? 3 : 2;
+        using SB = ScanBf16Smem<DK, MSB, ST>;
+        static_assert(SB2::kBytes + 1024 <= 228 * 1024, "bf16 scan shared memory");
+        CUtensorMap tq, tk, tv;
+        const uint64_t Tn = (uint64_t)(T_total > 0 ? T_total : 1);
+        if (!make_tmap_bf16(&tq, q, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, true) ||
+            !make_tmap_bf16(&tk, k, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, true) ||
+            !make_tmap_bf16(&tv, v, (uint64_t)H * DV, Tn, (uint64_t)H * DV, MSB, 32, false))
+            return GDN_ERR_CUDA;
+        auto kb = gdn_scan_bf16_kernel<DK, DV, MSB, ST>;
+        if (cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SB::kBytes) != cudaSuccess)
+            return GDN_ERR_LAUNCH;
+        {
+            ProfScope prof("gdn_scan_bf16_kernel", st);
+            kb<<<dim3((unsigned)N, H, DV / MSB), 256, SB::kBytes, st>>>(
+                tq, tk, tv, meta, chunk_off, chunk_tab, reinterpret_cast<const uint8_t*>(op), state_in,
+                static_cast<__nv_bfloat16*>(out), state_out, H, status);
+        }
+        return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
     }
     // state rows per CTA and CTAs per SM of the scan (compile-time tuning knobs)
     constexpr int MS = GDN_SCAN_MS;

@@ -41,8 +41,14 @@
 
 namespace gdn {
 
-constexpr int kOpStride = 64 * 32 + 128;   // floats per (chunk, head) in the operator workspace
-constexpr int kGateOff = 64 * 32;          // gates: Gamma[32], delta[32], Gamma_31, pad
+// Per-(chunk, head) operator record in the workspace.  It is the byte image that the scan kernels
+// copy straight into shared memory: the TF32 hi and lo parts of [T''; P T''] (64 x 32, K-major,
+// 128-byte swizzle) followed by the gate vectors Gamma[32], delta[32], Gamma_31 (fp32, padded).
+constexpr uint32_t kOpHi = 0;
+constexpr uint32_t kOpLo = 8192;
+constexpr uint32_t kOpGate = 16384;
+constexpr uint32_t kOpCopyBytes = 16384 + 80 * 4;   // staged per chunk (operator + gates)
+constexpr uint32_t kOpBytes = 16384 + 512;          // record stride in the workspace
 
 template <typename T>
 struct ExactTF32 { static constexpr bool value = false; };
@@ -72,25 +78,22 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, flo
     }
 }
 
-__device__ __forceinline__ void st_shared_f4(uint32_t addr, float a, float b, float c, float d)
+// Shared-memory stores by 32-bit shared address.  No memory clobber: the compiler may move other
+// loads and stores across them (none of the kernels' threads reads back what it stores before a
+// fence or barrier, and those carry the clobber that orders everything).
+__device__ __forceinline__ void sts4(uint32_t base, uint32_t off, float a, float b, float c, float d)
 {
-    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(base + off), "f"(a), "f"(b), "f"(c), "f"(d));
 }
-__device__ __forceinline__ void st_shared_f32(uint32_t addr, float a)
+__device__ __forceinline__ void sts1(uint32_t base, uint32_t off, float a)
 {
-    asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(a) : "memory");
-}
-__device__ __forceinline__ float ld_shared_f32(uint32_t addr)
-{
-    float a;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(a) : "r"(addr) : "memory");
-    return a;
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(base + off), "f"(a));
 }
 
 // Stores 8 consecutive K-elements (k0 % 8 == 0) of row r of a K-major SW128 tile of R rows, as hi
 // (and lo when SPLIT) parts.
 template <bool SPLIT>
-__device__ __forceinline__ void put8(uint32_t hi_base, uint32_t lo_base, int r, int k0, int R, const float (&x)[8])
+__device__ __forceinline__ void put8(uint32_t hi, uint32_t lo, int r, int k0, int R, const float (&x)[8])
 {
     using namespace sm100;
     const uint32_t o0 = sw128_off(r, k0, R), o1 = sw128_off(r, k0 + 4, R);
@@ -98,13 +101,13 @@ __device__ __forceinline__ void put8(uint32_t hi_base, uint32_t lo_base, int r, 
         float h[8], l[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) tf32_split(x[i], h[i], l[i]);
-        st_shared_f4(hi_base + o0, h[0], h[1], h[2], h[3]);
-        st_shared_f4(hi_base + o1, h[4], h[5], h[6], h[7]);
-        st_shared_f4(lo_base + o0, l[0], l[1], l[2], l[3]);
-        st_shared_f4(lo_base + o1, l[4], l[5], l[6], l[7]);
+        sts4(hi, o0, h[0], h[1], h[2], h[3]);
+        sts4(hi, o1, h[4], h[5], h[6], h[7]);
+        sts4(lo, o0, l[0], l[1], l[2], l[3]);
+        sts4(lo, o1, l[4], l[5], l[6], l[7]);
     } else {
-        st_shared_f4(hi_base + o0, x[0], x[1], x[2], x[3]);
-        st_shared_f4(hi_base + o1, x[4], x[5], x[6], x[7]);
+        sts4(hi, o0, x[0], x[1], x[2], x[3]);
+        sts4(hi, o1, x[4], x[5], x[6], x[7]);
     }
 }
 
@@ -347,25 +350,27 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, 
             P[i * L::LD + j] = dd * P[i * L::LD + j];
         }
         __syncthreads();
-        // T = (I + A)^-1, one lane per column j with the column in registers (entries above the
-        // diagonal are zero, so every lane runs the same unrolled recurrence); T'' = T diag(beta).
+        // T = (I + A)^-1 by forward substitution, one lane per column j of T with the column in
+        // registers.  Column-oriented: once t[i] is final it is subtracted, times column i of A,
+        // from every later row, so each of the 31 steps is a set of independent FMAs.
+        // T'' = T diag(beta).
         if (warp == 0) {
             const int j = lane;
             float t[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                float acc = 0.f;
+            for (int r = 0; r < 32; ++r) t[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
-                for (int m = 0; m < i; ++m) acc = fmaf(G[i * L::LD + m], t[m], acc);
-                t[i] = (i == j) ? 1.f : ((i < j) ? 0.f : -acc);
+            for (int i = 0; i < 31; ++i) {
+#pragma unroll
+                for (int r = i + 1; r < 32; ++r) t[r] = fmaf(-G[r * L::LD + i], t[i], t[r]);
             }
             const float bj = bet[j];
 #pragma unroll
             for (int i = 0; i < 32; ++i) Tm[i * L::LD + j] = t[i] * bj;
         }
         __syncthreads();
-        // operator rows [T''; P T''] and the gates
-        float* dst = op + ((size_t)gc * H + h) * kOpStride;
+        // operator record: [T''; P T''] split into TF32 hi/lo in the swizzled image, and the gates
+        uint8_t* dst = reinterpret_cast<uint8_t*>(op) + ((size_t)gc * H + h) * kOpBytes;
         for (int idx = tid; idx < 64 * 32; idx += 128) {
             const int i = idx >> 5, j = idx & 31;
             float val;
@@ -377,13 +382,20 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, 
                 for (int m = j; m <= ii; ++m) acc = fmaf(P[ii * L::LD + m], Tm[m * L::LD + j], acc);
                 val = acc;
             }
-            dst[idx] = val;
+            float hi, lo;
+            tf32_split(val, hi, lo);
+            const uint32_t o = sw128_off(i, j, 64);
+            *reinterpret_cast<float*>(dst + kOpHi + o) = hi;
+            *reinterpret_cast<float*>(dst + kOpLo + o) = lo;
         }
-        if (tid < 32) {
+        if (tid < 80) {
+            float* gt = reinterpret_cast<float*>(dst + kOpGate);
             const float gl = gam[31];
-            dst[kGateOff + tid] = expf(gam[tid]);
-            dst[kGateOff + 32 + tid] = expf(gl - gam[tid]);
-            if (tid == 0) dst[kGateOff + 64] = expf(gl);
+            float val = 0.f;
+            if (tid < 32) val = expf(gam[tid]);
+            else if (tid < 64) val = expf(gl - gam[tid - 32]);
+            else if (tid == 64) val = expf(gl);
+            gt[tid] = val;
         }
         __syncthreads();
         cur = nxt;
@@ -411,7 +423,7 @@ struct ScanSmem {
     static constexpr uint32_t kAKQ = 64 * DK * 4;                     // [K;Q], 64 x DK
     static constexpr uint32_t kAKT = DK * 32 * 4;                     // K^T, DK x 32
     static constexpr uint32_t kAB = 64 * 32 * 4;                      // [T'';PT''], 64 x 32
-    static constexpr uint32_t kB32 = ((MS * 32 * 4) + 1023) & ~1023u; // MS x 32 B-operand tile
+    static constexpr uint32_t kB32 = ((2 * MS * 32 * 4) + 1023) & ~1023u; // [hi; lo] 2MS x 32 tile
     // one stage
     static constexpr uint32_t oAKQh = 0;
     static constexpr uint32_t oAKQl = oAKQh + kAKQ;
@@ -419,17 +431,16 @@ struct ScanSmem {
     static constexpr uint32_t oAKTl = oAKTh + kAKT;
     static constexpr uint32_t oABh = oAKTl + (EXACT ? 0 : kAKT);
     static constexpr uint32_t oABl = oABh + kAB;
-    static constexpr uint32_t oV = oABl + kAB;                        // fp32 [MS][33] (V^T, padded)
-    static constexpr uint32_t oGate = oV + 33 * MS * 4;               // fp32 [80]
-    static constexpr uint32_t kStage = ((oGate + 80 * 4) + 1023) & ~1023u;
+    static constexpr uint32_t oGate = oABl + kAB;                     // fp32 [80] (copied with the operator)
+    static constexpr uint32_t oV = oGate + 80 * 4;                    // fp32 [MS][33] (V^T, padded)
+    static constexpr uint32_t kStage = ((oV + 33 * MS * 4) + 1023) & ~1023u;
     // shared by all stages
-    static constexpr uint32_t oBSh = STAGES * kStage;                 // S as B operand: MS x DK
-    static constexpr uint32_t oBSl = oBSh + MS * DK * 4;
-    static constexpr uint32_t oBYh = oBSl + MS * DK * 4;              // Y as B: MS x 32
-    static constexpr uint32_t oBYl = oBYh + kB32;
-    static constexpr uint32_t oBUh = oBYl + kB32;                     // U~ as B: MS x 32
-    static constexpr uint32_t oBUl = oBUh + kB32;
-    static constexpr uint32_t oBar = oBUl + kB32;                     // full[S], empty[S], a, b, c
+    // B operands hold hi rows 0..MS-1 and lo rows MS..2MS-1 of one tile, so one MMA of N = 2MS
+    // forms both the hi and the lo product of the split
+    static constexpr uint32_t oBS = STAGES * kStage;                  // S: 2MS x DK
+    static constexpr uint32_t oBY = oBS + 2 * MS * DK * 4;            // Y: 2MS x 32
+    static constexpr uint32_t oBU = oBY + kB32;                       // U~: 2MS x 32
+    static constexpr uint32_t oBar = oBU + kB32;                      // full[S], empty[S], a, b, c
     static constexpr uint32_t oTmem = oBar + 8 * (2 * STAGES + 4);   // + drain barrier
     static constexpr uint32_t oAbort = oTmem + 4;
     static constexpr uint32_t kTotal = oAbort + 4;
@@ -490,27 +501,25 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(tslot, 128);
+        tmem_alloc(tslot, 256);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t tD1 = tmem, tD2 = tmem + 32, tD3 = tmem + 64;   // accumulator columns
+    const uint32_t tD1 = tmem, tD2 = tmem + 64, tD3 = tmem + 128;  // accumulators, 2MS columns each
 
     if (warp >= 4) {
         // ------------------------------------------------------------------ producers
-        // Per chunk and thread: DK/64 blocks of 4 tokens x 8 features of K or Q, two 8-float
-        // groups of the [T''; P T''] operator, one 8-element group of the V slice, one gate value.
+        // Per chunk and thread: DK/64 blocks of 4 tokens x 8 features of K or Q and one 8-element
+        // group of the V slice; the [T''; P T''] image and the gates come by one bulk copy.
         const int ptid = tid - 128;
         constexpr int NB = DK / 64;
         constexpr int NVG = 4 * MS;                    // 8-element groups in the V slice
         struct Pre {
             Raw8<T> kq[NB][4];
-            Raw8<float> ab[2];
             Raw8<T> vv;
-            float gt;
         };
         auto load_chunk = [&](Pre& p, int cl) {
             const int gc = c_begin + cl;
@@ -529,18 +538,12 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                     else p.kq[u][r].zero();
                 }
             }
-            const float* opc = op + ((size_t)gc * H + h) * kOpStride;
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int idx = ptid + 128 * u;
-                p.ab[u].load(opc + (idx >> 2) * 32 + (idx & 3) * 8);
-            }
+            (void)gc;
             if (ptid < NVG) {
                 const int j = ptid / (MS / 8), cg = ptid % (MS / 8);
                 if (j < Lr) p.vv.load(v + ((size_t)(t0 + j) * H + h) * DV + r0 + cg * 8);
                 else p.vv.zero();
             }
-            p.gt = (ptid < 65) ? __ldg(opc + kGateOff + ptid) : 0.f;
         };
         auto store_chunk = [&](const Pre& p, int s) {
             const uint32_t st = sbase + s * L::kStage;
@@ -563,23 +566,16 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                     for (int e = 0; e < 8; ++e) {
                         const uint32_t o = sw128_off(kg * 8 + e, 4 * jg, DK);
                         if constexpr (EXACT) {
-                            st_shared_f4(st + L::oAKTh + o, x[0][e], x[1][e], x[2][e], x[3][e]);
+                            sts4(st + L::oAKTh, o, x[0][e], x[1][e], x[2][e], x[3][e]);
                         } else {
                             float hi[4], lo[4];
 #pragma unroll
                             for (int r = 0; r < 4; ++r) tf32_split(x[r][e], hi[r], lo[r]);
-                            st_shared_f4(st + L::oAKTh + o, hi[0], hi[1], hi[2], hi[3]);
-                            st_shared_f4(st + L::oAKTl + o, lo[0], lo[1], lo[2], lo[3]);
+                            sts4(st + L::oAKTh, o, hi[0], hi[1], hi[2], hi[3]);
+                            sts4(st + L::oAKTl, o, lo[0], lo[1], lo[2], lo[3]);
                         }
                     }
                 }
-            }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int idx = ptid + 128 * u;
-                float x[8];
-                p.ab[u].get(x);
-                put8<true>(st + L::oABh, st + L::oABl, idx >> 2, (idx & 3) * 8, 64, x);
             }
             if (ptid < NVG) {
                 const int j = ptid / (MS / 8), cg = ptid % (MS / 8);
@@ -589,7 +585,6 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
 #pragma unroll
                 for (int e = 0; e < 8; ++e) Vt[(cg * 8 + e) * 33 + j] = x[e];
             }
-            if (ptid < 80) stf[L::oGate / 4 + ptid] = p.gt;
         };
 
         Pre cur, nxt;
@@ -605,6 +600,13 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                 if (*abort_flag) break;
             }
             GDN_SCAN_TRACE(cl, 11);
+            if (ptid == 0) {
+                // operator image and gates: one bulk copy, counted by the same barrier
+                mbar_expect_tx(&full[s], kOpCopyBytes);
+                bulk_load(sbase + s * L::kStage + L::oABh,
+                          reinterpret_cast<const uint8_t*>(op) + ((size_t)(c_begin + cl) * H + h) * kOpBytes,
+                          kOpCopyBytes, &full[s]);
+            }
             store_chunk(cur, s);
             fence_async_smem();
             mbar_arrive(&full[s]);
@@ -622,9 +624,8 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
             S[i] = (state_in && owns) ? state_in[(((size_t)n * H + h) * DV + r0 + i) * DK + c_own] : 0.f;
 
         const float scale = rsqrtf((float)DK);
-        constexpr uint32_t idA = idesc_tf32(64, MS);
-        constexpr uint32_t idB = idesc_tf32(64, MS);
-        constexpr uint32_t idC = idesc_tf32(DK, MS);
+        constexpr uint32_t idA1 = idesc_tf32(64, MS), idA2 = idesc_tf32(64, 2 * MS);
+        constexpr uint32_t idC1 = idesc_tf32(DK, MS), idC2 = idesc_tf32(DK, 2 * MS);
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         const int row16 = warp * 16 + lane;          // accumulator row of an M=64 product in this lane
         const int tok = (warp < 2) ? row16 : (row16 - 32);
@@ -638,9 +639,8 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                 for (int i = 0; i < MS; ++i) {
                     float hi, lo;
                     tf32_split(S[i], hi, lo);
-                    const uint32_t o = sw128_off(i, c_own, MS);
-                    st_shared_f32(sbase + L::oBSh + o, hi);
-                    st_shared_f32(sbase + L::oBSl + o, lo);
+                    sts1(sbase + L::oBS, sw128_off(i, c_own, 2 * MS), hi);
+                    sts1(sbase + L::oBS, sw128_off(MS + i, c_own, 2 * MS), lo);
                 }
             }
             if (cl == nch) break;
@@ -652,7 +652,7 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
             const uint32_t st = sbase + s * L::kStage;
             const float* stf = reinterpret_cast<const float*>(sm + s * L::kStage);
 
-            // ---- MMA_a: [X; Z] = [K; Q] S^T
+            // ---- MMA_a: [X; Z] = [K; Q] S^T   (N = 2MS: columns [0, MS) hi, [MS, 2MS) lo)
             if (tid == 0) {
                 if (!mbar_wait(&full[s], (uint32_t)(cl / STAGES) & 1u, abort_flag)) {
                     tc_abort(status, abort_flag);
@@ -660,13 +660,12 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                     GDN_SCAN_TRACE(cl, 2);
                     tc_fence_after();
                     const uint64_t ah = sw128_desc(st + L::oAKQh, 0, 64), al = sw128_desc(st + L::oAKQl, 0, 64);
-                    const uint64_t bh = sw128_desc(sbase + L::oBSh, 0, MS), bl = sw128_desc(sbase + L::oBSl, 0, MS);
+                    const uint64_t b = sw128_desc(sbase + L::oBS, 0, 2 * MS);
 #pragma unroll
                     for (int ks = 0; ks < DK / 8; ++ks) {
-                        const uint64_t oa = sw128_ks_off(ks, 64), ob = sw128_ks_off(ks, MS);
-                        mma_tf32(tD1, ah + oa, bh + ob, idA, ks > 0);
-                        mma_tf32(tD1, ah + oa, bl + ob, idA, 1);
-                        if constexpr (!EXACT) mma_tf32(tD1, al + oa, bh + ob, idA, 1);
+                        const uint64_t oa = sw128_ks_off(ks, 64), ob = sw128_ks_off(ks, 2 * MS);
+                        mma_tf32(tD1, ah + oa, b + ob, idA2, ks > 0);
+                        if constexpr (!EXACT) mma_tf32(tD1, al + oa, b + ob, idA1, 1);   // lo x hi rows
                     }
                     mma_commit(bar_a);
                     GDN_SCAN_TRACE(cl, 3);
@@ -675,6 +674,7 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                 }
             }
             named_bar(2, 128);
+            GDN_SCAN_TRACE(cl, 13);
             if (*abort_flag) { aborted = true; break; }
             tc_fence_after();
             const int64_t t0 = seq_t0 + (int64_t)cl * kChunk;
@@ -685,25 +685,31 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
             const float del = (lane < 16 && warp < 2) ? gate[32 + tok] : 0.f;
             const float GamC = gate[64];
             float za[MS];
+            {
+                float xh[MS], xl[MS];
+                tmem_ld<MS>(tD1 + lane_base, xh);
+                tmem_ld<MS>(tD1 + lane_base + MS, xl);
+                tmem_ld_wait();
+                GDN_SCAN_TRACE(cl, 14);
+#pragma unroll
+                for (int i = 0; i < MS; ++i) za[i] = xh[i] + xl[i];
+            }
             if (warp < 2) {
                 // Y = V - diag(Gamma) X  ->  B operand of MMA_b (row i of S, K index = token)
-                float x[MS];
-                tmem_ld<MS>(tD1 + lane_base, x);
-                tmem_ld_wait();
                 if (lane < 16) {
+                    float vt[MS];
+#pragma unroll
+                    for (int i = 0; i < MS; ++i) vt[i] = Vs[i * 33 + tok];
 #pragma unroll
                     for (int i = 0; i < MS; ++i) {
                         float hi, lo;
-                        tf32_split(Vs[i * 33 + tok] - Gam * x[i], hi, lo);
-                        const uint32_t o = sw128_off(i, tok, MS);
-                        st_shared_f32(sbase + L::oBYh + o, hi);
-                        st_shared_f32(sbase + L::oBYl + o, lo);
+                        tf32_split(vt[i] - Gam * za[i], hi, lo);
+                        sts1(sbase + L::oBY, sw128_off(i, tok, 2 * MS), hi);
+                        sts1(sbase + L::oBY, sw128_off(MS + i, tok, 2 * MS), lo);
                     }
                 }
+                GDN_SCAN_TRACE(cl, 15);
                 fence_async_smem();
-            } else {
-                tmem_ld<MS>(tD1 + lane_base, za);    // Z rows, token i = row16 - 32
-                tmem_ld_wait();
             }
             tc_fence_before();
             named_bar(2, 128);
@@ -712,13 +718,12 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                 GDN_SCAN_TRACE(cl, 5);
                 tc_fence_after();
                 const uint64_t ah = sw128_desc(st + L::oABh, 0, 64), al = sw128_desc(st + L::oABl, 0, 64);
-                const uint64_t bh = sw128_desc(sbase + L::oBYh, 0, MS), bl = sw128_desc(sbase + L::oBYl, 0, MS);
+                const uint64_t b = sw128_desc(sbase + L::oBY, 0, 2 * MS);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t oa = sw128_ks_off(ks, 64), ob = sw128_ks_off(ks, MS);
-                    mma_tf32(tD2, ah + oa, bh + ob, idB, ks > 0);
-                    mma_tf32(tD2, ah + oa, bl + ob, idB, 1);
-                    mma_tf32(tD2, al + oa, bh + ob, idB, 1);
+                    const uint64_t oa = sw128_ks_off(ks, 64), ob = sw128_ks_off(ks, 2 * MS);
+                    mma_tf32(tD2, ah + oa, b + ob, idA2, ks > 0);
+                    mma_tf32(tD2, al + oa, b + ob, idA1, 1);       // lo x hi rows
                 }
                 mma_commit(bar_b);
                 if (!mbar_wait(bar_b, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
@@ -728,9 +733,12 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
             if (*abort_flag) { aborted = true; break; }
             tc_fence_after();
             {
-                float u[MS];
+                float u[MS], ul[MS];
                 tmem_ld<MS>(tD2 + lane_base, u);
+                tmem_ld<MS>(tD2 + lane_base + MS, ul);
                 tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < MS; ++i) u[i] += ul[i];
                 if (warp < 2) {
                     // U~ = diag(delta) U  ->  B operand of MMA_c
                     if (lane < 16) {
@@ -738,9 +746,8 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                         for (int i = 0; i < MS; ++i) {
                             float hi, lo;
                             tf32_split(del * u[i], hi, lo);
-                            const uint32_t o = sw128_off(i, tok, MS);
-                            st_shared_f32(sbase + L::oBUh + o, hi);
-                            st_shared_f32(sbase + L::oBUl + o, lo);
+                            sts1(sbase + L::oBU, sw128_off(i, tok, 2 * MS), hi);
+                            sts1(sbase + L::oBU, sw128_off(MS + i, tok, 2 * MS), lo);
                         }
                     }
                     fence_async_smem();
@@ -759,13 +766,12 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                 GDN_SCAN_TRACE(cl, 7);
                 tc_fence_after();
                 const uint64_t ah = sw128_desc(st + L::oAKTh, 0, DK), al = sw128_desc(st + L::oAKTl, 0, DK);
-                const uint64_t bh = sw128_desc(sbase + L::oBUh, 0, MS), bl = sw128_desc(sbase + L::oBUl, 0, MS);
+                const uint64_t b = sw128_desc(sbase + L::oBU, 0, 2 * MS);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t oa = sw128_ks_off(ks, DK), ob = sw128_ks_off(ks, MS);
-                    mma_tf32(tD3, ah + oa, bh + ob, idC, ks > 0);
-                    mma_tf32(tD3, ah + oa, bl + ob, idC, 1);
-                    if constexpr (!EXACT) mma_tf32(tD3, al + oa, bh + ob, idC, 1);
+                    const uint64_t oa = sw128_ks_off(ks, DK), ob = sw128_ks_off(ks, 2 * MS);
+                    mma_tf32(tD3, ah + oa, b + ob, idC2, ks > 0);
+                    if constexpr (!EXACT) mma_tf32(tD3, al + oa, b + ob, idC1, 1);   // lo x hi rows
                 }
                 mma_commit(bar_c);
                 mma_commit(&empty[s]);
@@ -778,11 +784,12 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
             {
                 // S' = Gamma_31 S + dS   (row c_own of dS^T; for dk = 64 the M=64 layout puts row
                 // 16w+t in lane 32w+t, which is c_own of that lane)
-                float ds[MS];
+                float ds[MS], dl[MS];
                 tmem_ld<MS>(tD3 + lane_base, ds);
+                tmem_ld<MS>(tD3 + lane_base + MS, dl);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < MS; ++i) S[i] = fmaf(GamC, S[i], ds[i]);
+                for (int i = 0; i < MS; ++i) S[i] = fmaf(GamC, S[i], ds[i] + dl[i]);
             }
             GDN_SCAN_TRACE(cl, 9);
             tc_fence_before();
@@ -802,7 +809,7 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
         mbar_wait(bar_drain, 0, &never, 100000000ull);
     }
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 128);
+    if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 }  // namespace gdn

@@ -1,0 +1,362 @@
+// gdn_scan_bf16.cuh -- chunk-sequential scan of the chunked prefill for bf16 q/k/v (sm_100a).
+//
+// Same algebra as gdn_scan_tc_kernel (see gdn_prefill_tc.cuh): per chunk
+//
+//   MMA_a  [X ; Z]     = [K ; Q] S^T            M=64,  N=3MS, K=dk   kind::f16 (bf16)
+//   MMA_b  [U ; P U]   = [T'' ; P T''] Y        M=64,  N=2MS, K=32   kind::tf32 (3xTF32)
+//   MMA_c  (dS)^T      = K^T (diag(delta) U)    M=dk,  N=3MS, K=32   kind::f16 (bf16)
+//
+// What is specific to bf16 inputs:
+//   * q and k are exact bf16 values, so [K; Q] is used as stored: the tensor-memory-access engine
+//     copies the chunk's rows straight from global memory into the 128-byte-swizzled operand layout,
+//     and K^T for MMA_c is the same bytes read through an M-major descriptor.
+//   * The fp32 operand on the other side (S, U~) is split into three bf16 parts that carry its 24
+//     significant bits, stacked along N; one bf16 MMA (K=16) forms all three partial products, and
+//     the epilogue adds the three column blocks.  The result is fp32-accurate like the 3xTF32 split
+//     and needs half as many MMA instructions (bf16 takes 16 K-elements per instruction, TF32 8).
+//   * One producer thread stages each chunk with bulk copies (K/Q/V tiles by tensor map, the
+//     [T''; P T''] image and gates from the workspace) tracked by one transaction barrier; no thread
+//     converts or stores staged operands.
+//   * Rows of the last chunk of a sequence that lie beyond its end may hold the next sequence's
+//     tokens (or zeros past the tensor); the epilogues zero Y for them, the operator [T''; P T'']
+//     has zero columns for them, and their outputs are not stored, so they never contribute.
+#pragma once
+
+#include <cuda.h>
+
+#include "gdn_common.cuh"
+#include "gdn_prefill_tc.cuh"
+#include "gdn_sm100.cuh"
+
+namespace gdn {
+
+template <int DK, int MS, int STAGES>
+struct ScanBf16Smem {
+    static constexpr int NP = DK / 64;                                // 64-element panels of dk
+    // one stage
+    static constexpr uint32_t oAKQ = 0;                               // [K;Q] bf16: NP panels x 64 rows x 128 B
+    static constexpr uint32_t oOp = oAKQ + NP * 8192;                 // operator image + gates
+    static constexpr uint32_t oV = oOp + ((kOpCopyBytes + 1023) & ~1023u);   // V tile: 32 rows x MS bf16
+    static constexpr uint32_t kStage = ((oV + 32 * MS * 2) + 1023) & ~1023u;
+    static constexpr uint32_t kStageTx = NP * 2 * 4096 + kOpCopyBytes + 32 * MS * 2;
+    // shared by all stages
+    static constexpr uint32_t oBS = STAGES * kStage;                  // S parts: NP panels x 3MS rows x 128 B
+    static constexpr uint32_t oBY = oBS + NP * 3 * MS * 128;          // Y hi/lo (tf32): 2MS rows x 128 B
+    static constexpr uint32_t oBU = oBY + ((2 * MS * 128 + 1023) & ~1023u);  // U~ parts (bf16): 3MS rows x 128 B
+    static constexpr uint32_t oBar = oBU + ((3 * MS * 128 + 1023) & ~1023u);
+    static constexpr uint32_t oTmem = oBar + 8 * (2 * STAGES + 4);
+    static constexpr uint32_t oAbort = oTmem + 4;
+    static constexpr uint32_t kTotal = oAbort + 4;
+    static constexpr uint32_t kBytes = kTotal + 1024;
+};
+
+template <int DK, int DV, int MS, int STAGES>
+__global__ void __launch_bounds__(256, 1) gdn_scan_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                               const __grid_constant__ CUtensorMap tm_k,
+                                                               const __grid_constant__ CUtensorMap tm_v,
+                                                               const int* __restrict__ meta,
+                                                               const int* __restrict__ chunk_off,
+                                                               const int4* __restrict__ chunk_tab,
+                                                               const uint8_t* __restrict__ op,
+                                                               const float* state_in,
+                                                               __nv_bfloat16* __restrict__ out,
+                                                               float* state_out, int H, int* status)
+{
+    using namespace sm100;
+    using L = ScanBf16Smem<DK, MS, STAGES>;
+    static_assert(MS == 32, "bf16 scan: 32 state rows per CTA");
+    static_assert(DK == 64 || DK == 128, "DK");
+    static_assert(DV % MS == 0, "DV");
+    constexpr int NP = L::NP;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::oBar);
+    uint64_t* empty = full + STAGES;
+    uint64_t* bar_a = empty + STAGES;
+    uint64_t* bar_b = bar_a + 1;
+    uint64_t* bar_c = bar_a + 2;
+    uint64_t* bar_drain = bar_a + 3;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::oTmem);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::oAbort);
+
+    if (meta[1]) return;   // bad cu_seqlens: nothing is written
+    const int n = blockIdx.x, h = blockIdx.y, r0 = blockIdx.z * MS;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c_begin = chunk_off[n], c_end = chunk_off[n + 1];
+    const int nch = c_end - c_begin;
+    int64_t seq_t0 = 0, seq_end = 0;
+    if (nch > 0) {
+        const int4 first = chunk_tab[c_begin], last = chunk_tab[c_end - 1];
+        seq_t0 = first.y;
+        seq_end = (int64_t)last.y + last.z;
+    }
+
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(bar_a, 1);
+        mbar_init(bar_b, 1);
+        mbar_init(bar_c, 1);
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tslot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    // accumulators: D1 [X;Z] 3MS columns, D2 [U;PU] 2MS columns, D3 dS^T 3MS columns
+    const uint32_t tD1 = tmem, tD2 = tmem + 96, tD3 = tmem + 160;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------------ producer (one thread)
+        if (lane == 0) {
+            for (int cl = 0; cl < nch; ++cl) {
+                const int s = cl % STAGES;
+                if (cl >= STAGES &&
+                    !mbar_wait(&empty[s], (uint32_t)((cl / STAGES) - 1) & 1u, abort_flag)) {
+                    tc_abort(status, abort_flag);
+                    break;
+                }
+                const uint32_t st = sbase + s * L::kStage;
+                const int t0 = (int)(seq_t0 + (int64_t)cl * kChunk);
+                const int gc = c_begin + cl;
+                mbar_arrive_expect_tx(&full[s], L::kStageTx);
+#pragma unroll
+                for (int p = 0; p < NP; ++p) {
+                    tma_load_2d(st + L::oAKQ + p * 8192, &tm_k, h * DK + p * 64, t0, &full[s]);
+                    tma_load_2d(st + L::oAKQ + p * 8192 + 4096, &tm_q, h * DK + p * 64, t0, &full[s]);
+                }
+                bulk_load(st + L::oOp, op + ((size_t)gc * H + h) * kOpBytes, kOpCopyBytes, &full[s]);
+                tma_load_2d(st + L::oV, &tm_v, h * DV + r0, t0, &full[s]);
+            }
+        }
+    } else if (warp < 4) {
+        // ------------------------------------------------------------------ consumers
+        // thread (warp, lane) owns column c of the state slice: S[0..MS)[c]
+        const int c_own = (DK == 128) ? (warp * 32 + lane) : (warp * 16 + lane);
+        const bool owns = (DK == 128) || (lane < 16);
+        const int odd = lane & 1;
+        float S[MS];
+#pragma unroll
+        for (int i = 0; i < MS; ++i)
+            S[i] = (state_in && owns) ? state_in[(((size_t)n * H + h) * DV + r0 + i) * DK + c_own] : 0.f;
+
+        const float scale = rsqrtf((float)DK);
+        constexpr uint32_t idA = idesc_bf16(64, 3 * MS);
+        constexpr uint32_t idB1 = idesc_tf32(64, MS), idB2 = idesc_tf32(64, 2 * MS);
+        constexpr uint32_t idC = idesc_bf16(DK, 3 * MS, true);
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int row16 = warp * 16 + lane;          // accumulator row of an M=64 product in this lane
+        const int tok = (warp < 2) ? row16 : (row16 - 32);
+        bool aborted = false;
+
+        for (int cl = 0; cl <= nch; ++cl) {
+            // S -> three bf16 parts, B operand of MMA_a (rows: part * MS + i, K index: c_own).
+            // Lanes pair up (xor 1) so that every store writes two adjacent columns of one row.
+            {
+                // all lanes take part in the exchange; only lanes that own a column store
+#pragma unroll
+                for (int i = 0; i < MS; i += 2) {
+                    uint32_t a1, a2, a3, b1, b2, b3;
+                    bf16_split3(S[i], a1, a2, a3);       // row i
+                    bf16_split3(S[i + 1], b1, b2, b3);   // row i + 1
+                    // even lane keeps row i and sends its row-(i+1) parts; odd lane the reverse
+                    const uint32_t s1 = odd ? a1 : b1, s2 = odd ? a2 : b2, s3 = odd ? a3 : b3;
+                    const uint32_t t1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+                    const uint32_t t2 = __shfl_xor_sync(0xffffffffu, s2, 1);
+                    const uint32_t t3 = __shfl_xor_sync(0xffffffffu, s3, 1);
+                    const int row = odd ? i + 1 : i;
+                    const int kc = c_own & ~1;
+                    const uint32_t w1 = odd ? (t1 | (b1 << 16)) : (a1 | (t1 << 16));
+                    const uint32_t w2 = odd ? (t2 | (b2 << 16)) : (a2 | (t2 << 16));
+                    const uint32_t w3 = odd ? (t3 | (b3 << 16)) : (a3 | (t3 << 16));
+                    if (owns) {
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBS + sw128_off_h(row, kc, 3 * MS)), "r"(w1));
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBS + sw128_off_h(MS + row, kc, 3 * MS)), "r"(w2));
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBS + sw128_off_h(2 * MS + row, kc, 3 * MS)), "r"(w3));
+                    }
+                }
+            }
+            if (cl == nch) break;
+            fence_async_smem();
+            tc_fence_before();
+            named_bar(2, 128);      // every column of S written before MMA_a reads it
+            const int s = cl % STAGES;
+            const uint32_t st = sbase + s * L::kStage;
+            const uint8_t* stp = sm + s * L::kStage;
+
+            // ---- MMA_a: [X; Z] = [K; Q] S^T  (column blocks: the three parts of S)
+            if (tid == 0) {
+                if (!mbar_wait(&full[s], (uint32_t)(cl / STAGES) & 1u, abort_flag)) {
+                    tc_abort(status, abort_flag);
+                } else {
+                    tc_fence_after();
+                    const uint64_t a = sw128_desc(st + L::oAKQ, 0, 64);
+                    const uint64_t b = sw128_desc(sbase + L::oBS, 0, 3 * MS);
+#pragma unroll
+                    for (int ks = 0; ks < DK / 16; ++ks)
+                        mma_bf16(tD1, a + sw128_ks_off(ks, 64), b + sw128_ks_off(ks, 3 * MS), idA, ks > 0);
+                    mma_commit(bar_a);
+                    if (!mbar_wait(bar_a, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
+                }
+            }
+            named_bar(2, 128);
+            if (*abort_flag) { aborted = true; break; }
+            tc_fence_after();
+            const int64_t t0 = seq_t0 + (int64_t)cl * kChunk;
+            const int Lr = (int)((seq_end - t0) < kChunk ? (seq_end - t0) : kChunk);
+            const float* gate = reinterpret_cast<const float*>(stp + L::oOp + kOpGate);
+            const float Gam = (lane < 16) ? gate[tok] : 0.f;
+            const float del = (lane < 16 && warp < 2) ? gate[32 + tok] : 0.f;
+            const float GamC = gate[64];
+            float za[MS];
+            {
+                float x1[MS], x2[MS], x3[MS];
+                tmem_ld<MS>(tD1 + lane_base, x1);
+                tmem_ld<MS>(tD1 + lane_base + MS, x2);
+                tmem_ld<MS>(tD1 + lane_base + 2 * MS, x3);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < MS; ++i) za[i] = x1[i] + x2[i] + x3[i];
+            }
+            if (warp < 2) {
+                // Y = V - diag(Gamma) X (zero for rows past the sequence end) -> tf32 hi/lo rows of MMA_b's B
+                if (lane < 16) {
+                    float vt[MS];
+                    const uint4* vrow = reinterpret_cast<const uint4*>(stp + L::oV + tok * MS * 2);
+#pragma unroll
+                    for (int q4 = 0; q4 < MS / 8; ++q4) {
+                        const uint4 u = vrow[q4];
+                        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(hv[e]);
+                            vt[q4 * 8 + 2 * e] = f.x;
+                            vt[q4 * 8 + 2 * e + 1] = f.y;
+                        }
+                    }
+                    const bool live = tok < Lr;
+#pragma unroll
+                    for (int i = 0; i < MS; ++i) {
+                        float hi, lo;
+                        tf32_split(live ? vt[i] - Gam * za[i] : 0.f, hi, lo);
+                        sts1(sbase + L::oBY, sw128_off(i, tok, 2 * MS), hi);
+                        sts1(sbase + L::oBY, sw128_off(MS + i, tok, 2 * MS), lo);
+                    }
+                }
+                fence_async_smem();
+            }
+            tc_fence_before();
+            named_bar(2, 128);
+            // ---- MMA_b: [U; PU] = [T''; PT''] Y  (3xTF32: hi x [hi|lo] rows, lo x hi rows)
+            if (tid == 0) {
+                tc_fence_after();
+                const uint64_t ah = sw128_desc(st + L::oOp + kOpHi, 0, 64), al = sw128_desc(st + L::oOp + kOpLo, 0, 64);
+                const uint64_t b = sw128_desc(sbase + L::oBY, 0, 2 * MS);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t oa = sw128_ks_off(ks, 64), ob = sw128_ks_off(ks, 2 * MS);
+                    mma_tf32(tD2, ah + oa, b + ob, idB2, ks > 0);
+                    mma_tf32(tD2, al + oa, b + ob, idB1, 1);
+                }
+                mma_commit(bar_b);
+                if (!mbar_wait(bar_b, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
+            }
+            named_bar(2, 128);
+            if (*abort_flag) { aborted = true; break; }
+            tc_fence_after();
+            {
+                float u[MS], ul[MS];
+                tmem_ld<MS>(tD2 + lane_base, u);
+                tmem_ld<MS>(tD2 + lane_base + MS, ul);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < MS; ++i) u[i] += ul[i];
+                if (warp < 2) {
+                    // U~ = diag(delta) U -> three bf16 parts, B operand of MMA_c (rows part*MS + i,
+                    // K index = token); token lanes pair up (xor 1) to write two tokens per store
+                    if (lane < 16) {
+#pragma unroll
+                        for (int i = 0; i < MS; i += 2) {
+                            uint32_t a1, a2, a3, b1, b2, b3;
+                            bf16_split3(del * u[i], a1, a2, a3);
+                            bf16_split3(del * u[i + 1], b1, b2, b3);
+                            const uint32_t s1 = odd ? a1 : b1, s2 = odd ? a2 : b2, s3 = odd ? a3 : b3;
+                            const uint32_t t1 = __shfl_xor_sync(0x0000ffffu, s1, 1);
+                            const uint32_t t2 = __shfl_xor_sync(0x0000ffffu, s2, 1);
+                            const uint32_t t3 = __shfl_xor_sync(0x0000ffffu, s3, 1);
+                            const int row = odd ? i + 1 : i;
+                            const int kt = tok & ~1;
+                            const uint32_t w1 = odd ? (t1 | (b1 << 16)) : (a1 | (t1 << 16));
+                            const uint32_t w2 = odd ? (t2 | (b2 << 16)) : (a2 | (t2 << 16));
+                            const uint32_t w3 = odd ? (t3 | (b3 << 16)) : (a3 | (t3 << 16));
+                            asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBU + sw128_off_h(row, kt, 3 * MS)), "r"(w1));
+                            asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBU + sw128_off_h(MS + row, kt, 3 * MS)), "r"(w2));
+                            asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBU + sw128_off_h(2 * MS + row, kt, 3 * MS)), "r"(w3));
+                        }
+                    }
+                    fence_async_smem();
+                } else if (lane < 16 && tok < Lr) {
+                    // O = s (diag(Gamma) Z + P U)
+                    float o[MS];
+#pragma unroll
+                    for (int i = 0; i < MS; ++i) o[i] = scale * fmaf(Gam, za[i], u[i]);
+                    store_row<MS>(out + ((size_t)(t0 + tok) * H + h) * DV + r0, o);
+                }
+            }
+            tc_fence_before();
+            named_bar(2, 128);
+            // ---- MMA_c: dS^T = K^T U~  (K^T read M-major from the K rows; frees the stage)
+            if (tid == 0) {
+                tc_fence_after();
+                const uint64_t a = sw128_desc_mn(st + L::oAKQ, 8192, 1024);
+                const uint64_t b = sw128_desc(sbase + L::oBU, 0, 3 * MS);
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+                    mma_bf16(tD3, a + (uint64_t)(ks * 128), b + sw128_ks_off(ks, 3 * MS), idC, ks > 0);
+                mma_commit(bar_c);
+                mma_commit(&empty[s]);
+                if (!mbar_wait(bar_c, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
+            }
+            named_bar(2, 128);
+            if (*abort_flag) { aborted = true; break; }
+            tc_fence_after();
+            {
+                // S' = Gamma_31 S + dS (row c_own of dS^T; for dk = 64 the M=64 layout puts row
+                // 16w+t in lane 32w+t, which is c_own of that lane)
+                float d1[MS], d2[MS], d3[MS];
+                tmem_ld<MS>(tD3 + lane_base, d1);
+                tmem_ld<MS>(tD3 + lane_base + MS, d2);
+                tmem_ld<MS>(tD3 + lane_base + 2 * MS, d3);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < MS; ++i) S[i] = fmaf(GamC, S[i], (d1[i] + d2[i]) + d3[i]);
+            }
+            tc_fence_before();
+        }
+        if (state_out && owns && !aborted) {
+#pragma unroll
+            for (int i = 0; i < MS; ++i) state_out[(((size_t)n * H + h) * DV + r0 + i) * DK + c_own] = S[i];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *abort_flag) {
+        // after a timeout, give copies and MMAs still in flight a bounded time to finish
+        mma_commit(bar_drain);
+        volatile int never = 0;
+        mbar_wait(bar_drain, 0, &never, 100000000ull);
+    }
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+}  // namespace gdn

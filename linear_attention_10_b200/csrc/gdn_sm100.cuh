@@ -65,6 +65,40 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Adds `bytes` to the transaction count of the current phase without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// ------------------------------------------------------------------------------------------------
+// Bulk copies into this CTA's shared memory (the tensor-memory-access engine; no multicast).
+// ------------------------------------------------------------------------------------------------
+// 2-D tiled load described by a tensor map (a __grid_constant__ kernel parameter); completes `bar`
+// by the tile's byte count.  x must be a multiple of 16 bytes / element size.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+// Contiguous copy; src, dst 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // ------------------------------------------------------------------------------------------------
 // fences and named barriers
 // ------------------------------------------------------------------------------------------------
@@ -104,6 +138,18 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem], kind::f16 with bf16 operands and fp32 accumulation.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -183,6 +229,33 @@ __host__ __device__ constexpr uint64_t sw128_ks_off(int ks, int R)
     return (uint64_t)((ks >> 2) * (R * 8) + (ks & 3) * 2);
 }
 
+// Same layout with 16-bit elements: 64 elements per 128-byte row.
+__device__ __forceinline__ uint32_t sw128_off_h(int r, int k, int R)
+{
+    return (uint32_t)((k >> 6) * (R * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
+                      ((((k & 63) >> 3) ^ (r & 7)) << 4) + ((k & 7) << 1));
+}
+
+// Descriptor of a tile read M/N-major (the M index runs along the 128-byte rows): 8-row groups of
+// the K index are `sbo` bytes apart, 64-element blocks of the M index `lbo` bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t addr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+
+// Instruction descriptor: kind::f16 with bf16 A and B, fp32 accumulator; A K-major or M-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_m_major = false)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_m_major ? 1u : 0u) << 15) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
 // Instruction descriptor: kind::tf32, fp32 accumulator, both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N)
 {
@@ -197,6 +270,21 @@ __device__ __forceinline__ void tf32_split(float x, float& hi, float& lo)
 {
     hi = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
     lo = x - hi;
+}
+
+// Three-way bf16 split x = b1 + b2 + b3 (bit patterns returned in the low 16 bits): each part keeps
+// the leading 8 significant bits of what the previous parts left, so b1 + b2 + b3 carries 24
+// significant bits -- fp32 precision.  With an operand that is exactly bf16, the three products
+// on bf16 tensor cores give an fp32-accurate product.
+__device__ __forceinline__ void bf16_split3(float x, uint32_t& b1, uint32_t& b2, uint32_t& b3)
+{
+    const uint32_t u1 = __float_as_uint(x) & 0xFFFF0000u;
+    const float r1 = x - __uint_as_float(u1);
+    const uint32_t u2 = __float_as_uint(r1) & 0xFFFF0000u;
+    const float r2 = r1 - __uint_as_float(u2);
+    b1 = u1 >> 16;
+    b2 = u2 >> 16;
+    b3 = __float_as_uint(r2) >> 16;
 }
 
 }  // namespace sm100
