@@ -209,7 +209,7 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
             return GDN_ERR_LAUNCH;
         {
             ProfScope prof("gdn_scan_bf16_kernel", st);
-            kb<<<dim3((unsigned)N, H, DV / MSB), 256, SB::kBytes, st>>>(
+            kb<<<dim3((unsigned)N, H, DV / MSB), 288, SB::kBytes, st>>>(
                 tq, tk, tv, meta, chunk_off, chunk_tab, reinterpret_cast<const uint8_t*>(op), state_in,
                 static_cast<__nv_bfloat16*>(out), state_out, H, status);
         }

@@ -178,9 +178,12 @@ __device__ __forceinline__ void tc_abort(int* status, volatile int* abort_flag)
     }
 }
 
-// Optional phase-timing hook of the scan kernel (compiled out unless a build defines it).
+// Optional phase-timing hooks (compiled out unless a build defines them).
 #ifndef GDN_SCAN_TRACE
 #define GDN_SCAN_TRACE(chunk, slot)
+#endif
+#ifndef GDN_PREP_TRACE
+#define GDN_PREP_TRACE(iter, slot)
 #endif
 
 // Synchronisation rule of both kernels: exactly one thread performs each bounded mbarrier wait and
@@ -284,6 +287,7 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, 
     if ((int)blockIdx.x < nitems) load_item(cur, blockIdx.x);
 
     for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++iter) {
+        GDN_PREP_TRACE(iter, 0);
         if (item + (int)gridDim.x < nitems) load_item(nxt, item + gridDim.x);
         const int gc = cur.gc, h = cur.h;
 
@@ -308,6 +312,7 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, 
         }
         fence_async_smem();
         __syncthreads();
+        GDN_PREP_TRACE(iter, 1);
 
         // Gram matrices on the tensor cores: D[r][n] = [K;Q]_r . K_n  (M=64, N=32, K=DK)
         if (tid == 0) {
@@ -326,6 +331,7 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, 
             if (!mbar_wait(bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
         }
         __syncthreads();
+        GDN_PREP_TRACE(iter, 2);
         if (*abort_flag) break;
         tc_fence_after();
         {
@@ -341,6 +347,7 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, 
         }
         tc_fence_before();
         __syncthreads();
+        GDN_PREP_TRACE(iter, 3);
 
         // gates: A (strictly lower) and P (lower incl. diagonal)
         for (int idx = tid; idx < C * C; idx += 128) {
@@ -350,6 +357,7 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, 
             P[i * L::LD + j] = dd * P[i * L::LD + j];
         }
         __syncthreads();
+        GDN_PREP_TRACE(iter, 4);
         // T = (I + A)^-1 by forward substitution, one lane per column j of T with the column in
         // registers.  Column-oriented: once t[i] is final it is subtracted, times column i of A,
         // from every later row, so each of the 31 steps is a set of independent FMAs.
@@ -369,6 +377,7 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, 
             for (int i = 0; i < 32; ++i) Tm[i * L::LD + j] = t[i] * bj;
         }
         __syncthreads();
+        GDN_PREP_TRACE(iter, 5);
         // operator record: [T''; P T''] split into TF32 hi/lo in the swizzled image, and the gates
         uint8_t* dst = reinterpret_cast<uint8_t*>(op) + ((size_t)gc * H + h) * kOpBytes;
         for (int idx = tid; idx < 64 * 32; idx += 128) {
@@ -398,6 +407,7 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, 
             gt[tid] = val;
         }
         __syncthreads();
+        GDN_PREP_TRACE(iter, 6);
         cur = nxt;
     }
     tc_fence_before();

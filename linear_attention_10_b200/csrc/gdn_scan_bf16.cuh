@@ -51,7 +51,7 @@ struct ScanBf16Smem {
 };
 
 template <int DK, int DV, int MS, int STAGES>
-__global__ void __launch_bounds__(256, 1) gdn_scan_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
+__global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                                const __grid_constant__ CUtensorMap tm_k,
                                                                const __grid_constant__ CUtensorMap tm_v,
                                                                const int* __restrict__ meta,
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(256, 1) gdn_scan_bf16_kernel(const __grid_cons
     // accumulators: D1 [X;Z] 3MS columns, D2 [U;PU] 2MS columns, D3 dS^T 3MS columns
     const uint32_t tD1 = tmem, tD2 = tmem + 96, tD3 = tmem + 160;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------------------------ producer (one thread)
         if (lane == 0) {
             for (int cl = 0; cl < nch; ++cl) {
@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(256, 1) gdn_scan_bf16_kernel(const __grid_cons
                 const uint32_t st = sbase + s * L::kStage;
                 const int t0 = (int)(seq_t0 + (int64_t)cl * kChunk);
                 const int gc = c_begin + cl;
+                GDN_SCAN_TRACE(cl, 11);
                 mbar_arrive_expect_tx(&full[s], L::kStageTx);
 #pragma unroll
                 for (int p = 0; p < NP; ++p) {
@@ -138,57 +139,60 @@ __global__ void __launch_bounds__(256, 1) gdn_scan_bf16_kernel(const __grid_cons
                 tma_load_2d(st + L::oV, &tm_v, h * DV + r0, t0, &full[s]);
             }
         }
-    } else if (warp < 4) {
-        // ------------------------------------------------------------------ consumers
-        // thread (warp, lane) owns column c of the state slice: S[0..MS)[c]
-        const int c_own = (DK == 128) ? (warp * 32 + lane) : (warp * 16 + lane);
-        const bool owns = (DK == 128) || (lane < 16);
+    } else {
+        // ------------------------------------------------------------------ consumers (8 warps)
+        // Every product is issued with M = 128 (same cost as M = 64), so an accumulator row r sits
+        // in TMEM lane r: warp w reads lane quarter q4 = w % 4, and the two warps of a quarter
+        // (w and w + 4) split the columns: this thread handles the MH columns [hf*MH, hf*MH + MH)
+        // of each column block.
+        constexpr int MH = MS / 2;
+        const int q4 = warp & 3, hf = warp >> 2;
+        // state: this thread holds S[hf*MH + ii][c_own], ii < MH (column c_own = TMEM lane of dS^T)
+        const int c_own = q4 * 32 + lane;
+        const bool owns = c_own < DK;
         const int odd = lane & 1;
-        float S[MS];
+        float S[MH];
 #pragma unroll
-        for (int i = 0; i < MS; ++i)
-            S[i] = (state_in && owns) ? state_in[(((size_t)n * H + h) * DV + r0 + i) * DK + c_own] : 0.f;
+        for (int ii = 0; ii < MH; ++ii)
+            S[ii] = (state_in && owns) ? state_in[(((size_t)n * H + h) * DV + r0 + hf * MH + ii) * DK + c_own] : 0.f;
 
         const float scale = rsqrtf((float)DK);
-        constexpr uint32_t idA = idesc_bf16(64, 3 * MS);
-        constexpr uint32_t idB1 = idesc_tf32(64, MS), idB2 = idesc_tf32(64, 2 * MS);
-        constexpr uint32_t idC = idesc_bf16(DK, 3 * MS, true);
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const int row16 = warp * 16 + lane;          // accumulator row of an M=64 product in this lane
-        const int tok = (warp < 2) ? row16 : (row16 - 32);
+        constexpr uint32_t idA = idesc_bf16(128, 3 * MS);
+        constexpr uint32_t idB1 = idesc_tf32(128, MS), idB2 = idesc_tf32(128, 2 * MS);
+        constexpr uint32_t idC = idesc_bf16(128, 3 * MS, true);
+        const uint32_t lane_q = (uint32_t)(q4 * 32) << 16;
         bool aborted = false;
 
         for (int cl = 0; cl <= nch; ++cl) {
+            GDN_SCAN_TRACE(cl, 0);
             // S -> three bf16 parts, B operand of MMA_a (rows: part * MS + i, K index: c_own).
             // Lanes pair up (xor 1) so that every store writes two adjacent columns of one row.
-            {
-                // all lanes take part in the exchange; only lanes that own a column store
 #pragma unroll
-                for (int i = 0; i < MS; i += 2) {
-                    uint32_t a1, a2, a3, b1, b2, b3;
-                    bf16_split3(S[i], a1, a2, a3);       // row i
-                    bf16_split3(S[i + 1], b1, b2, b3);   // row i + 1
-                    // even lane keeps row i and sends its row-(i+1) parts; odd lane the reverse
-                    const uint32_t s1 = odd ? a1 : b1, s2 = odd ? a2 : b2, s3 = odd ? a3 : b3;
-                    const uint32_t t1 = __shfl_xor_sync(0xffffffffu, s1, 1);
-                    const uint32_t t2 = __shfl_xor_sync(0xffffffffu, s2, 1);
-                    const uint32_t t3 = __shfl_xor_sync(0xffffffffu, s3, 1);
-                    const int row = odd ? i + 1 : i;
-                    const int kc = c_own & ~1;
-                    const uint32_t w1 = odd ? (t1 | (b1 << 16)) : (a1 | (t1 << 16));
-                    const uint32_t w2 = odd ? (t2 | (b2 << 16)) : (a2 | (t2 << 16));
-                    const uint32_t w3 = odd ? (t3 | (b3 << 16)) : (a3 | (t3 << 16));
-                    if (owns) {
-                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBS + sw128_off_h(row, kc, 3 * MS)), "r"(w1));
-                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBS + sw128_off_h(MS + row, kc, 3 * MS)), "r"(w2));
-                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBS + sw128_off_h(2 * MS + row, kc, 3 * MS)), "r"(w3));
-                    }
+            for (int ii = 0; ii < MH; ii += 2) {
+                uint32_t a1, a2, a3, b1, b2, b3;
+                bf16_split3(S[ii], a1, a2, a3);
+                bf16_split3(S[ii + 1], b1, b2, b3);
+                const uint32_t t1 = __shfl_xor_sync(0xffffffffu, odd ? a1 : b1, 1);
+                const uint32_t t2 = __shfl_xor_sync(0xffffffffu, odd ? a2 : b2, 1);
+                const uint32_t t3 = __shfl_xor_sync(0xffffffffu, odd ? a3 : b3, 1);
+                const int row = hf * MH + (odd ? ii + 1 : ii);
+                const int kc = c_own & ~1;
+                if (owns) {
+                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBS + sw128_off_h(row, kc, 3 * MS)),
+                                 "r"(odd ? (t1 | (b1 << 16)) : (a1 | (t1 << 16))));
+                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBS + sw128_off_h(MS + row, kc, 3 * MS)),
+                                 "r"(odd ? (t2 | (b2 << 16)) : (a2 | (t2 << 16))));
+                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBS + sw128_off_h(2 * MS + row, kc, 3 * MS)),
+                                 "r"(odd ? (t3 | (b3 << 16)) : (a3 | (t3 << 16))));
                 }
             }
             if (cl == nch) break;
+            GDN_SCAN_TRACE(cl, 10);
             fence_async_smem();
+            GDN_SCAN_TRACE(cl, 12);
             tc_fence_before();
-            named_bar(2, 128);      // every column of S written before MMA_a reads it
+            named_bar(2, 256);      // every column of S written before MMA_a reads it
+            GDN_SCAN_TRACE(cl, 1);
             const int s = cl % STAGES;
             const uint32_t st = sbase + s * L::kStage;
             const uint8_t* stp = sm + s * L::kStage;
@@ -198,6 +202,7 @@ __global__ void __launch_bounds__(256, 1) gdn_scan_bf16_kernel(const __grid_cons
                 if (!mbar_wait(&full[s], (uint32_t)(cl / STAGES) & 1u, abort_flag)) {
                     tc_abort(status, abort_flag);
                 } else {
+                    GDN_SCAN_TRACE(cl, 2);
                     tc_fence_after();
                     const uint64_t a = sw128_desc(st + L::oAKQ, 0, 64);
                     const uint64_t b = sw128_desc(sbase + L::oBS, 0, 3 * MS);
@@ -205,59 +210,64 @@ __global__ void __launch_bounds__(256, 1) gdn_scan_bf16_kernel(const __grid_cons
                     for (int ks = 0; ks < DK / 16; ++ks)
                         mma_bf16(tD1, a + sw128_ks_off(ks, 64), b + sw128_ks_off(ks, 3 * MS), idA, ks > 0);
                     mma_commit(bar_a);
+                    GDN_SCAN_TRACE(cl, 3);
                     if (!mbar_wait(bar_a, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
+                    GDN_SCAN_TRACE(cl, 4);
                 }
             }
-            named_bar(2, 128);
+            named_bar(2, 256);
+            GDN_SCAN_TRACE(cl, 13);
             if (*abort_flag) { aborted = true; break; }
             tc_fence_after();
             const int64_t t0 = seq_t0 + (int64_t)cl * kChunk;
             const int Lr = (int)((seq_end - t0) < kChunk ? (seq_end - t0) : kChunk);
             const float* gate = reinterpret_cast<const float*>(stp + L::oOp + kOpGate);
-            const float Gam = (lane < 16) ? gate[tok] : 0.f;
-            const float del = (lane < 16 && warp < 2) ? gate[32 + tok] : 0.f;
+            const float Gam = gate[lane];           // token `lane` (quarters 0 and 1)
+            const float del = gate[32 + lane];
             const float GamC = gate[64];
-            float za[MS];
-            {
-                float x1[MS], x2[MS], x3[MS];
-                tmem_ld<MS>(tD1 + lane_base, x1);
-                tmem_ld<MS>(tD1 + lane_base + MS, x2);
-                tmem_ld<MS>(tD1 + lane_base + 2 * MS, x3);
+            float za[MH];
+            if (q4 < 2) {
+                // quarter 0: X rows (token = lane), quarter 1: Z rows (token = lane)
+                float x1[MH], x2[MH], x3[MH];
+                tmem_ld<MH>(tD1 + lane_q + hf * MH, x1);
+                tmem_ld<MH>(tD1 + lane_q + MS + hf * MH, x2);
+                tmem_ld<MH>(tD1 + lane_q + 2 * MS + hf * MH, x3);
                 tmem_ld_wait();
+                GDN_SCAN_TRACE(cl, 14);
 #pragma unroll
-                for (int i = 0; i < MS; ++i) za[i] = x1[i] + x2[i] + x3[i];
+                for (int i = 0; i < MH; ++i) za[i] = (x1[i] + x2[i]) + x3[i];
             }
-            if (warp < 2) {
-                // Y = V - diag(Gamma) X (zero for rows past the sequence end) -> tf32 hi/lo rows of MMA_b's B
-                if (lane < 16) {
-                    float vt[MS];
-                    const uint4* vrow = reinterpret_cast<const uint4*>(stp + L::oV + tok * MS * 2);
+            if (q4 == 0) {
+                // Y = V - diag(Gamma) X (zero past the sequence end) -> tf32 hi/lo rows of MMA_b's B
+                float vt[MH];
+                const uint4* vrow = reinterpret_cast<const uint4*>(stp + L::oV + lane * MS * 2 + hf * MH * 2);
 #pragma unroll
-                    for (int q4 = 0; q4 < MS / 8; ++q4) {
-                        const uint4 u = vrow[q4];
-                        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
+                for (int q8 = 0; q8 < MH / 8; ++q8) {
+                    const uint4 u = vrow[q8];
+                    const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = __bfloat1622float2(hv[e]);
-                            vt[q4 * 8 + 2 * e] = f.x;
-                            vt[q4 * 8 + 2 * e + 1] = f.y;
-                        }
-                    }
-                    const bool live = tok < Lr;
-#pragma unroll
-                    for (int i = 0; i < MS; ++i) {
-                        float hi, lo;
-                        tf32_split(live ? vt[i] - Gam * za[i] : 0.f, hi, lo);
-                        sts1(sbase + L::oBY, sw128_off(i, tok, 2 * MS), hi);
-                        sts1(sbase + L::oBY, sw128_off(MS + i, tok, 2 * MS), lo);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(hv[e]);
+                        vt[q8 * 8 + 2 * e] = f.x;
+                        vt[q8 * 8 + 2 * e + 1] = f.y;
                     }
                 }
+                const bool live = lane < Lr;
+#pragma unroll
+                for (int i = 0; i < MH; ++i) {
+                    float hi, lo;
+                    tf32_split(live ? vt[i] - Gam * za[i] : 0.f, hi, lo);
+                    sts1(sbase + L::oBY, sw128_off(hf * MH + i, lane, 2 * MS), hi);
+                    sts1(sbase + L::oBY, sw128_off(MS + hf * MH + i, lane, 2 * MS), lo);
+                }
+                GDN_SCAN_TRACE(cl, 15);
                 fence_async_smem();
             }
             tc_fence_before();
-            named_bar(2, 128);
+            named_bar(2, 256);
             // ---- MMA_b: [U; PU] = [T''; PT''] Y  (3xTF32: hi x [hi|lo] rows, lo x hi rows)
             if (tid == 0) {
+                GDN_SCAN_TRACE(cl, 5);
                 tc_fence_after();
                 const uint64_t ah = sw128_desc(st + L::oOp + kOpHi, 0, 64), al = sw128_desc(st + L::oOp + kOpLo, 0, 64);
                 const uint64_t b = sw128_desc(sbase + L::oBY, 0, 2 * MS);
@@ -269,53 +279,52 @@ __global__ void __launch_bounds__(256, 1) gdn_scan_bf16_kernel(const __grid_cons
                 }
                 mma_commit(bar_b);
                 if (!mbar_wait(bar_b, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
+                GDN_SCAN_TRACE(cl, 6);
             }
-            named_bar(2, 128);
+            named_bar(2, 256);
             if (*abort_flag) { aborted = true; break; }
             tc_fence_after();
-            {
-                float u[MS], ul[MS];
-                tmem_ld<MS>(tD2 + lane_base, u);
-                tmem_ld<MS>(tD2 + lane_base + MS, ul);
+            if (q4 < 2) {
+                float u[MH], ul[MH];
+                tmem_ld<MH>(tD2 + lane_q + hf * MH, u);
+                tmem_ld<MH>(tD2 + lane_q + MS + hf * MH, ul);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < MS; ++i) u[i] += ul[i];
-                if (warp < 2) {
+                for (int i = 0; i < MH; ++i) u[i] += ul[i];
+                if (q4 == 0) {
                     // U~ = diag(delta) U -> three bf16 parts, B operand of MMA_c (rows part*MS + i,
-                    // K index = token); token lanes pair up (xor 1) to write two tokens per store
-                    if (lane < 16) {
+                    // K index = token = lane); token lanes pair up to write two tokens per store
 #pragma unroll
-                        for (int i = 0; i < MS; i += 2) {
-                            uint32_t a1, a2, a3, b1, b2, b3;
-                            bf16_split3(del * u[i], a1, a2, a3);
-                            bf16_split3(del * u[i + 1], b1, b2, b3);
-                            const uint32_t s1 = odd ? a1 : b1, s2 = odd ? a2 : b2, s3 = odd ? a3 : b3;
-                            const uint32_t t1 = __shfl_xor_sync(0x0000ffffu, s1, 1);
-                            const uint32_t t2 = __shfl_xor_sync(0x0000ffffu, s2, 1);
-                            const uint32_t t3 = __shfl_xor_sync(0x0000ffffu, s3, 1);
-                            const int row = odd ? i + 1 : i;
-                            const int kt = tok & ~1;
-                            const uint32_t w1 = odd ? (t1 | (b1 << 16)) : (a1 | (t1 << 16));
-                            const uint32_t w2 = odd ? (t2 | (b2 << 16)) : (a2 | (t2 << 16));
-                            const uint32_t w3 = odd ? (t3 | (b3 << 16)) : (a3 | (t3 << 16));
-                            asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBU + sw128_off_h(row, kt, 3 * MS)), "r"(w1));
-                            asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBU + sw128_off_h(MS + row, kt, 3 * MS)), "r"(w2));
-                            asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBU + sw128_off_h(2 * MS + row, kt, 3 * MS)), "r"(w3));
-                        }
+                    for (int i = 0; i < MH; i += 2) {
+                        uint32_t a1, a2, a3, b1, b2, b3;
+                        bf16_split3(del * u[i], a1, a2, a3);
+                        bf16_split3(del * u[i + 1], b1, b2, b3);
+                        const uint32_t t1 = __shfl_xor_sync(0xffffffffu, odd ? a1 : b1, 1);
+                        const uint32_t t2 = __shfl_xor_sync(0xffffffffu, odd ? a2 : b2, 1);
+                        const uint32_t t3 = __shfl_xor_sync(0xffffffffu, odd ? a3 : b3, 1);
+                        const int row = hf * MH + (odd ? i + 1 : i);
+                        const int kt = lane & ~1;
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBU + sw128_off_h(row, kt, 3 * MS)),
+                                     "r"(odd ? (t1 | (b1 << 16)) : (a1 | (t1 << 16))));
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBU + sw128_off_h(MS + row, kt, 3 * MS)),
+                                     "r"(odd ? (t2 | (b2 << 16)) : (a2 | (t2 << 16))));
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBU + sw128_off_h(2 * MS + row, kt, 3 * MS)),
+                                     "r"(odd ? (t3 | (b3 << 16)) : (a3 | (t3 << 16))));
                     }
                     fence_async_smem();
-                } else if (lane < 16 && tok < Lr) {
-                    // O = s (diag(Gamma) Z + P U)
-                    float o[MS];
+                } else if (lane < Lr) {
+                    // O = s (diag(Gamma) Z + P U) for token `lane`, this thread's MH columns
+                    float o[MH];
 #pragma unroll
-                    for (int i = 0; i < MS; ++i) o[i] = scale * fmaf(Gam, za[i], u[i]);
-                    store_row<MS>(out + ((size_t)(t0 + tok) * H + h) * DV + r0, o);
+                    for (int i = 0; i < MH; ++i) o[i] = scale * fmaf(Gam, za[i], u[i]);
+                    store_row<MH>(out + ((size_t)(t0 + lane) * H + h) * DV + r0 + hf * MH, o);
                 }
             }
             tc_fence_before();
-            named_bar(2, 128);
+            named_bar(2, 256);
             // ---- MMA_c: dS^T = K^T U~  (K^T read M-major from the K rows; frees the stage)
             if (tid == 0) {
+                GDN_SCAN_TRACE(cl, 7);
                 tc_fence_after();
                 const uint64_t a = sw128_desc_mn(st + L::oAKQ, 8192, 1024);
                 const uint64_t b = sw128_desc(sbase + L::oBU, 0, 3 * MS);
@@ -325,26 +334,28 @@ __global__ void __launch_bounds__(256, 1) gdn_scan_bf16_kernel(const __grid_cons
                 mma_commit(bar_c);
                 mma_commit(&empty[s]);
                 if (!mbar_wait(bar_c, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
+                GDN_SCAN_TRACE(cl, 8);
             }
-            named_bar(2, 128);
+            named_bar(2, 256);
             if (*abort_flag) { aborted = true; break; }
             tc_fence_after();
             {
-                // S' = Gamma_31 S + dS (row c_own of dS^T; for dk = 64 the M=64 layout puts row
-                // 16w+t in lane 32w+t, which is c_own of that lane)
-                float d1[MS], d2[MS], d3[MS];
-                tmem_ld<MS>(tD3 + lane_base, d1);
-                tmem_ld<MS>(tD3 + lane_base + MS, d2);
-                tmem_ld<MS>(tD3 + lane_base + 2 * MS, d3);
+                // S' = Gamma_31 S + dS  (row c_own of dS^T, this thread's half of the S rows)
+                float d1[MH], d2[MH], d3[MH];
+                tmem_ld<MH>(tD3 + lane_q + hf * MH, d1);
+                tmem_ld<MH>(tD3 + lane_q + MS + hf * MH, d2);
+                tmem_ld<MH>(tD3 + lane_q + 2 * MS + hf * MH, d3);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < MS; ++i) S[i] = fmaf(GamC, S[i], (d1[i] + d2[i]) + d3[i]);
+                for (int i = 0; i < MH; ++i) S[i] = fmaf(GamC, S[i], (d1[i] + d2[i]) + d3[i]);
             }
+            GDN_SCAN_TRACE(cl, 9);
             tc_fence_before();
         }
         if (state_out && owns && !aborted) {
 #pragma unroll
-            for (int i = 0; i < MS; ++i) state_out[(((size_t)n * H + h) * DV + r0 + i) * DK + c_own] = S[i];
+            for (int ii = 0; ii < MH; ++ii)
+                state_out[(((size_t)n * H + h) * DV + r0 + hf * MH + ii) * DK + c_own] = S[ii];
         }
     }
     tc_fence_before();

@@ -186,11 +186,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32])
           "=r"(u[24]), "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
         : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&r)[8])
+{
+    uint32_t* u = reinterpret_cast<uint32_t*>(r);
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
+                 : "r"(taddr));
+}
 template <int N>
 __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&r)[N])
 {
-    static_assert(N == 16 || N == 32, "tmem_ld: 16 or 32 columns");
-    if constexpr (N == 16) tmem_ld16(taddr, r);
+    static_assert(N == 8 || N == 16 || N == 32, "tmem_ld: 8, 16 or 32 columns");
+    if constexpr (N == 8) tmem_ld8(taddr, r);
+    else if constexpr (N == 16) tmem_ld16(taddr, r);
     else tmem_ld32(taddr, r);
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
