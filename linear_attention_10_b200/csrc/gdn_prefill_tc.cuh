@@ -216,7 +216,7 @@ struct PrepSmem {
 };
 
 template <typename T, int DK>
-__global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                        const float* __restrict__ g, const float* __restrict__ beta,
                                                        const int* __restrict__ meta,
                                                        const int4* __restrict__ chunk_tab, float* __restrict__ op,
@@ -378,24 +378,31 @@ __global__ void __launch_bounds__(128) gdn_prep_kernel(const T* __restrict__ q, 
         }
         __syncthreads();
         GDN_PREP_TRACE(iter, 5);
-        // operator record: [T''; P T''] split into TF32 hi/lo in the swizzled image, and the gates
+        // operator record: [T''; P T''] split into TF32 hi/lo in the swizzled image, and the gates.
+        // Thread (row group rg, column j) keeps column j of T'' in registers and forms 8 rows of
+        // P T'' with full 32-term sums (P is zero above and T'' below the diagonal).
         uint8_t* dst = reinterpret_cast<uint8_t*>(op) + ((size_t)gc * H + h) * kOpBytes;
-        for (int idx = tid; idx < 64 * 32; idx += 128) {
-            const int i = idx >> 5, j = idx & 31;
-            float val;
-            if (i < 32) {
-                val = Tm[i * L::LD + j];
-            } else {
-                const int ii = i - 32;
+        {
+            const int j = tid & 31, rg = tid >> 5;
+            float tc[32];
+#pragma unroll
+            for (int m = 0; m < 32; ++m) tc[m] = Tm[m * L::LD + j];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int i = rg * 8 + r;
                 float acc = 0.f;
-                for (int m = j; m <= ii; ++m) acc = fmaf(P[ii * L::LD + m], Tm[m * L::LD + j], acc);
-                val = acc;
+#pragma unroll
+                for (int m = 0; m < 32; ++m) acc = fmaf(P[i * L::LD + m], tc[m], acc);
+                float hi, lo;
+                tf32_split(Tm[i * L::LD + j], hi, lo);          // row i of T''
+                uint32_t o = sw128_off(i, j, 64);
+                *reinterpret_cast<float*>(dst + kOpHi + o) = hi;
+                *reinterpret_cast<float*>(dst + kOpLo + o) = lo;
+                tf32_split(acc, hi, lo);                         // row 32 + i: (P T'')_i
+                o = sw128_off(32 + i, j, 64);
+                *reinterpret_cast<float*>(dst + kOpHi + o) = hi;
+                *reinterpret_cast<float*>(dst + kOpLo + o) = lo;
             }
-            float hi, lo;
-            tf32_split(val, hi, lo);
-            const uint32_t o = sw128_off(i, j, 64);
-            *reinterpret_cast<float*>(dst + kOpHi + o) = hi;
-            *reinterpret_cast<float*>(dst + kOpLo + o) = lo;
         }
         if (tid < 80) {
             float* gt = reinterpret_cast<float*>(dst + kOpGate);

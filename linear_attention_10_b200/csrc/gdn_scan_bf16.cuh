@@ -40,10 +40,13 @@ struct ScanBf16Smem {
     static constexpr uint32_t kStage = ((oV + 32 * MS * 2) + 1023) & ~1023u;
     static constexpr uint32_t kStageTx = NP * 2 * 4096 + kOpCopyBytes + 32 * MS * 2;
     // shared by all stages
-    static constexpr uint32_t oBS = STAGES * kStage;                  // S parts: NP panels x 3MS rows x 128 B
-    static constexpr uint32_t oBY = oBS + NP * 3 * MS * 128;          // Y hi/lo (tf32): 2MS rows x 128 B
-    static constexpr uint32_t oBU = oBY + ((2 * MS * 128 + 1023) & ~1023u);  // U~ parts (bf16): 3MS rows x 128 B
-    static constexpr uint32_t oBar = oBU + ((3 * MS * 128 + 1023) & ~1023u);
+    // B operands of the bf16 products are stored N-major (N = 3 parts x MS, two 64-wide N-blocks)
+    static constexpr uint32_t kLboS = DK * 128;                       // N-block stride of S parts
+    static constexpr uint32_t kLboU = 32 * 128;                       // N-block stride of U~ parts
+    static constexpr uint32_t oBS = STAGES * kStage;                  // S parts, N-major: 2 x DK rows x 128 B
+    static constexpr uint32_t oBY = oBS + 2 * kLboS;                  // Y hi/lo (tf32, K-major): 2MS rows x 128 B
+    static constexpr uint32_t oBU = oBY + ((2 * MS * 128 + 1023) & ~1023u);  // U~ parts, N-major: 2 x 32 rows x 128 B
+    static constexpr uint32_t oBar = oBU + 2 * kLboU;
     static constexpr uint32_t oTmem = oBar + 8 * (2 * STAGES + 4);
     static constexpr uint32_t oAbort = oTmem + 4;
     static constexpr uint32_t kTotal = oAbort + 4;
@@ -150,42 +153,39 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
         // state: this thread holds S[hf*MH + ii][c_own], ii < MH (column c_own = TMEM lane of dS^T)
         const int c_own = q4 * 32 + lane;
         const bool owns = c_own < DK;
-        const int odd = lane & 1;
         float S[MH];
 #pragma unroll
         for (int ii = 0; ii < MH; ++ii)
             S[ii] = (state_in && owns) ? state_in[(((size_t)n * H + h) * DV + r0 + hf * MH + ii) * DK + c_own] : 0.f;
 
         const float scale = rsqrtf((float)DK);
-        constexpr uint32_t idA = idesc_bf16(128, 3 * MS);
+        constexpr uint32_t idA = idesc_bf16(128, 3 * MS, false, true);
         constexpr uint32_t idB1 = idesc_tf32(128, MS), idB2 = idesc_tf32(128, 2 * MS);
-        constexpr uint32_t idC = idesc_bf16(128, 3 * MS, true);
+        constexpr uint32_t idC = idesc_bf16(128, 3 * MS, true, true);
         const uint32_t lane_q = (uint32_t)(q4 * 32) << 16;
         bool aborted = false;
 
-        for (int cl = 0; cl <= nch; ++cl) {
-            GDN_SCAN_TRACE(cl, 0);
-            // S -> three bf16 parts, B operand of MMA_a (rows: part * MS + i, K index: c_own).
-            // Lanes pair up (xor 1) so that every store writes two adjacent columns of one row.
+        // Writes this thread's MH consecutive N-values (N = part * MS + hf * MH + i) of K-row `k` of an
+        // N-major B tile as three bf16 parts: two 16-byte stores per part.
+        auto put_parts = [&](uint32_t tile, uint32_t lbo, int k, const float (&x)[MH]) {
+            uint32_t w[3][MH / 2];
 #pragma unroll
-            for (int ii = 0; ii < MH; ii += 2) {
-                uint32_t a1, a2, a3, b1, b2, b3;
-                bf16_split3(S[ii], a1, a2, a3);
-                bf16_split3(S[ii + 1], b1, b2, b3);
-                const uint32_t t1 = __shfl_xor_sync(0xffffffffu, odd ? a1 : b1, 1);
-                const uint32_t t2 = __shfl_xor_sync(0xffffffffu, odd ? a2 : b2, 1);
-                const uint32_t t3 = __shfl_xor_sync(0xffffffffu, odd ? a3 : b3, 1);
-                const int row = hf * MH + (odd ? ii + 1 : ii);
-                const int kc = c_own & ~1;
-                if (owns) {
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBS + sw128_off_h(row, kc, 3 * MS)),
-                                 "r"(odd ? (t1 | (b1 << 16)) : (a1 | (t1 << 16))));
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBS + sw128_off_h(MS + row, kc, 3 * MS)),
-                                 "r"(odd ? (t2 | (b2 << 16)) : (a2 | (t2 << 16))));
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBS + sw128_off_h(2 * MS + row, kc, 3 * MS)),
-                                 "r"(odd ? (t3 | (b3 << 16)) : (a3 | (t3 << 16))));
+            for (int i = 0; i < MH; i += 2) bf16x2_split3(x[i], x[i + 1], w[0][i / 2], w[1][i / 2], w[2][i / 2]);
+#pragma unroll
+            for (int p = 0; p < 3; ++p) {
+#pragma unroll
+                for (int g = 0; g < MH / 8; ++g) {
+                    const int n0 = p * MS + hf * MH + g * 8;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(tile + sw128_off_nmaj(n0, k, lbo)),
+                                 "r"(w[p][g * 4]), "r"(w[p][g * 4 + 1]), "r"(w[p][g * 4 + 2]), "r"(w[p][g * 4 + 3]));
                 }
             }
+        };
+
+        for (int cl = 0; cl <= nch; ++cl) {
+            GDN_SCAN_TRACE(cl, 0);
+            // S -> three bf16 parts, N-major B operand of MMA_a (N = part * MS + row, K = dk column)
+            if (owns) put_parts(sbase + L::oBS, L::kLboS, c_own, S);
             if (cl == nch) break;
             GDN_SCAN_TRACE(cl, 10);
             fence_async_smem();
@@ -205,10 +205,10 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
                     GDN_SCAN_TRACE(cl, 2);
                     tc_fence_after();
                     const uint64_t a = sw128_desc(st + L::oAKQ, 0, 64);
-                    const uint64_t b = sw128_desc(sbase + L::oBS, 0, 3 * MS);
+                    const uint64_t b = sw128_desc_mn(sbase + L::oBS, L::kLboS, 1024);
 #pragma unroll
                     for (int ks = 0; ks < DK / 16; ++ks)
-                        mma_bf16(tD1, a + sw128_ks_off(ks, 64), b + sw128_ks_off(ks, 3 * MS), idA, ks > 0);
+                        mma_bf16(tD1, a + sw128_ks_off(ks, 64), b + (uint64_t)(ks * 128), idA, ks > 0);
                     mma_commit(bar_a);
                     GDN_SCAN_TRACE(cl, 3);
                     if (!mbar_wait(bar_a, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
@@ -292,25 +292,11 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
 #pragma unroll
                 for (int i = 0; i < MH; ++i) u[i] += ul[i];
                 if (q4 == 0) {
-                    // U~ = diag(delta) U -> three bf16 parts, B operand of MMA_c (rows part*MS + i,
-                    // K index = token = lane); token lanes pair up to write two tokens per store
+                    // U~ = diag(delta) U -> three bf16 parts, N-major B operand of MMA_c
+                    // (N = part * MS + i, K = token = lane)
 #pragma unroll
-                    for (int i = 0; i < MH; i += 2) {
-                        uint32_t a1, a2, a3, b1, b2, b3;
-                        bf16_split3(del * u[i], a1, a2, a3);
-                        bf16_split3(del * u[i + 1], b1, b2, b3);
-                        const uint32_t t1 = __shfl_xor_sync(0xffffffffu, odd ? a1 : b1, 1);
-                        const uint32_t t2 = __shfl_xor_sync(0xffffffffu, odd ? a2 : b2, 1);
-                        const uint32_t t3 = __shfl_xor_sync(0xffffffffu, odd ? a3 : b3, 1);
-                        const int row = hf * MH + (odd ? i + 1 : i);
-                        const int kt = lane & ~1;
-                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBU + sw128_off_h(row, kt, 3 * MS)),
-                                     "r"(odd ? (t1 | (b1 << 16)) : (a1 | (t1 << 16))));
-                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBU + sw128_off_h(MS + row, kt, 3 * MS)),
-                                     "r"(odd ? (t2 | (b2 << 16)) : (a2 | (t2 << 16))));
-                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sbase + L::oBU + sw128_off_h(2 * MS + row, kt, 3 * MS)),
-                                     "r"(odd ? (t3 | (b3 << 16)) : (a3 | (t3 << 16))));
-                    }
+                    for (int i = 0; i < MH; ++i) u[i] *= del;
+                    put_parts(sbase + L::oBU, L::kLboU, lane, u);
                     fence_async_smem();
                 } else if (lane < Lr) {
                     // O = s (diag(Gamma) Z + P U) for token `lane`, this thread's MH columns
@@ -327,10 +313,10 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
                 GDN_SCAN_TRACE(cl, 7);
                 tc_fence_after();
                 const uint64_t a = sw128_desc_mn(st + L::oAKQ, 8192, 1024);
-                const uint64_t b = sw128_desc(sbase + L::oBU, 0, 3 * MS);
+                const uint64_t b = sw128_desc_mn(sbase + L::oBU, L::kLboU, 1024);
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks)
-                    mma_bf16(tD3, a + (uint64_t)(ks * 128), b + sw128_ks_off(ks, 3 * MS), idC, ks > 0);
+                    mma_bf16(tD3, a + (uint64_t)(ks * 128), b + (uint64_t)(ks * 128), idC, ks > 0);
                 mma_commit(bar_c);
                 mma_commit(&empty[s]);
                 if (!mbar_wait(bar_c, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);

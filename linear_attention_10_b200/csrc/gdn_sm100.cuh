@@ -3,6 +3,7 @@
 // and the shared-memory matrix descriptors of the 128-byte-swizzled K-major operand layout.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace gdn {
@@ -257,11 +258,37 @@ __device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t addr, uint32_t lbo, u
     return d;
 }
 
-// Instruction descriptor: kind::f16 with bf16 A and B, fp32 accumulator; A K-major or M-major.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_m_major = false)
+// Instruction descriptor: kind::f16 with bf16 A and B, fp32 accumulator; each operand K-major or
+// M/N-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_m_major = false, bool b_n_major = false)
 {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_m_major ? 1u : 0u) << 15) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_m_major ? 1u : 0u) << 15) | ((b_n_major ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Byte offset of element (n, k) of a 16-bit tile stored N-major with the 128-byte swizzle: N runs
+// along 128-byte rows (64 elements), one row per K index, 8 K-rows per 1024-byte group; 64-wide
+// N-blocks are `lbo` bytes apart.
+__device__ __forceinline__ uint32_t sw128_off_nmaj(int n, int k, uint32_t lbo)
+{
+    return (uint32_t)((n >> 6) * lbo + (k >> 3) * 1024 + (k & 7) * 128 + (((((n & 63) >> 3) ^ (k & 7))) << 4) +
+                      ((n & 7) << 1));
+}
+
+// Three-way bf16 split of two values at once, packed in pairs (first value in the low half), for
+// N-major tiles where the two values are adjacent along N.  Rounding to nearest at each stage;
+// every remainder is exact in fp32, so the three parts carry the value's 24 significant bits.
+__device__ __forceinline__ void bf16x2_split3(float x, float y, uint32_t& p1, uint32_t& p2, uint32_t& p3)
+{
+    __nv_bfloat162 h1 = __floats2bfloat162_rn(x, y);
+    const float2 f1 = __bfloat1622float2(h1);
+    const float rx = x - f1.x, ry = y - f1.y;
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(rx, ry);
+    const float2 f2 = __bfloat1622float2(h2);
+    __nv_bfloat162 h3 = __floats2bfloat162_rn(rx - f2.x, ry - f2.y);
+    p1 = *reinterpret_cast<uint32_t*>(&h1);
+    p2 = *reinterpret_cast<uint32_t*>(&h2);
+    p3 = *reinterpret_cast<uint32_t*>(&h3);
 }
 
 // Instruction descriptor: kind::tf32, fp32 accumulator, both operands K-major.
