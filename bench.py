@@ -59,6 +59,7 @@ KERNELS = {
     "gdn_scan_tc_kernel": dict(bound="tensor", flops_per_token_head=flops_scan(), split=3),
     "gdn_scan_bf16_kernel": dict(bound="tensor", flops_per_token_head=flops_scan(), split=3),
     "gdn_prep_kernel": dict(bound="tensor", flops_per_token_head=flops_prep(), split=3),
+    "gdn_prep_bf16_kernel": dict(bound="tensor", flops_per_token_head=flops_prep(), split=3),
     "gdn_plan_kernel": dict(bound="latency"),
     "gdn_decode_step_kernel": dict(bound="hbm"),
 }

@@ -16,6 +16,7 @@
 #include "gdn_decode.cuh"
 #include "gdn_plan.cuh"
 #include "gdn_prefill_tc.cuh"
+#include "gdn_prep_bf16.cuh"
 #include "gdn_scan_bf16.cuh"
 
 namespace gdn {
@@ -177,7 +178,29 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
     }
     if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
 
-    if (lay.nc_max > 0 && T_total > 0) {
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    CUtensorMap tq{}, tk{}, tv{};
+    if constexpr (kBf16) {
+        const uint64_t Tn = (uint64_t)(T_total > 0 ? T_total : 1);
+        if (!make_tmap_bf16(&tq, q, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, true) ||
+            !make_tmap_bf16(&tk, k, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, true) ||
+            !make_tmap_bf16(&tv, v, (uint64_t)H * DV, Tn, (uint64_t)H * DV, 32, 32, false))
+            return GDN_ERR_CUDA;
+    }
+    if constexpr (kBf16) {
+      if (lay.nc_max > 0 && T_total > 0) {
+        using PL = PrepBf16Smem<DK>;
+        auto k1 = gdn_prep_bf16_kernel<DK>;
+        if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PL::kBytes) != cudaSuccess)
+            return GDN_ERR_LAUNCH;
+        const int64_t items = lay.nc_max * (int64_t)H;
+        const int64_t cap = (int64_t)g_num_sms * 4;
+        const unsigned grid = (unsigned)(items < cap ? items : cap);
+        ProfScope prof("gdn_prep_bf16_kernel", st);
+        k1<<<grid, 128, PL::kBytes, st>>>(tq, tk, g, beta, meta, chunk_tab, reinterpret_cast<uint8_t*>(op), H, status);
+        if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
+      }
+    } else if (lay.nc_max > 0 && T_total > 0) {
         using PL = PrepSmem<T, DK>;
         auto k1 = gdn_prep_kernel<T, DK>;
         if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PL::kBytes) != cudaSuccess)
@@ -198,12 +221,7 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         constexpr int ST = (SB3::kBytes + 1024 <= 228 * 1024) ? 3 : 2;
         using SB = ScanBf16Smem<DK, MSB, ST>;
         static_assert(SB2::kBytes + 1024 <= 228 * 1024, "bf16 scan shared memory");
-        CUtensorMap tq, tk, tv;
-        const uint64_t Tn = (uint64_t)(T_total > 0 ? T_total : 1);
-        if (!make_tmap_bf16(&tq, q, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, true) ||
-            !make_tmap_bf16(&tk, k, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, true) ||
-            !make_tmap_bf16(&tv, v, (uint64_t)H * DV, Tn, (uint64_t)H * DV, MSB, 32, false))
-            return GDN_ERR_CUDA;
+        static_assert(MSB == 32, "the V tensor map boxes 32 columns");
         auto kb = gdn_scan_bf16_kernel<DK, DV, MSB, ST>;
         if (cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SB::kBytes) != cudaSuccess)
             return GDN_ERR_LAUNCH;

@@ -89,6 +89,11 @@ __device__ __forceinline__ void sts1(uint32_t base, uint32_t off, float a)
 {
     asm volatile("st.shared.f32 [%0], %1;" ::"r"(base + off), "f"(a));
 }
+// Global store with the same property (no memory clobber).
+__device__ __forceinline__ void stg1(void* p, float a)
+{
+    asm volatile("st.global.f32 [%0], %1;" ::"l"(p), "f"(a));
+}
 
 // Stores 8 consecutive K-elements (k0 % 8 == 0) of row r of a K-major SW128 tile of R rows, as hi
 // (and lo when SPLIT) parts.

@@ -1,0 +1,285 @@
+// gdn_prep_bf16.cuh -- per-(chunk, head) WY/UT operator for bf16 q/k (sm_100a).
+//
+// Builds the same record as gdn_prep_kernel (gdn_prefill_tc.cuh): the TF32 hi/lo image of
+// [T''; P T''] and the gates of one chunk of 32 rows, where (chunk-local cumulative log-gate gamma)
+//
+//   A = strictly-lower(diag(beta) (D o K K^T)),  P = lower-incl-diagonal(D o Q K^T),
+//   D_ij = exp(gamma_i - gamma_j),  T = (I + A)^-1,  T'' = T diag(beta).
+//
+// What is specific to bf16 inputs: the chunk's [K; Q] rows are exact bf16 values, so the tensor-
+// memory-access engine copies them straight into the 128-byte-swizzled operand layout (two items
+// in flight per CTA) and one bf16 tensor-core product (M = 128, N = 32, K = dk) forms both Gram
+// matrices exactly in fp32.  The gates are applied while the Gram rows come out of tensor memory.
+// The inverse uses the 2 x 2 block form with 16 x 16 blocks,
+//
+//   T11 = (I + A11)^-1,  T22 = (I + A22)^-1  (forward substitution, in parallel),
+//   T21 = -T22 (A21 T11),
+//
+// which shortens the dependent chain of the substitution from 31 steps to 15.
+#pragma once
+
+#include <cuda.h>
+
+#include "gdn_common.cuh"
+#include "gdn_prefill_tc.cuh"
+#include "gdn_sm100.cuh"
+
+namespace gdn {
+
+template <int DK>
+struct PrepBf16Smem {
+    static constexpr int NP = DK / 64;
+    static constexpr uint32_t kTile = NP * 8192;                      // [K;Q] bf16: NP panels x 64 rows x 128 B
+    static constexpr uint32_t oTile = 0;                              // two buffers
+    static constexpr int LD = 33;
+    static constexpr uint32_t oG = 2 * kTile;                         // [32][33] A
+    static constexpr uint32_t oP = oG + 32 * LD * 4;                  // [32][33] P
+    static constexpr uint32_t oT = oP + 32 * LD * 4;                  // [32][33] T
+    static constexpr uint32_t oM = oT + 32 * LD * 4;                  // [16][17] A21 T11
+    static constexpr uint32_t oGam = oM + 16 * 17 * 4;
+    static constexpr uint32_t oBet = oGam + 128;
+    static constexpr uint32_t oBar = oBet + 128;                      // tile_full[2], mma, drain
+    static constexpr uint32_t oTmem = oBar + 32;
+    static constexpr uint32_t oAbort = oTmem + 4;
+    static constexpr uint32_t kTotal = oAbort + 4;
+    static constexpr uint32_t kBytes = kTotal + 1024;
+};
+
+template <int DK>
+__global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                               const __grid_constant__ CUtensorMap tm_k,
+                                                               const float* __restrict__ g,
+                                                               const float* __restrict__ beta,
+                                                               const int* __restrict__ meta,
+                                                               const int4* __restrict__ chunk_tab,
+                                                               uint8_t* __restrict__ op, int H, int* status)
+{
+    using namespace sm100;
+    using L = PrepBf16Smem<DK>;
+    constexpr int NP = L::NP;
+    constexpr int LD = L::LD;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    float* G = reinterpret_cast<float*>(sm + L::oG);
+    float* P = reinterpret_cast<float*>(sm + L::oP);
+    float* Tm = reinterpret_cast<float*>(sm + L::oT);
+    float* M1 = reinterpret_cast<float*>(sm + L::oM);
+    float* gam = reinterpret_cast<float*>(sm + L::oGam);
+    float* bet = reinterpret_cast<float*>(sm + L::oBet);
+    uint64_t* tile_full = reinterpret_cast<uint64_t*>(sm + L::oBar);
+    uint64_t* mma_bar = tile_full + 2;
+    uint64_t* drain = tile_full + 3;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::oTmem);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::oAbort);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nitems = meta[0] * H;
+    if (tid == 0) {
+        mbar_init(&tile_full[0], 1);
+        mbar_init(&tile_full[1], 1);
+        mbar_init(mma_bar, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tslot, 32);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+
+    // copies the [K; Q] rows of one item into tile buffer `b` (thread 0 only)
+    auto issue_tile = [&](int item, int b) {
+        const int gc = item / H, h = item % H;
+        const int t0 = chunk_tab[gc].y;
+        const uint32_t dst = sbase + L::oTile + b * L::kTile;
+        mbar_arrive_expect_tx(&tile_full[b], NP * 2 * 4096);
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            tma_load_2d(dst + p * 8192, &tm_k, h * DK + p * 64, t0, &tile_full[b]);
+            tma_load_2d(dst + p * 8192 + 4096, &tm_q, h * DK + p * 64, t0, &tile_full[b]);
+        }
+    };
+    // gate inputs of one item (lanes of warp 2; zero past the chunk's rows)
+    auto load_gates = [&](int item, float& gv, float& bv) {
+        const int gc = item / H, h = item % H;
+        const int4 ct = chunk_tab[gc];
+        const bool ok = lane < ct.z;
+        gv = ok ? __ldg(g + (size_t)(ct.y + lane) * H + h) : 0.f;
+        bv = ok ? __ldg(beta + (size_t)(ct.y + lane) * H + h) : 0.f;
+    };
+
+    if (tid == 0) {
+        if ((int)blockIdx.x < nitems) issue_tile(blockIdx.x, 0);
+        if ((int)(blockIdx.x + gridDim.x) < nitems) issue_tile(blockIdx.x + gridDim.x, 1);
+    }
+    float gv_cur = 0.f, bv_cur = 0.f;
+    if (warp == 2 && (int)blockIdx.x < nitems) load_gates(blockIdx.x, gv_cur, bv_cur);
+
+    constexpr uint32_t idG = idesc_bf16(128, 32);
+    uint32_t iter = 0;
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++iter) {
+        GDN_PREP_TRACE(iter, 0);
+        const int b = iter & 1;
+        const int gc = item / H, h = item % H;
+        const int Lr = chunk_tab[gc].z;
+
+        // Gram products D[r][n] = [K; Q]_r . K_n on the tensor cores (rows 64..127 unused)
+        if (tid == 0) {
+            if (!mbar_wait(&tile_full[b], (iter >> 1) & 1u, abort_flag)) {
+                tc_abort(status, abort_flag);
+            } else {
+                tc_fence_after();
+                const uint64_t a = sw128_desc(sbase + L::oTile + b * L::kTile, 0, 64);
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks) {
+                    const uint64_t o = sw128_ks_off(ks, 64);
+                    mma_bf16(tmem, a + o, a + o, idG, ks > 0);
+                }
+                mma_commit(mma_bar);
+                if (!mbar_wait(mma_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
+                // the tile buffer is free again: fetch the item after next into it
+                else if (item + 2 * (int)gridDim.x < nitems) issue_tile(item + 2 * gridDim.x, b);
+            }
+        }
+        if (warp == 2) {
+            // local cumulative log-gate and beta of this item; then prefetch the next item's
+            float gv = gv_cur;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, gv, o);
+                if (lane >= o) gv += y;
+            }
+            gam[lane] = gv * 1.4426950408889634f;    // log2(e) * gamma: gates become exp2 of differences
+            bet[lane] = bv_cur;
+            if (item + (int)gridDim.x < nitems) load_gates(item + gridDim.x, gv_cur, bv_cur);
+        }
+        __syncthreads();
+        GDN_PREP_TRACE(iter, 1);
+        if (*abort_flag) break;
+        tc_fence_after();
+        if (warp < 2) {
+            // lane r of warp 0: row r of K K^T -> A;  lane r of warp 1: row r of Q K^T -> P
+            float d[32];
+            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), d);
+            tmem_ld_wait();
+            GDN_PREP_TRACE(iter, 5);
+            const int r = lane;
+            float gj[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) gj[j] = gam[j];
+            const float gr = gam[r], br = bet[r];
+            const uint32_t dst = sbase + ((warp == 0) ? L::oG : L::oP) + (uint32_t)(r * LD * 4);
+            const float wr = (warp == 0) ? br : 1.f;
+            const int lim = (warp == 0) ? r : r + 1;      // strictly lower for A, incl. diagonal for P
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sts1(dst, (uint32_t)(j * 4), (j < lim) ? wr * exp2f(gr - gj[j]) * d[j] : 0.f);
+            GDN_PREP_TRACE(iter, 6);
+        }
+        tc_fence_before();
+        __syncthreads();
+        GDN_PREP_TRACE(iter, 2);
+
+        // T11 (lanes 0..15, column j) and T22 (lanes 16..31, column j - 16) by forward substitution
+        if (warp == 0) {
+            const int blk = lane >> 4, j = lane & 15, o = blk * 16;
+            float t[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) t[r] = (r == j) ? 1.f : 0.f;
+#pragma unroll
+            for (int i = 0; i < 15; ++i) {
+#pragma unroll
+                for (int r = i + 1; r < 16; ++r) t[r] = fmaf(-G[(o + r) * LD + o + i], t[i], t[r]);
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                Tm[(o + r) * LD + o + j] = t[r];
+                Tm[(o + r) * LD + (16 - o) + j] = 0.f;   // upper-right block (overwritten below for blk 1)
+            }
+        }
+        __syncthreads();
+        {
+            // M1 = A21 T11 (16 x 16): two outputs per thread
+            const int r = tid >> 3, c = (tid & 7) * 2;
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const float am = G[(16 + r) * LD + m];
+                a0 = fmaf(am, Tm[m * LD + c], a0);
+                a1 = fmaf(am, Tm[m * LD + c + 1], a1);
+            }
+            M1[r * 17 + c] = a0;
+            M1[r * 17 + c + 1] = a1;
+        }
+        __syncthreads();
+        {
+            // T21 = -T22 M1
+            const int r = tid >> 3, c = (tid & 7) * 2;
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const float tm = Tm[(16 + r) * LD + 16 + m];
+                a0 = fmaf(tm, M1[m * 17 + c], a0);
+                a1 = fmaf(tm, M1[m * 17 + c + 1], a1);
+            }
+            Tm[(16 + r) * LD + c] = -a0;
+            Tm[(16 + r) * LD + c + 1] = -a1;
+        }
+        __syncthreads();
+        GDN_PREP_TRACE(iter, 3);
+
+        // operator record: rows i of T'' = T diag(beta) and of P T'', TF32 hi/lo, swizzled image
+        uint8_t* dst = op + ((size_t)gc * H + h) * kOpBytes;
+        {
+            const int j = lane, rg = warp;
+            const float bj = bet[j];
+            float tc[32];
+#pragma unroll
+            for (int m = 0; m < 32; ++m) tc[m] = Tm[m * LD + j] * bj;
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+                const int i = rg * 8 + rr;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < 32; ++m) acc = fmaf(P[i * LD + m], tc[m], acc);
+                float hi, lo;
+                tf32_split(Tm[i * LD + j] * bj, hi, lo);
+                uint32_t o = sw128_off(i, j, 64);
+                stg1(dst + kOpHi + o, hi);
+                stg1(dst + kOpLo + o, lo);
+                tf32_split(acc, hi, lo);
+                o = sw128_off(32 + i, j, 64);
+                stg1(dst + kOpHi + o, hi);
+                stg1(dst + kOpLo + o, lo);
+            }
+        }
+        if (tid < 80) {
+            float* gt = reinterpret_cast<float*>(dst + kOpGate);
+            const float gl = gam[31];
+            float val = 0.f;
+            if (tid < 32) val = exp2f(gam[tid]);
+            else if (tid < 64) val = exp2f(gl - gam[tid - 32]);
+            else if (tid == 64) val = exp2f(gl);
+            gt[tid] = val;
+        }
+        (void)Lr;
+        __syncthreads();
+        GDN_PREP_TRACE(iter, 4);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *abort_flag) {
+        // after a timeout, give copies and an MMA still in flight a bounded time to finish
+        mma_commit(drain);
+        volatile int never = 0;
+        mbar_wait(drain, 0, &never, 100000000ull);
+    }
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 32);
+}
+
+}  // namespace gdn
