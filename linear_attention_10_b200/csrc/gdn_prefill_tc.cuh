@@ -49,6 +49,10 @@ constexpr uint32_t kOpLo = 8192;
 constexpr uint32_t kOpGate = 16384;
 constexpr uint32_t kOpCopyBytes = 16384 + 80 * 4;   // staged per chunk (operator + gates)
 constexpr uint32_t kOpBytes = 16384 + 512;          // record stride in the workspace
+// bf16-input path: [T''; P T''] as three bf16 parts (each 64 x 32, K-major, 64-byte swizzle)
+constexpr uint32_t kOpBPart = 4096;
+constexpr uint32_t kOpBGate = 3 * kOpBPart;
+constexpr uint32_t kOpBCopyBytes = 3 * kOpBPart + 80 * 4;
 
 template <typename T>
 struct ExactTF32 { static constexpr bool value = false; };
@@ -89,10 +93,14 @@ __device__ __forceinline__ void sts1(uint32_t base, uint32_t off, float a)
 {
     asm volatile("st.shared.f32 [%0], %1;" ::"r"(base + off), "f"(a));
 }
-// Global store with the same property (no memory clobber).
+// Global stores with the same property (no memory clobber).
 __device__ __forceinline__ void stg1(void* p, float a)
 {
     asm volatile("st.global.f32 [%0], %1;" ::"l"(p), "f"(a));
+}
+__device__ __forceinline__ void stg32(void* p, uint32_t a)
+{
+    asm volatile("st.global.b32 [%0], %1;" ::"l"(p), "r"(a));
 }
 
 // Stores 8 consecutive K-elements (k0 % 8 == 0) of row r of a K-major SW128 tile of R rows, as hi

@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
         GDN_PREP_TRACE(iter, 3);
 
         // operator record: rows i of T'' = T diag(beta) and of P T'', TF32 hi/lo, swizzled image
-        uint8_t* dst = op + ((size_t)gc * H + h) * kOpBytes;
+        uint8_t* dst = op + ((size_t)gc * H + h) * kOpBytes;   // record stride shared with the fp32 path
         {
             const int j = lane, rg = warp;
             const float bj = bet[j];
@@ -246,19 +246,27 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
                 float acc = 0.f;
 #pragma unroll
                 for (int m = 0; m < 32; ++m) acc = fmaf(P[i * LD + m], tc[m], acc);
-                float hi, lo;
-                tf32_split(Tm[i * LD + j] * bj, hi, lo);
-                uint32_t o = sw128_off(i, j, 64);
-                stg1(dst + kOpHi + o, hi);
-                stg1(dst + kOpLo + o, lo);
-                tf32_split(acc, hi, lo);
-                o = sw128_off(32 + i, j, 64);
-                stg1(dst + kOpHi + o, hi);
-                stg1(dst + kOpLo + o, lo);
+                // three bf16 parts, lanes j and j+1 packed into one 32-bit store by the even lane
+                const float tv = Tm[i * LD + j] * bj;
+                const float tn = __shfl_xor_sync(0xffffffffu, tv, 1);
+                const float an = __shfl_xor_sync(0xffffffffu, acc, 1);
+                if ((j & 1) == 0) {
+                    uint32_t w1, w2, w3;
+                    bf16x2_split3(tv, tn, w1, w2, w3);
+                    uint32_t o = sw64_off_h(i, j);
+                    stg32(dst + o, w1);
+                    stg32(dst + kOpBPart + o, w2);
+                    stg32(dst + 2 * kOpBPart + o, w3);
+                    bf16x2_split3(acc, an, w1, w2, w3);
+                    o = sw64_off_h(32 + i, j);
+                    stg32(dst + o, w1);
+                    stg32(dst + kOpBPart + o, w2);
+                    stg32(dst + 2 * kOpBPart + o, w3);
+                }
             }
         }
         if (tid < 80) {
-            float* gt = reinterpret_cast<float*>(dst + kOpGate);
+            float* gt = reinterpret_cast<float*>(dst + kOpBGate);
             const float gl = gam[31];
             float val = 0.f;
             if (tid < 32) val = exp2f(gam[tid]);

@@ -36,16 +36,16 @@ struct ScanBf16Smem {
     // one stage
     static constexpr uint32_t oAKQ = 0;                               // [K;Q] bf16: NP panels x 64 rows x 128 B
     static constexpr uint32_t oOp = oAKQ + NP * 8192;                 // operator image + gates
-    static constexpr uint32_t oV = oOp + ((kOpCopyBytes + 1023) & ~1023u);   // V tile: 32 rows x MS bf16
+    static constexpr uint32_t oV = oOp + ((kOpBCopyBytes + 1023) & ~1023u);  // V tile: 32 rows x MS bf16
     static constexpr uint32_t kStage = ((oV + 32 * MS * 2) + 1023) & ~1023u;
-    static constexpr uint32_t kStageTx = NP * 2 * 4096 + kOpCopyBytes + 32 * MS * 2;
+    static constexpr uint32_t kStageTx = NP * 2 * 4096 + kOpBCopyBytes + 32 * MS * 2;
     // shared by all stages
     // B operands of the bf16 products are stored N-major (N = 3 parts x MS, two 64-wide N-blocks)
     static constexpr uint32_t kLboS = DK * 128;                       // N-block stride of S parts
     static constexpr uint32_t kLboU = 32 * 128;                       // N-block stride of U~ parts
     static constexpr uint32_t oBS = STAGES * kStage;                  // S parts, N-major: 2 x DK rows x 128 B
-    static constexpr uint32_t oBY = oBS + 2 * kLboS;                  // Y hi/lo (tf32, K-major): 2MS rows x 128 B
-    static constexpr uint32_t oBU = oBY + ((2 * MS * 128 + 1023) & ~1023u);  // U~ parts, N-major: 2 x 32 rows x 128 B
+    static constexpr uint32_t oBY = oBS + 2 * kLboS;                  // Y parts, N-major: 2 x 32 rows x 128 B
+    static constexpr uint32_t oBU = oBY + 2 * kLboU;                  // U~ parts, N-major: 2 x 32 rows x 128 B
     static constexpr uint32_t oBar = oBU + 2 * kLboU;
     static constexpr uint32_t oTmem = oBar + 8 * (2 * STAGES + 4);
     static constexpr uint32_t oAbort = oTmem + 4;
@@ -108,15 +108,15 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(tslot, 256);
+        tmem_alloc(tslot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    // accumulators: D1 [X;Z] 3MS columns, D2 [U;PU] 2MS columns, D3 dS^T 3MS columns
-    const uint32_t tD1 = tmem, tD2 = tmem + 96, tD3 = tmem + 160;
+    // accumulators: D1 [X;Z], D2 [U;PU], D3 dS^T, 3MS columns each (one block per bf16 part)
+    const uint32_t tD1 = tmem, tD2 = tmem + 128, tD3 = tmem + 256;
 
     if (warp == 8) {
         // ------------------------------------------------------------------ producer (one thread)
@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
                     tma_load_2d(st + L::oAKQ + p * 8192, &tm_k, h * DK + p * 64, t0, &full[s]);
                     tma_load_2d(st + L::oAKQ + p * 8192 + 4096, &tm_q, h * DK + p * 64, t0, &full[s]);
                 }
-                bulk_load(st + L::oOp, op + ((size_t)gc * H + h) * kOpBytes, kOpCopyBytes, &full[s]);
+                bulk_load(st + L::oOp, op + ((size_t)gc * H + h) * kOpBytes, kOpBCopyBytes, &full[s]);
                 tma_load_2d(st + L::oV, &tm_v, h * DV + r0, t0, &full[s]);
             }
         }
@@ -160,7 +160,8 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
 
         const float scale = rsqrtf((float)DK);
         constexpr uint32_t idA = idesc_bf16(128, 3 * MS, false, true);
-        constexpr uint32_t idB1 = idesc_tf32(128, MS), idB2 = idesc_tf32(128, 2 * MS);
+        constexpr uint32_t idB3 = idesc_bf16(128, 3 * MS, false, true), idB2 = idesc_bf16(128, 2 * MS, false, true),
+                           idB1 = idesc_bf16(128, MS, false, true);
         constexpr uint32_t idC = idesc_bf16(128, 3 * MS, true, true);
         const uint32_t lane_q = (uint32_t)(q4 * 32) << 16;
         bool aborted = false;
@@ -221,7 +222,7 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
             tc_fence_after();
             const int64_t t0 = seq_t0 + (int64_t)cl * kChunk;
             const int Lr = (int)((seq_end - t0) < kChunk ? (seq_end - t0) : kChunk);
-            const float* gate = reinterpret_cast<const float*>(stp + L::oOp + kOpGate);
+            const float* gate = reinterpret_cast<const float*>(stp + L::oOp + kOpBGate);
             const float Gam = gate[lane];           // token `lane` (quarters 0 and 1)
             const float del = gate[32 + lane];
             const float GamC = gate[64];
@@ -254,28 +255,24 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
                 }
                 const bool live = lane < Lr;
 #pragma unroll
-                for (int i = 0; i < MH; ++i) {
-                    float hi, lo;
-                    tf32_split(live ? vt[i] - Gam * za[i] : 0.f, hi, lo);
-                    sts1(sbase + L::oBY, sw128_off(hf * MH + i, lane, 2 * MS), hi);
-                    sts1(sbase + L::oBY, sw128_off(MS + hf * MH + i, lane, 2 * MS), lo);
-                }
+                for (int i = 0; i < MH; ++i) vt[i] = live ? vt[i] - Gam * za[i] : 0.f;
+                put_parts(sbase + L::oBY, L::kLboU, lane, vt);     // N = part * MS + i, K = token
                 GDN_SCAN_TRACE(cl, 15);
                 fence_async_smem();
             }
             tc_fence_before();
             named_bar(2, 256);
-            // ---- MMA_b: [U; PU] = [T''; PT''] Y  (3xTF32: hi x [hi|lo] rows, lo x hi rows)
+            // ---- MMA_b: [U; PU] = [T''; PT''] Y  (bf16 parts: a1 x [y1|y2|y3] + a2 x [y1|y2] + a3 x y1)
             if (tid == 0) {
                 GDN_SCAN_TRACE(cl, 5);
                 tc_fence_after();
-                const uint64_t ah = sw128_desc(st + L::oOp + kOpHi, 0, 64), al = sw128_desc(st + L::oOp + kOpLo, 0, 64);
-                const uint64_t b = sw128_desc(sbase + L::oBY, 0, 2 * MS);
+                const uint64_t b = sw128_desc_mn(sbase + L::oBY, L::kLboU, 1024);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t oa = sw128_ks_off(ks, 64), ob = sw128_ks_off(ks, 2 * MS);
-                    mma_tf32(tD2, ah + oa, b + ob, idB2, ks > 0);
-                    mma_tf32(tD2, al + oa, b + ob, idB1, 1);
+                for (int ks = 0; ks < 2; ++ks) {
+                    const uint64_t ob = (uint64_t)(ks * 128), oa = (uint64_t)(ks * 2);
+                    mma_bf16(tD2, sw64_desc(st + L::oOp) + oa, b + ob, idB3, ks > 0);
+                    mma_bf16(tD2, sw64_desc(st + L::oOp + kOpBPart) + oa, b + ob, idB2, 1);
+                    mma_bf16(tD2, sw64_desc(st + L::oOp + 2 * kOpBPart) + oa, b + ob, idB1, 1);
                 }
                 mma_commit(bar_b);
                 if (!mbar_wait(bar_b, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
@@ -285,12 +282,13 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
             if (*abort_flag) { aborted = true; break; }
             tc_fence_after();
             if (q4 < 2) {
-                float u[MH], ul[MH];
+                float u[MH], u2[MH], u3[MH];
                 tmem_ld<MH>(tD2 + lane_q + hf * MH, u);
-                tmem_ld<MH>(tD2 + lane_q + MS + hf * MH, ul);
+                tmem_ld<MH>(tD2 + lane_q + MS + hf * MH, u2);
+                tmem_ld<MH>(tD2 + lane_q + 2 * MS + hf * MH, u3);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < MH; ++i) u[i] += ul[i];
+                for (int i = 0; i < MH; ++i) u[i] = (u[i] + u2[i]) + u3[i];
                 if (q4 == 0) {
                     // U~ = diag(delta) U -> three bf16 parts, N-major B operand of MMA_c
                     // (N = part * MS + i, K = token = lane)
@@ -353,7 +351,7 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
         mbar_wait(bar_drain, 0, &never, 100000000ull);
     }
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 256);
+    if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace gdn

@@ -266,6 +266,23 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_m_major =
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// 16-bit K-major tile with the 64-byte swizzle (rows of 32 elements): 8-row groups of 512 bytes;
+// the 16-byte chunks of row r are permuted by XOR with ((r / 2) % 4).
+__device__ __forceinline__ uint32_t sw64_off_h(int r, int k)
+{
+    return (uint32_t)((r >> 3) * 512 + (r & 7) * 64 + ((((k >> 3) ^ ((r >> 1) & 3))) << 4) + ((k & 7) << 1));
+}
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t addr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;
+    d |= (uint64_t)(512u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)4u << 61;                          // 64-byte swizzle
+    return d;
+}
+
 // Byte offset of element (n, k) of a 16-bit tile stored N-major with the 128-byte swizzle: N runs
 // along 128-byte rows (64 elements), one row per K index, 8 K-rows per 1024-byte group; 64-wide
 // N-blocks are `lbo` bytes apart.
