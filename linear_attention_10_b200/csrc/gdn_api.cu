@@ -197,7 +197,8 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         const int64_t cap = (int64_t)g_num_sms * 4;
         const unsigned grid = (unsigned)(items < cap ? items : cap);
         ProfScope prof("gdn_prep_bf16_kernel", st);
-        k1<<<grid, 128, PL::kBytes, st>>>(tq, tk, g, beta, meta, chunk_tab, reinterpret_cast<uint8_t*>(op), H, status);
+        k1<<<grid, 128, PL::kBytes, st>>>(tq, tk, g, beta, meta, chunk_off, chunk_tab, reinterpret_cast<uint8_t*>(op),
+                                          H, status);
         if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
       }
     } else if (lay.nc_max > 0 && T_total > 0) {
@@ -216,18 +217,18 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         // bf16 inputs: operands staged by tensor maps, bf16 tensor-core products for K and Q
         constexpr int MSB = 32;
-        using SB2 = ScanBf16Smem<DK, MSB, 2>;
         using SB3 = ScanBf16Smem<DK, MSB, 3>;
-        constexpr int ST = (SB3::kBytes + 1024 <= 228 * 1024) ? 3 : 2;
+        using SB4 = ScanBf16Smem<DK, MSB, 4>;
+        constexpr int ST = (SB4::kBytes <= 227 * 1024) ? 4 : 3;
         using SB = ScanBf16Smem<DK, MSB, ST>;
-        static_assert(SB2::kBytes + 1024 <= 228 * 1024, "bf16 scan shared memory");
+        static_assert(SB3::kBytes <= 227 * 1024, "bf16 scan shared memory");
         static_assert(MSB == 32, "the V tensor map boxes 32 columns");
         auto kb = gdn_scan_bf16_kernel<DK, DV, MSB, ST>;
         if (cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SB::kBytes) != cudaSuccess)
             return GDN_ERR_LAUNCH;
         {
             ProfScope prof("gdn_scan_bf16_kernel", st);
-            kb<<<dim3((unsigned)N, H, DV / MSB), 288, SB::kBytes, st>>>(
+            kb<<<dim3((unsigned)N, H, DV / MSB), kScanBf16Threads, SB::kBytes, st>>>(
                 tq, tk, tv, meta, chunk_off, chunk_tab, reinterpret_cast<const uint8_t*>(op), state_in,
                 static_cast<__nv_bfloat16*>(out), state_out, H, status);
         }

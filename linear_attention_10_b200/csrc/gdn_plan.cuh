@@ -18,7 +18,7 @@ struct PrefillLayout {
     size_t off_meta;      // int32[8]: [0] chunk count, [1] seqlens error flag
     size_t off_chunk_off; // int32[N + 1]: first global chunk of each sequence
     size_t off_chunk_tab; // int4[nc_max]: (sequence, first token, rows, 0)
-    size_t off_op;        // [nc_max][H] operator records of 16896 bytes: [T''; P T''] image, gates
+    size_t off_op;        // [nc_max][H] operator records (up to 25088 bytes each)
     size_t total;
 
     static size_t align(size_t x) { return (x + 255) & ~size_t(255); }
@@ -30,7 +30,7 @@ struct PrefillLayout {
         off_meta = o;      o = align(o + 8 * sizeof(int));
         off_chunk_off = o; o = align(o + (size_t)(N + 1) * sizeof(int));
         off_chunk_tab = o; o = align(o + (size_t)nc_max * sizeof(int4));
-        off_op = o;        o = align(o + (size_t)nc_max * H * (16384 + 512));
+        off_op = o;        o = align(o + (size_t)nc_max * H * 25088);   // largest record of the two paths
         total = o;
         (void)dk;
     }

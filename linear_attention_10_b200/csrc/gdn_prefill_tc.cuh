@@ -49,10 +49,14 @@ constexpr uint32_t kOpLo = 8192;
 constexpr uint32_t kOpGate = 16384;
 constexpr uint32_t kOpCopyBytes = 16384 + 80 * 4;   // staged per chunk (operator + gates)
 constexpr uint32_t kOpBytes = 16384 + 512;          // record stride in the workspace
-// bf16-input path: [T''; P T''] as three bf16 parts (each 64 x 32, K-major, 64-byte swizzle)
+// bf16-input path record: three bf16 parts (each 64 x 32, K-major, 64-byte swizzle) of
+// [T''; P T''], then three of the cross-chunk Gram matrix G' = [K; Q] K_prev^T (the chunk's rows
+// against the previous chunk's keys in the same sequence), then the gates.
 constexpr uint32_t kOpBPart = 4096;
-constexpr uint32_t kOpBGate = 3 * kOpBPart;
-constexpr uint32_t kOpBCopyBytes = 3 * kOpBPart + 80 * 4;
+constexpr uint32_t kOpBCross = 3 * kOpBPart;
+constexpr uint32_t kOpBGate = 6 * kOpBPart;
+constexpr uint32_t kOpBCopyBytes = 6 * kOpBPart + 80 * 4;
+constexpr uint32_t kOpBytesB = 25088;
 
 template <typename T>
 struct ExactTF32 { static constexpr bool value = false; };
@@ -101,6 +105,10 @@ __device__ __forceinline__ void stg1(void* p, float a)
 __device__ __forceinline__ void stg32(void* p, uint32_t a)
 {
     asm volatile("st.global.b32 [%0], %1;" ::"l"(p), "r"(a));
+}
+__device__ __forceinline__ void stg128(void* p, const uint32_t (&w)[4])
+{
+    asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
 }
 
 // Stores 8 consecutive K-elements (k0 % 8 == 0) of row r of a K-major SW128 tile of R rows, as hi

@@ -31,15 +31,16 @@ struct PrepBf16Smem {
     static constexpr int NP = DK / 64;
     static constexpr uint32_t kTile = NP * 8192;                      // [K;Q] bf16: NP panels x 64 rows x 128 B
     static constexpr uint32_t oTile = 0;                              // two buffers
+    static constexpr uint32_t oPrev = 2 * kTile;                      // previous chunk's K: NP x 32 rows x 128 B
     static constexpr int LD = 33;
-    static constexpr uint32_t oG = 2 * kTile;                         // [32][33] A
+    static constexpr uint32_t oG = oPrev + NP * 4096;                 // [32][33] A
     static constexpr uint32_t oP = oG + 32 * LD * 4;                  // [32][33] P
     static constexpr uint32_t oT = oP + 32 * LD * 4;                  // [32][33] T
     static constexpr uint32_t oM = oT + 32 * LD * 4;                  // [16][17] A21 T11
     static constexpr uint32_t oGam = oM + 16 * 17 * 4;
     static constexpr uint32_t oBet = oGam + 128;
-    static constexpr uint32_t oBar = oBet + 128;                      // tile_full[2], mma, drain
-    static constexpr uint32_t oTmem = oBar + 32;
+    static constexpr uint32_t oBar = oBet + 128;                      // tile_full[2], mma, drain, prev_full
+    static constexpr uint32_t oTmem = oBar + 40;
     static constexpr uint32_t oAbort = oTmem + 4;
     static constexpr uint32_t kTotal = oAbort + 4;
     static constexpr uint32_t kBytes = kTotal + 1024;
@@ -51,6 +52,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
                                                                const float* __restrict__ g,
                                                                const float* __restrict__ beta,
                                                                const int* __restrict__ meta,
+                                                               const int* __restrict__ chunk_off,
                                                                const int4* __restrict__ chunk_tab,
                                                                uint8_t* __restrict__ op, int H, int* status)
 {
@@ -70,6 +72,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
     uint64_t* tile_full = reinterpret_cast<uint64_t*>(sm + L::oBar);
     uint64_t* mma_bar = tile_full + 2;
     uint64_t* drain = tile_full + 3;
+    uint64_t* prev_full = tile_full + 4;
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::oTmem);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::oAbort);
 
@@ -80,11 +83,12 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
         mbar_init(&tile_full[1], 1);
         mbar_init(mma_bar, 1);
         mbar_init(drain, 1);
+        mbar_init(prev_full, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(tslot, 32);
+        tmem_alloc(tslot, 64);      // columns 0..31: Gram products, 32..63: cross-chunk Gram
         tmem_relinquish();
     }
     tc_fence_before();
@@ -92,6 +96,8 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
+    // whether chunk gc has a previous chunk in its sequence (then the cross-chunk Gram is built)
+    auto has_prev = [&](int gc) { return gc > chunk_off[chunk_tab[gc].x]; };
     // copies the [K; Q] rows of one item into tile buffer `b` (thread 0 only)
     auto issue_tile = [&](int item, int b) {
         const int gc = item / H, h = item % H;
@@ -103,6 +109,17 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
             tma_load_2d(dst + p * 8192, &tm_k, h * DK + p * 64, t0, &tile_full[b]);
             tma_load_2d(dst + p * 8192 + 4096, &tm_q, h * DK + p * 64, t0, &tile_full[b]);
         }
+    };
+    // copies the previous chunk's K rows of one item into the single previous-K buffer (thread 0
+    // only; issued once the buffer's last reader has completed).  An item that starts its sequence
+    // loads its own K rows instead, so that the buffer's barrier completes once per item.
+    auto issue_prev = [&](int item) {
+        const int gc = item / H, h = item % H;
+        const int t0 = chunk_tab[gc].y;
+        const int tp = has_prev(gc) ? t0 - kChunk : t0;
+        mbar_arrive_expect_tx(prev_full, NP * 4096);
+#pragma unroll
+        for (int p = 0; p < NP; ++p) tma_load_2d(sbase + L::oPrev + p * 4096, &tm_k, h * DK + p * 64, tp, prev_full);
     };
     // gate inputs of one item (lanes of warp 2; zero past the chunk's rows)
     auto load_gates = [&](int item, float& gv, float& bv) {
@@ -116,6 +133,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
     if (tid == 0) {
         if ((int)blockIdx.x < nitems) issue_tile(blockIdx.x, 0);
         if ((int)(blockIdx.x + gridDim.x) < nitems) issue_tile(blockIdx.x + gridDim.x, 1);
+        if ((int)blockIdx.x < nitems) issue_prev(blockIdx.x);
     }
     float gv_cur = 0.f, bv_cur = 0.f;
     if (warp == 2 && (int)blockIdx.x < nitems) load_gates(blockIdx.x, gv_cur, bv_cur);
@@ -127,10 +145,12 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
         const int b = iter & 1;
         const int gc = item / H, h = item % H;
         const int Lr = chunk_tab[gc].z;
+        const bool prev = has_prev(gc);
 
         // Gram products D[r][n] = [K; Q]_r . K_n on the tensor cores (rows 64..127 unused)
         if (tid == 0) {
-            if (!mbar_wait(&tile_full[b], (iter >> 1) & 1u, abort_flag)) {
+            if (!mbar_wait(&tile_full[b], (iter >> 1) & 1u, abort_flag) ||
+                !mbar_wait(prev_full, iter & 1u, abort_flag)) {
                 tc_abort(status, abort_flag);
             } else {
                 tc_fence_after();
@@ -140,10 +160,21 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
                     const uint64_t o = sw128_ks_off(ks, 64);
                     mma_bf16(tmem, a + o, a + o, idG, ks > 0);
                 }
+                if (prev) {
+                    // G' = [K; Q] K_prev^T
+                    const uint64_t bp = sw128_desc(sbase + L::oPrev, 0, 32);
+#pragma unroll
+                    for (int ks = 0; ks < DK / 16; ++ks)
+                        mma_bf16(tmem + 32, a + sw128_ks_off(ks, 64), bp + sw128_ks_off(ks, 32), idG, ks > 0);
+                }
                 mma_commit(mma_bar);
                 if (!mbar_wait(mma_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
-                // the tile buffer is free again: fetch the item after next into it
-                else if (item + 2 * (int)gridDim.x < nitems) issue_tile(item + 2 * gridDim.x, b);
+                // the buffers are free again: fetch the item after next, and the next item's
+                // previous-chunk keys
+                else {
+                    if (item + 2 * (int)gridDim.x < nitems) issue_tile(item + 2 * gridDim.x, b);
+                    if (item + (int)gridDim.x < nitems) issue_prev(item + gridDim.x);
+                }
             }
         }
         if (warp == 2) {
@@ -179,6 +210,25 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
 #pragma unroll
             for (int j = 0; j < 32; ++j) sts1(dst, (uint32_t)(j * 4), (j < lim) ? wr * exp2f(gr - gj[j]) * d[j] : 0.f);
             GDN_PREP_TRACE(iter, 6);
+            if (prev) {
+                // row (32 w + r) of G' -> three bf16 parts, K-major 64-byte-swizzled A operand rows
+                float e[32];
+                tmem_ld32(tmem + 32 + ((uint32_t)(warp * 32) << 16), e);
+                tmem_ld_wait();
+                uint8_t* rec = op + ((size_t)gc * H + h) * kOpBytesB + kOpBCross;
+                const int row = warp * 32 + r;
+#pragma unroll
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    uint32_t w1[4], w2[4], w3[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        bf16x2_split3(e[c8 * 8 + 2 * q], e[c8 * 8 + 2 * q + 1], w1[q], w2[q], w3[q]);
+                    const uint32_t o = sw64_off_h(row, c8 * 8);
+                    stg128(rec + o, w1);
+                    stg128(rec + kOpBPart + o, w2);
+                    stg128(rec + 2 * kOpBPart + o, w3);
+                }
+            }
         }
         tc_fence_before();
         __syncthreads();
@@ -233,7 +283,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
         GDN_PREP_TRACE(iter, 3);
 
         // operator record: rows i of T'' = T diag(beta) and of P T'', TF32 hi/lo, swizzled image
-        uint8_t* dst = op + ((size_t)gc * H + h) * kOpBytes;   // record stride shared with the fp32 path
+        uint8_t* dst = op + ((size_t)gc * H + h) * kOpBytesB;
         {
             const int j = lane, rg = warp;
             const float bj = bet[j];
@@ -287,7 +337,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
         mbar_wait(drain, 0, &never, 100000000ull);
     }
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 32);
+    if (warp == 0) tmem_dealloc(tmem, 64);
 }
 
 }  // namespace gdn

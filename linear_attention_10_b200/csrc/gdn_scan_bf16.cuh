@@ -1,25 +1,43 @@
 // gdn_scan_bf16.cuh -- chunk-sequential scan of the chunked prefill for bf16 q/k/v (sm_100a).
 //
-// Same algebra as gdn_scan_tc_kernel (see gdn_prefill_tc.cuh): per chunk
+// Same algebra as gdn_scan_tc_kernel (see gdn_prefill_tc.cuh).  With S_c the state after chunk c
+// (S_-1 the initial state), chunk c needs X_c = K_c S_{c-1}^T and Z_c = Q_c S_{c-1}^T.  Because
 //
-//   MMA_a  [X ; Z]     = [K ; Q] S^T            M=64,  N=3MS, K=dk   kind::f16 (bf16)
-//   MMA_b  [U ; P U]   = [T'' ; P T''] Y        M=64,  N=2MS, K=32   kind::tf32 (3xTF32)
-//   MMA_c  (dS)^T      = K^T (diag(delta) U)    M=dk,  N=3MS, K=32   kind::f16 (bf16)
+//   S_{c-1} = Gamma_{c-1} S_{c-2} + U~_{c-1}^T K_{c-1}          (Gamma_{c-1}: total decay of c-1)
+//
+// the same products also read
+//
+//   [X_c; Z_c] = Gamma_{c-1} W_c + G'_c U~_{c-1},   W_c = [K_c; Q_c] S_{c-2}^T,
+//                                                   G'_c = [K_c; Q_c] K_{c-1}^T  (from the prep kernel)
+//
+// so the big product W_c can run one chunk early, off the dependent chain, and the chain of one
+// chunk shrinks to four steps:
+//
+//   MMA_x  D1 = G'_c U~_{c-1}              M=64, N=3MS, K=32  (three bf16 parts each side)
+//   epilogue  Y = V - diag(Gamma)(Gamma_{c-1} W_c + D1)
+//   MMA_b  [U; P U] = [T''; P T''] Y       M=64, N=3MS, K=32
+//   epilogue  U~ = diag(delta) U -> MMA_x of the next chunk;  O = s (diag(Gamma) Z + P U)
+//
+// Two thread groups share the work:
+//   * chain warps (0, 1, 4, 5): the two epilogues above; thread 0 issues MMA_b, MMA_x and
+//     MMA_c = K^T U~ (the state increment);
+//   * state warps (2, 3, 6, 7, 8, 9, 12, 13): S_c = Gamma_c S_{c-1} + (MMA_c result), the state's
+//     three bf16 parts as an operand, and W_{c+2} = [K; Q]_{c+2} S_c^T (issued by one of them);
+// and one producer thread (warp 10) stages each chunk's K/Q/V tiles and operator record with bulk
+// copies.  Every product is issued with M = 128 (the same cost as M = 64), so an accumulator row r
+// sits in tensor-memory lane r.
 //
 // What is specific to bf16 inputs:
 //   * q and k are exact bf16 values, so [K; Q] is used as stored: the tensor-memory-access engine
-//     copies the chunk's rows straight from global memory into the 128-byte-swizzled operand layout,
-//     and K^T for MMA_c is the same bytes read through an M-major descriptor.
-//   * The fp32 operand on the other side (S, U~) is split into three bf16 parts that carry its 24
-//     significant bits, stacked along N; one bf16 MMA (K=16) forms all three partial products, and
-//     the epilogue adds the three column blocks.  The result is fp32-accurate like the 3xTF32 split
-//     and needs half as many MMA instructions (bf16 takes 16 K-elements per instruction, TF32 8).
-//   * One producer thread stages each chunk with bulk copies (K/Q/V tiles by tensor map, the
-//     [T''; P T''] image and gates from the workspace) tracked by one transaction barrier; no thread
-//     converts or stores staged operands.
+//     copies the chunk's rows straight into the 128-byte-swizzled operand layout, and K^T for MMA_c
+//     is the same bytes read through an M-major descriptor.
+//   * The fp32 operands (S, Y, U~, the operator [T''; P T''] and G') are split into three bf16
+//     parts that carry their 24 significant bits; the parts of one side are stacked along N, and
+//     a1 x [b1|b2|b3] + a2 x [b1|b2] + a3 x b1 keeps every partial product above 2^-24 relative,
+//     so the results are fp32-accurate like the 3xTF32 split.
 //   * Rows of the last chunk of a sequence that lie beyond its end may hold the next sequence's
-//     tokens (or zeros past the tensor); the epilogues zero Y for them, the operator [T''; P T'']
-//     has zero columns for them, and their outputs are not stored, so they never contribute.
+//     tokens (or zeros past the tensor); the epilogue zeroes Y for them, the operator has zero
+//     columns for them, and their outputs are not stored, so they never contribute.
 #pragma once
 
 #include <cuda.h>
@@ -35,51 +53,75 @@ struct ScanBf16Smem {
     static constexpr int NP = DK / 64;                                // 64-element panels of dk
     // one stage
     static constexpr uint32_t oAKQ = 0;                               // [K;Q] bf16: NP panels x 64 rows x 128 B
-    static constexpr uint32_t oOp = oAKQ + NP * 8192;                 // operator image + gates
+    static constexpr uint32_t oOp = oAKQ + NP * 8192;                 // operator record: parts, G' parts, gates
     static constexpr uint32_t oV = oOp + ((kOpBCopyBytes + 1023) & ~1023u);  // V tile: 32 rows x MS bf16
     static constexpr uint32_t kStage = ((oV + 32 * MS * 2) + 1023) & ~1023u;
     static constexpr uint32_t kStageTx = NP * 2 * 4096 + kOpBCopyBytes + 32 * MS * 2;
     // shared by all stages
     // B operands of the bf16 products are stored N-major (N = 3 parts x MS, two 64-wide N-blocks)
     static constexpr uint32_t kLboS = DK * 128;                       // N-block stride of S parts
-    static constexpr uint32_t kLboU = 32 * 128;                       // N-block stride of U~ parts
+    static constexpr uint32_t kLboU = 32 * 128;                       // N-block stride of Y / U~ parts
     static constexpr uint32_t oBS = STAGES * kStage;                  // S parts, N-major: 2 x DK rows x 128 B
     static constexpr uint32_t oBY = oBS + 2 * kLboS;                  // Y parts, N-major: 2 x 32 rows x 128 B
     static constexpr uint32_t oBU = oBY + 2 * kLboU;                  // U~ parts, N-major: 2 x 32 rows x 128 B
     static constexpr uint32_t oBar = oBU + 2 * kLboU;
-    static constexpr uint32_t oTmem = oBar + 8 * (2 * STAGES + 4);
+    // full[STAGES], empty[STAGES], bar_x, bar_b, bar_c, bar_w[2], s_done, drain[2]
+    static constexpr int kBars = 2 * STAGES + 8;
+    static constexpr uint32_t oTmem = oBar + 8 * kBars;
     static constexpr uint32_t oAbort = oTmem + 4;
     static constexpr uint32_t kTotal = oAbort + 4;
     static constexpr uint32_t kBytes = kTotal + 1024;
 };
 
+constexpr int kScanBf16Threads = 448;
+
+// Writes the MH consecutive N-values (N = part * MS + hf * MH + i) of K-row `k` of an N-major
+// B tile as three bf16 parts: MH/8 16-byte stores per part.
+template <int MS, int MH>
+__device__ __forceinline__ void put_parts(uint32_t tile, uint32_t lbo, int k, int hf, const float (&x)[MH])
+{
+    using namespace sm100;
+    uint32_t w[3][MH / 2];
+#pragma unroll
+    for (int i = 0; i < MH; i += 2) bf16x2_split3(x[i], x[i + 1], w[0][i / 2], w[1][i / 2], w[2][i / 2]);
+#pragma unroll
+    for (int p = 0; p < 3; ++p) {
+#pragma unroll
+        for (int g = 0; g < MH / 8; ++g) {
+            const int n0 = p * MS + hf * MH + g * 8;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(tile + sw128_off_nmaj(n0, k, lbo)),
+                         "r"(w[p][g * 4]), "r"(w[p][g * 4 + 1]), "r"(w[p][g * 4 + 2]), "r"(w[p][g * 4 + 3]));
+        }
+    }
+}
+
 template <int DK, int DV, int MS, int STAGES>
-__global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
-                                                               const __grid_constant__ CUtensorMap tm_k,
-                                                               const __grid_constant__ CUtensorMap tm_v,
-                                                               const int* __restrict__ meta,
-                                                               const int* __restrict__ chunk_off,
-                                                               const int4* __restrict__ chunk_tab,
-                                                               const uint8_t* __restrict__ op,
-                                                               const float* state_in,
-                                                               __nv_bfloat16* __restrict__ out,
-                                                               float* state_out, int H, int* status)
+__global__ void __launch_bounds__(kScanBf16Threads, 1)
+    gdn_scan_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const int* __restrict__ meta,
+                         const int* __restrict__ chunk_off, const int4* __restrict__ chunk_tab,
+                         const uint8_t* __restrict__ op, const float* state_in, __nv_bfloat16* __restrict__ out,
+                         float* state_out, int H, int* status)
 {
     using namespace sm100;
     using L = ScanBf16Smem<DK, MS, STAGES>;
     static_assert(MS == 32, "bf16 scan: 32 state rows per CTA");
     static_assert(DK == 64 || DK == 128, "DK");
     static_assert(DV % MS == 0, "DV");
+    static_assert(STAGES >= 3, "W of chunk c + 2 is issued while chunks c and c + 1 are resident");
     constexpr int NP = L::NP;
+    constexpr int MH = MS / 2;                // columns of a column block handled by one thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::oBar);
     uint64_t* empty = full + STAGES;
-    uint64_t* bar_a = empty + STAGES;
-    uint64_t* bar_b = bar_a + 1;
-    uint64_t* bar_c = bar_a + 2;
-    uint64_t* bar_drain = bar_a + 3;
+    uint64_t* bar_x = empty + STAGES;         // MMA_c(c) and MMA_x(c + 1) done
+    uint64_t* bar_b = bar_x + 1;              // MMA_b done
+    uint64_t* bar_c = bar_x + 2;              // MMA_c done
+    uint64_t* bar_w = bar_x + 3;              // [2]: W of even / odd chunks done
+    uint64_t* s_done = bar_x + 5;             // the state warps have read the MMA_c result
+    uint64_t* drain = bar_x + 6;              // [2]
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::oTmem);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::oAbort);
 
@@ -100,10 +142,7 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(bar_a, 1);
-        mbar_init(bar_b, 1);
-        mbar_init(bar_c, 1);
-        mbar_init(bar_drain, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(bar_x + i, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -115,131 +154,103 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    // accumulators: D1 [X;Z], D2 [U;PU], D3 dS^T, 3MS columns each (one block per bf16 part)
-    const uint32_t tD1 = tmem, tD2 = tmem + 128, tD3 = tmem + 256;
+    // accumulators, 3MS columns each (one block per bf16 part of the B operand):
+    // D1 G'U~, D2 [U;PU], D3 (dS)^T, DW[2] W of even / odd chunks
+    static_assert(15 * MS <= 512, "tensor memory");
+    const uint32_t tD1 = tmem, tD2 = tmem + 3 * MS, tD3 = tmem + 6 * MS;
+    const uint32_t tDW0 = tmem + 9 * MS, tDW1 = tmem + 12 * MS;
 
-    if (warp == 8) {
+    constexpr uint32_t idW = idesc_bf16(128, 3 * MS, false, true);
+    constexpr uint32_t idB3 = idesc_bf16(128, 3 * MS, false, true), idB2 = idesc_bf16(128, 2 * MS, false, true),
+                       idB1 = idesc_bf16(128, MS, false, true);
+    constexpr uint32_t idC = idesc_bf16(128, 3 * MS, true, true);
+
+    // chunk-local index -> stage and the parity of its fill
+    auto stage_of = [](int c) { return c % STAGES; };
+    auto phase_of = [](int c) { return (uint32_t)(c / STAGES) & 1u; };
+
+    const bool chain = warp < 8 && (warp & 3) < 2;
+    const bool sgrp = (warp < 8) ? ((warp & 3) >= 2) : (warp == 8 || warp == 9 || warp == 12 || warp == 13);
+
+    if (warp == 10) {
         // ------------------------------------------------------------------ producer (one thread)
         if (lane == 0) {
+            int issued = 0;
             for (int cl = 0; cl < nch; ++cl) {
-                const int s = cl % STAGES;
-                if (cl >= STAGES &&
-                    !mbar_wait(&empty[s], (uint32_t)((cl / STAGES) - 1) & 1u, abort_flag)) {
+                const int s = stage_of(cl);
+                if (cl >= STAGES && !mbar_wait(&empty[s], (uint32_t)((cl / STAGES) - 1) & 1u, abort_flag)) {
                     tc_abort(status, abort_flag);
                     break;
                 }
                 const uint32_t st = sbase + s * L::kStage;
                 const int t0 = (int)(seq_t0 + (int64_t)cl * kChunk);
                 const int gc = c_begin + cl;
-                GDN_SCAN_TRACE(cl, 11);
                 mbar_arrive_expect_tx(&full[s], L::kStageTx);
 #pragma unroll
                 for (int p = 0; p < NP; ++p) {
                     tma_load_2d(st + L::oAKQ + p * 8192, &tm_k, h * DK + p * 64, t0, &full[s]);
                     tma_load_2d(st + L::oAKQ + p * 8192 + 4096, &tm_q, h * DK + p * 64, t0, &full[s]);
                 }
-                bulk_load(st + L::oOp, op + ((size_t)gc * H + h) * kOpBytes, kOpBCopyBytes, &full[s]);
+                bulk_load(st + L::oOp, op + ((size_t)gc * H + h) * kOpBytesB, kOpBCopyBytes, &full[s]);
                 tma_load_2d(st + L::oV, &tm_v, h * DV + r0, t0, &full[s]);
+                issued = cl + 1;
             }
+            // after an abort, copies still in flight land before the CTA exits (bounded)
+            volatile int never = 0;
+            for (int cl = (issued > STAGES ? issued - STAGES : 0); cl < issued; ++cl)
+                mbar_wait(&full[stage_of(cl)], phase_of(cl), &never, 100000000ull);
         }
-    } else {
-        // ------------------------------------------------------------------ consumers (8 warps)
-        // Every product is issued with M = 128 (same cost as M = 64), so an accumulator row r sits
-        // in TMEM lane r: warp w reads lane quarter q4 = w % 4, and the two warps of a quarter
-        // (w and w + 4) split the columns: this thread handles the MH columns [hf*MH, hf*MH + MH)
-        // of each column block.
-        constexpr int MH = MS / 2;
+    } else if (chain) {
+        // ------------------------------------------------------------------ chain warps
+        // quarter q4 = 0: X / Y / U~ rows (token = lane), q4 = 1: Z / O rows; hf: column half
         const int q4 = warp & 3, hf = warp >> 2;
-        // state: this thread holds S[hf*MH + ii][c_own], ii < MH (column c_own = TMEM lane of dS^T)
-        const int c_own = q4 * 32 + lane;
-        const bool owns = c_own < DK;
-        float S[MH];
-#pragma unroll
-        for (int ii = 0; ii < MH; ++ii)
-            S[ii] = (state_in && owns) ? state_in[(((size_t)n * H + h) * DV + r0 + hf * MH + ii) * DK + c_own] : 0.f;
-
-        const float scale = rsqrtf((float)DK);
-        constexpr uint32_t idA = idesc_bf16(128, 3 * MS, false, true);
-        constexpr uint32_t idB3 = idesc_bf16(128, 3 * MS, false, true), idB2 = idesc_bf16(128, 2 * MS, false, true),
-                           idB1 = idesc_bf16(128, MS, false, true);
-        constexpr uint32_t idC = idesc_bf16(128, 3 * MS, true, true);
         const uint32_t lane_q = (uint32_t)(q4 * 32) << 16;
-        bool aborted = false;
-
-        // Writes this thread's MH consecutive N-values (N = part * MS + hf * MH + i) of K-row `k` of an
-        // N-major B tile as three bf16 parts: two 16-byte stores per part.
-        auto put_parts = [&](uint32_t tile, uint32_t lbo, int k, const float (&x)[MH]) {
-            uint32_t w[3][MH / 2];
-#pragma unroll
-            for (int i = 0; i < MH; i += 2) bf16x2_split3(x[i], x[i + 1], w[0][i / 2], w[1][i / 2], w[2][i / 2]);
-#pragma unroll
-            for (int p = 0; p < 3; ++p) {
-#pragma unroll
-                for (int g = 0; g < MH / 8; ++g) {
-                    const int n0 = p * MS + hf * MH + g * 8;
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(tile + sw128_off_nmaj(n0, k, lbo)),
-                                 "r"(w[p][g * 4]), "r"(w[p][g * 4 + 1]), "r"(w[p][g * 4 + 2]), "r"(w[p][g * 4 + 3]));
-                }
-            }
-        };
-
-        for (int cl = 0; cl <= nch; ++cl) {
-            GDN_SCAN_TRACE(cl, 0);
-            // S -> three bf16 parts, N-major B operand of MMA_a (N = part * MS + row, K = dk column)
-            if (owns) put_parts(sbase + L::oBS, L::kLboS, c_own, S);
-            if (cl == nch) break;
-            GDN_SCAN_TRACE(cl, 10);
-            fence_async_smem();
-            GDN_SCAN_TRACE(cl, 12);
-            tc_fence_before();
-            named_bar(2, 256);      // every column of S written before MMA_a reads it
-            GDN_SCAN_TRACE(cl, 1);
-            const int s = cl % STAGES;
+        const float scale = rsqrtf((float)DK);
+        float GamPrev = 1.f;
+        for (int c = 0; c < nch; ++c) {
+            const int s = stage_of(c);
             const uint32_t st = sbase + s * L::kStage;
             const uint8_t* stp = sm + s * L::kStage;
-
-            // ---- MMA_a: [X; Z] = [K; Q] S^T  (column blocks: the three parts of S)
-            if (tid == 0) {
-                if (!mbar_wait(&full[s], (uint32_t)(cl / STAGES) & 1u, abort_flag)) {
-                    tc_abort(status, abort_flag);
-                } else {
-                    GDN_SCAN_TRACE(cl, 2);
-                    tc_fence_after();
-                    const uint64_t a = sw128_desc(st + L::oAKQ, 0, 64);
-                    const uint64_t b = sw128_desc_mn(sbase + L::oBS, L::kLboS, 1024);
-#pragma unroll
-                    for (int ks = 0; ks < DK / 16; ++ks)
-                        mma_bf16(tD1, a + sw128_ks_off(ks, 64), b + (uint64_t)(ks * 128), idA, ks > 0);
-                    mma_commit(bar_a);
-                    GDN_SCAN_TRACE(cl, 3);
-                    if (!mbar_wait(bar_a, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
-                    GDN_SCAN_TRACE(cl, 4);
-                }
-            }
-            named_bar(2, 256);
-            GDN_SCAN_TRACE(cl, 13);
-            if (*abort_flag) { aborted = true; break; }
+            GDN_SCAN_TRACE(c, 0);
+            bool ok = mbar_wait(&full[s], phase_of(c), abort_flag) &&
+                      mbar_wait(&bar_w[c & 1], (uint32_t)(c >> 1) & 1u, abort_flag);
+            GDN_SCAN_TRACE(c, 1);
+            if (ok && c > 0) ok = mbar_wait(bar_x, (uint32_t)(c - 1) & 1u, abort_flag);
+            if (!ok) tc_abort(status, abort_flag);
+            GDN_SCAN_TRACE(c, 2);
             tc_fence_after();
-            const int64_t t0 = seq_t0 + (int64_t)cl * kChunk;
+            const int64_t t0 = seq_t0 + (int64_t)c * kChunk;
             const int Lr = (int)((seq_end - t0) < kChunk ? (seq_end - t0) : kChunk);
             const float* gate = reinterpret_cast<const float*>(stp + L::oOp + kOpBGate);
-            const float Gam = gate[lane];           // token `lane` (quarters 0 and 1)
+            const float Gam = gate[lane];
             const float del = gate[32 + lane];
             const float GamC = gate[64];
+            // [X; Z] rows: Gamma_{c-1} W_c + G'_c U~_{c-1}  (chunk 0: W_0 = [K; Q] S_-1^T alone)
             float za[MH];
-            if (q4 < 2) {
-                // quarter 0: X rows (token = lane), quarter 1: Z rows (token = lane)
-                float x1[MH], x2[MH], x3[MH];
-                tmem_ld<MH>(tD1 + lane_q + hf * MH, x1);
-                tmem_ld<MH>(tD1 + lane_q + MS + hf * MH, x2);
-                tmem_ld<MH>(tD1 + lane_q + 2 * MS + hf * MH, x3);
-                tmem_ld_wait();
-                GDN_SCAN_TRACE(cl, 14);
+            {
+                float w1[MH], w2[MH], w3[MH];
+                const uint32_t tw = ((c & 1) ? tDW1 : tDW0) + lane_q + hf * MH;
+                tmem_ld<MH>(tw, w1);
+                tmem_ld<MH>(tw + MS, w2);
+                tmem_ld<MH>(tw + 2 * MS, w3);
+                if (c > 0) {
+                    float x1[MH], x2[MH], x3[MH];
+                    const uint32_t tx = tD1 + lane_q + hf * MH;
+                    tmem_ld<MH>(tx, x1);
+                    tmem_ld<MH>(tx + MS, x2);
+                    tmem_ld<MH>(tx + 2 * MS, x3);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < MH; ++i) za[i] = (x1[i] + x2[i]) + x3[i];
+                    for (int i = 0; i < MH; ++i) za[i] = fmaf(GamPrev, (w1[i] + w2[i]) + w3[i], (x1[i] + x2[i]) + x3[i]);
+                } else {
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < MH; ++i) za[i] = (w1[i] + w2[i]) + w3[i];
+                }
             }
+            GDN_SCAN_TRACE(c, 3);
             if (q4 == 0) {
-                // Y = V - diag(Gamma) X (zero past the sequence end) -> tf32 hi/lo rows of MMA_b's B
+                // Y = V - diag(Gamma) X (zero past the sequence end) -> bf16 parts of MMA_b's B
                 float vt[MH];
                 const uint4* vrow = reinterpret_cast<const uint4*>(stp + L::oV + lane * MS * 2 + hf * MH * 2);
 #pragma unroll
@@ -256,15 +267,14 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
                 const bool live = lane < Lr;
 #pragma unroll
                 for (int i = 0; i < MH; ++i) vt[i] = live ? vt[i] - Gam * za[i] : 0.f;
-                put_parts(sbase + L::oBY, L::kLboU, lane, vt);     // N = part * MS + i, K = token
-                GDN_SCAN_TRACE(cl, 15);
+                put_parts<MS, MH>(sbase + L::oBY, L::kLboU, lane, hf, vt);   // N = part * MS + i, K = token
                 fence_async_smem();
             }
             tc_fence_before();
-            named_bar(2, 256);
-            // ---- MMA_b: [U; PU] = [T''; PT''] Y  (bf16 parts: a1 x [y1|y2|y3] + a2 x [y1|y2] + a3 x y1)
+            if (named_bar_any(2, 128, *abort_flag)) break;
+            GDN_SCAN_TRACE(c, 4);
+            // ---- MMA_b: [U; PU] = [T''; PT''] Y
             if (tid == 0) {
-                GDN_SCAN_TRACE(cl, 5);
                 tc_fence_after();
                 const uint64_t b = sw128_desc_mn(sbase + L::oBY, L::kLboU, 1024);
 #pragma unroll
@@ -275,26 +285,24 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
                     mma_bf16(tD2, sw64_desc(st + L::oOp + 2 * kOpBPart) + oa, b + ob, idB1, 1);
                 }
                 mma_commit(bar_b);
-                if (!mbar_wait(bar_b, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
-                GDN_SCAN_TRACE(cl, 6);
             }
-            named_bar(2, 256);
-            if (*abort_flag) { aborted = true; break; }
+            if (!mbar_wait(bar_b, (uint32_t)c & 1u, abort_flag)) tc_abort(status, abort_flag);
+            GDN_SCAN_TRACE(c, 5);
             tc_fence_after();
-            if (q4 < 2) {
+            {
                 float u[MH], u2[MH], u3[MH];
-                tmem_ld<MH>(tD2 + lane_q + hf * MH, u);
-                tmem_ld<MH>(tD2 + lane_q + MS + hf * MH, u2);
-                tmem_ld<MH>(tD2 + lane_q + 2 * MS + hf * MH, u3);
+                const uint32_t tu = tD2 + lane_q + hf * MH;
+                tmem_ld<MH>(tu, u);
+                tmem_ld<MH>(tu + MS, u2);
+                tmem_ld<MH>(tu + 2 * MS, u3);
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < MH; ++i) u[i] = (u[i] + u2[i]) + u3[i];
                 if (q4 == 0) {
-                    // U~ = diag(delta) U -> three bf16 parts, N-major B operand of MMA_c
-                    // (N = part * MS + i, K = token = lane)
+                    // U~ = diag(delta) U -> bf16 parts, N-major B operand of MMA_c and MMA_x
 #pragma unroll
                     for (int i = 0; i < MH; ++i) u[i] *= del;
-                    put_parts(sbase + L::oBU, L::kLboU, lane, u);
+                    put_parts<MS, MH>(sbase + L::oBU, L::kLboU, lane, hf, u);
                     fence_async_smem();
                 } else if (lane < Lr) {
                     // O = s (diag(Gamma) Z + P U) for token `lane`, this thread's MH columns
@@ -305,36 +313,126 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
                 }
             }
             tc_fence_before();
-            named_bar(2, 256);
-            // ---- MMA_c: dS^T = K^T U~  (K^T read M-major from the K rows; frees the stage)
+            if (named_bar_any(2, 128, *abort_flag)) break;
+            GDN_SCAN_TRACE(c, 6);
             if (tid == 0) {
-                GDN_SCAN_TRACE(cl, 7);
                 tc_fence_after();
-                const uint64_t a = sw128_desc_mn(st + L::oAKQ, 8192, 1024);
-                const uint64_t b = sw128_desc_mn(sbase + L::oBU, L::kLboU, 1024);
+                // ---- MMA_c: (dS)^T = K^T U~, once the state warps have read the previous one
+                bool ok2 = (c == 0) || mbar_wait(s_done, (uint32_t)(c - 1) & 1u, abort_flag);
+                GDN_SCAN_TRACE(c, 8);
+                if (ok2) {
+                    const uint64_t a = sw128_desc_mn(st + L::oAKQ, 8192, 1024);
+                    const uint64_t b = sw128_desc_mn(sbase + L::oBU, L::kLboU, 1024);
 #pragma unroll
-                for (int ks = 0; ks < 2; ++ks)
-                    mma_bf16(tD3, a + (uint64_t)(ks * 128), b + (uint64_t)(ks * 128), idC, ks > 0);
-                mma_commit(bar_c);
-                mma_commit(&empty[s]);
-                if (!mbar_wait(bar_c, (uint32_t)cl & 1u, abort_flag)) tc_abort(status, abort_flag);
-                GDN_SCAN_TRACE(cl, 8);
+                    for (int ks = 0; ks < 2; ++ks)
+                        mma_bf16(tD3, a + (uint64_t)(ks * 128), b + (uint64_t)(ks * 128), idC, ks > 0);
+                    mma_commit(bar_c);
+                    GDN_SCAN_TRACE(c, 9);
+                    // ---- MMA_x of the next chunk: D1 = G'_{c+1} U~_c
+                    if (c + 1 < nch) {
+                        const int s1 = stage_of(c + 1);
+                        ok2 = mbar_wait(&full[s1], phase_of(c + 1), abort_flag);
+                        GDN_SCAN_TRACE(c, 10);
+                        if (ok2) {
+                            tc_fence_after();
+                            const uint32_t g = sbase + s1 * L::kStage + L::oOp + kOpBCross;
+#pragma unroll
+                            for (int ks = 0; ks < 2; ++ks) {
+                                const uint64_t ob = (uint64_t)(ks * 128), oa = (uint64_t)(ks * 2);
+                                mma_bf16(tD1, sw64_desc(g) + oa, b + ob, idB3, ks > 0);
+                                mma_bf16(tD1, sw64_desc(g + kOpBPart) + oa, b + ob, idB2, 1);
+                                mma_bf16(tD1, sw64_desc(g + 2 * kOpBPart) + oa, b + ob, idB1, 1);
+                            }
+                            mma_commit(bar_x);
+                        }
+                    }
+                }
+                if (!ok2) tc_abort(status, abort_flag);
+                GDN_SCAN_TRACE(c, 7);
             }
-            named_bar(2, 256);
-            if (*abort_flag) { aborted = true; break; }
+            GamPrev = GamC;
+        }
+    } else if (sgrp) {
+        // ------------------------------------------------------------------ state warps
+        // this thread holds S[hf*MH + ii][c_own], ii < MH (column c_own = TMEM lane of (dS)^T)
+        const int q4 = warp & 3, hf = (warp >> 2) & 1;
+        const int c_own = q4 * 32 + lane;
+        const bool owns = c_own < DK;
+        const uint32_t lane_q = (uint32_t)(q4 * 32) << 16;
+        const bool lead = (warp == 8 && lane == 0);
+        float S[MH];
+#pragma unroll
+        for (int ii = 0; ii < MH; ++ii)
+            S[ii] = (state_in && owns) ? state_in[(((size_t)n * H + h) * DV + r0 + hf * MH + ii) * DK + c_own] : 0.f;
+
+        // W_k = [K; Q]_k S^T into DW[k & 1], where the S parts hold the state entering chunk k - 1
+        auto issue_w = [&](int k) -> bool {
+            const int sk = stage_of(k);
+            if (!mbar_wait(&full[sk], phase_of(k), abort_flag)) return false;
+            tc_fence_after();
+            const uint64_t a = sw128_desc(sbase + sk * L::kStage + L::oAKQ, 0, 64);
+            const uint64_t b = sw128_desc_mn(sbase + L::oBS, L::kLboS, 1024);
+            const uint32_t d = (k & 1) ? tDW1 : tDW0;
+#pragma unroll
+            for (int ks = 0; ks < DK / 16; ++ks)
+                mma_bf16(d, a + sw128_ks_off(ks, 64), b + (uint64_t)(ks * 128), idW, ks > 0);
+            mma_commit(&bar_w[k & 1]);
+            return true;
+        };
+
+        bool aborted = false;
+        if (nch > 0) {
+            // the initial state serves both W_0 and W_1
+            if (owns) put_parts<MS, MH>(sbase + L::oBS, L::kLboS, c_own, hf, S);
+            fence_async_smem();
+            tc_fence_before();
+            named_bar(3, 256);
+            if (lead) {
+                tc_fence_after();
+                if (!issue_w(0) || (nch > 1 && !issue_w(1))) tc_abort(status, abort_flag);
+            }
+        }
+        for (int j = 0; j < nch; ++j) {
+            const int s = stage_of(j);
+            if (!mbar_wait(&full[s], phase_of(j), abort_flag) || !mbar_wait(bar_c, (uint32_t)j & 1u, abort_flag))
+                tc_abort(status, abort_flag);
+            if (lead) GDN_SCAN_TRACE(j, 12);
             tc_fence_after();
             {
-                // S' = Gamma_31 S + dS  (row c_own of dS^T, this thread's half of the S rows)
+                // S_j = Gamma_j S_{j-1} + dS_j  (row c_own of (dS)^T, this thread's half of the S rows)
+                const float GamC = reinterpret_cast<const float*>(sm + s * L::kStage + L::oOp + kOpBGate)[64];
                 float d1[MH], d2[MH], d3[MH];
-                tmem_ld<MH>(tD3 + lane_q + hf * MH, d1);
-                tmem_ld<MH>(tD3 + lane_q + MS + hf * MH, d2);
-                tmem_ld<MH>(tD3 + lane_q + 2 * MS + hf * MH, d3);
+                const uint32_t td = tD3 + lane_q + hf * MH;
+                tmem_ld<MH>(td, d1);
+                tmem_ld<MH>(td + MS, d2);
+                tmem_ld<MH>(td + 2 * MS, d3);
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < MH; ++i) S[i] = fmaf(GamC, S[i], (d1[i] + d2[i]) + d3[i]);
             }
-            GDN_SCAN_TRACE(cl, 9);
             tc_fence_before();
+            if (named_bar_any(3, 256, *abort_flag)) { aborted = true; break; }
+            if (lead) {
+                // (dS)^T is read and stage j has no reader left
+                mbar_arrive(s_done);
+                mbar_arrive(&empty[s]);
+                GDN_SCAN_TRACE(j, 13);
+            }
+            if (j + 2 < nch) {
+                // once W_{j+1} has finished reading the previous state's parts
+                if (!mbar_wait(&bar_w[(j + 1) & 1], (uint32_t)((j + 1) >> 1) & 1u, abort_flag))
+                    tc_abort(status, abort_flag);
+                if (owns) put_parts<MS, MH>(sbase + L::oBS, L::kLboS, c_own, hf, S);
+                fence_async_smem();
+                tc_fence_before();
+                if (named_bar_any(3, 256, *abort_flag)) { aborted = true; break; }
+                if (lead) {
+                    GDN_SCAN_TRACE(j, 14);
+                    tc_fence_after();
+                    if (!issue_w(j + 2)) tc_abort(status, abort_flag);
+                    GDN_SCAN_TRACE(j, 15);
+                }
+            }
         }
         if (state_out && owns && !aborted) {
 #pragma unroll
@@ -344,11 +442,12 @@ __global__ void __launch_bounds__(288, 1) gdn_scan_bf16_kernel(const __grid_cons
     }
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && *abort_flag) {
-        // after a timeout, give copies and MMAs still in flight a bounded time to finish
-        mma_commit(bar_drain);
+    if (*abort_flag && (tid == 0 || tid == 256)) {
+        // after a timeout, give the products this thread issued a bounded time to finish
+        uint64_t* d = drain + (tid == 0 ? 0 : 1);
+        mma_commit(d);
         volatile int never = 0;
-        mbar_wait(bar_drain, 0, &never, 100000000ull);
+        mbar_wait(d, 0, &never, 100000000ull);
     }
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 512);

@@ -112,6 +112,23 @@ __device__ __forceinline__ void named_bar(int id, int nthreads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Named barrier that also returns, to every participating thread, whether any of them passed
+// pred = true.  A group that leaves a loop on a flag another group may set at any moment takes the
+// decision from this value, so that all of its threads leave together.
+__device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
 // ------------------------------------------------------------------------------------------------
 // Tensor memory
 // ------------------------------------------------------------------------------------------------
