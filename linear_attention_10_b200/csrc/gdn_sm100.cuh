@@ -310,19 +310,20 @@ __device__ __forceinline__ uint32_t sw128_off_nmaj(int n, int k, uint32_t lbo)
 }
 
 // Three-way bf16 split of two values at once, packed in pairs (first value in the low half), for
-// N-major tiles where the two values are adjacent along N.  Rounding to nearest at each stage;
-// every remainder is exact in fp32, so the three parts carry the value's 24 significant bits.
+// N-major tiles where the two values are adjacent along N.  Each part is the top 16 bits of what
+// the previous parts left (truncation), and every remainder is exact in fp32: x = b1 + b2 + b3 + r
+// with |r| < 2^-23 |x|, so the three parts carry fp32 precision.  Only integer byte permutes,
+// masks and fp32 subtractions are used -- no format conversions, which issue at a quarter of the
+// fp32 rate and would make the split the slowest step of an epilogue.
 __device__ __forceinline__ void bf16x2_split3(float x, float y, uint32_t& p1, uint32_t& p2, uint32_t& p3)
 {
-    __nv_bfloat162 h1 = __floats2bfloat162_rn(x, y);
-    const float2 f1 = __bfloat1622float2(h1);
-    const float rx = x - f1.x, ry = y - f1.y;
-    __nv_bfloat162 h2 = __floats2bfloat162_rn(rx, ry);
-    const float2 f2 = __bfloat1622float2(h2);
-    __nv_bfloat162 h3 = __floats2bfloat162_rn(rx - f2.x, ry - f2.y);
-    p1 = *reinterpret_cast<uint32_t*>(&h1);
-    p2 = *reinterpret_cast<uint32_t*>(&h2);
-    p3 = *reinterpret_cast<uint32_t*>(&h3);
+    const uint32_t xb = __float_as_uint(x), yb = __float_as_uint(y);
+    p1 = __byte_perm(xb, yb, 0x7632);
+    const float rx = x - __uint_as_float(xb & 0xFFFF0000u), ry = y - __uint_as_float(yb & 0xFFFF0000u);
+    const uint32_t rxb = __float_as_uint(rx), ryb = __float_as_uint(ry);
+    p2 = __byte_perm(rxb, ryb, 0x7632);
+    const float sx = rx - __uint_as_float(rxb & 0xFFFF0000u), sy = ry - __uint_as_float(ryb & 0xFFFF0000u);
+    p3 = __byte_perm(__float_as_uint(sx), __float_as_uint(sy), 0x7632);
 }
 
 // Instruction descriptor: kind::tf32, fp32 accumulator, both operands K-major.
