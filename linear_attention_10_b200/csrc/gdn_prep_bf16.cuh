@@ -32,14 +32,15 @@ struct PrepBf16Smem {
     static constexpr uint32_t kTile = NP * 8192;                      // [K;Q] bf16: NP panels x 64 rows x 128 B
     static constexpr uint32_t oTile = 0;                              // two buffers
     static constexpr uint32_t oPrev = 2 * kTile;                      // previous chunk's K: NP x 32 rows x 128 B
-    static constexpr int LD = 33;
-    static constexpr uint32_t oG = oPrev + NP * 4096;                 // [32][33] A
-    static constexpr uint32_t oP = oG + 32 * LD * 4;                  // [32][33] P
-    static constexpr uint32_t oT = oP + 32 * LD * 4;                  // [32][33] T
+    static constexpr int LD = 36;                                     // row pitch: 16-byte rows, no bank conflicts
+    static constexpr uint32_t oG = oPrev + NP * 4096;                 // [32][LD] A
+    static constexpr uint32_t oP = oG + 32 * LD * 4;                  // [32][LD] P
+    static constexpr uint32_t oT = oP + 32 * LD * 4;                  // [32][LD] T
     static constexpr uint32_t oM = oT + 32 * LD * 4;                  // [16][17] A21 T11
     static constexpr uint32_t oGam = oM + 16 * 17 * 4;
     static constexpr uint32_t oBet = oGam + 128;
-    static constexpr uint32_t oBar = oBet + 128;                      // tile_full[2], mma, drain, prev_full
+    static constexpr uint32_t oAlph = oBet + 128;                     // per-token decays exp(g), one spare
+    static constexpr uint32_t oBar = oAlph + 136;                      // tile_full[2], mma, drain, prev_full
     static constexpr uint32_t oTmem = oBar + 40;
     static constexpr uint32_t oAbort = oTmem + 4;
     static constexpr uint32_t kTotal = oAbort + 4;
@@ -69,6 +70,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
     float* M1 = reinterpret_cast<float*>(sm + L::oM);
     float* gam = reinterpret_cast<float*>(sm + L::oGam);
     float* bet = reinterpret_cast<float*>(sm + L::oBet);
+    float* alph = reinterpret_cast<float*>(sm + L::oAlph);
     uint64_t* tile_full = reinterpret_cast<uint64_t*>(sm + L::oBar);
     uint64_t* mma_bar = tile_full + 2;
     uint64_t* drain = tile_full + 3;
@@ -187,6 +189,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
             }
             gam[lane] = gv * 1.4426950408889634f;    // log2(e) * gamma: gates become exp2 of differences
             bet[lane] = bv_cur;
+            alph[lane] = exp2f(gv_cur * 1.4426950408889634f);
             if (item + (int)gridDim.x < nitems) load_gates(item + gridDim.x, gv_cur, bv_cur);
         }
         __syncthreads();
@@ -199,16 +202,23 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
             tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), d);
             tmem_ld_wait();
             GDN_PREP_TRACE(iter, 5);
+            // lane r: decay ratios exp(gamma_r - gamma_j) = prod_{j < i <= r} exp(g_i) for j < r, as a
+            // running product from the diagonal down (one multiply per entry instead of an exp2)
             const int r = lane;
-            float gj[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) gj[j] = gam[j];
-            const float gr = gam[r], br = bet[r];
-            const uint32_t dst = sbase + ((warp == 0) ? L::oG : L::oP) + (uint32_t)(r * LD * 4);
-            const float wr = (warp == 0) ? br : 1.f;
+            const float wr = (warp == 0) ? bet[r] : 1.f;
             const int lim = (warp == 0) ? r : r + 1;      // strictly lower for A, incl. diagonal for P
+            float vals[32];
+            float a = 1.f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) sts1(dst, (uint32_t)(j * 4), (j < lim) ? wr * exp2f(gr - gj[j]) * d[j] : 0.f);
+            for (int j = 31; j >= 0; --j) {
+                a = (j >= r) ? 1.f : a * alph[j + 1];
+                vals[j] = (j < lim) ? wr * a * d[j] : 0.f;
+            }
+            const uint32_t dst = sbase + ((warp == 0) ? L::oG : L::oP) + (uint32_t)(r * LD * 4);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + q * 16), "f"(vals[4 * q]),
+                             "f"(vals[4 * q + 1]), "f"(vals[4 * q + 2]), "f"(vals[4 * q + 3]));
             GDN_PREP_TRACE(iter, 6);
             if (prev) {
                 // row (32 w + r) of G' -> three bf16 parts, K-major 64-byte-swizzled A operand rows
@@ -294,8 +304,15 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
             for (int rr = 0; rr < 8; ++rr) {
                 const int i = rg * 8 + rr;
                 float acc = 0.f;
+                const float4* prow = reinterpret_cast<const float4*>(P + i * LD);
 #pragma unroll
-                for (int m = 0; m < 32; ++m) acc = fmaf(P[i * LD + m], tc[m], acc);
+                for (int q = 0; q < 8; ++q) {
+                    const float4 pv = prow[q];
+                    acc = fmaf(pv.x, tc[4 * q], acc);
+                    acc = fmaf(pv.y, tc[4 * q + 1], acc);
+                    acc = fmaf(pv.z, tc[4 * q + 2], acc);
+                    acc = fmaf(pv.w, tc[4 * q + 3], acc);
+                }
                 // three bf16 parts, lanes j and j+1 packed into one 32-bit store by the even lane
                 const float tv = Tm[i * LD + j] * bj;
                 const float tn = __shfl_xor_sync(0xffffffffu, tv, 1);
