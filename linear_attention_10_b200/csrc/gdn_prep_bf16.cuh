@@ -40,8 +40,8 @@ struct PrepBf16Smem {
     static constexpr uint32_t oGam = oM + 16 * 17 * 4;
     static constexpr uint32_t oBet = oGam + 128;
     static constexpr uint32_t oAlph = oBet + 128;                     // per-token decays exp(g), one spare
-    static constexpr uint32_t oBar = oAlph + 136;                      // tile_full[2], mma, drain, prev_full
-    static constexpr uint32_t oTmem = oBar + 40;
+    static constexpr uint32_t oBar = oAlph + 136;                      // tile_full[2], mma, drain, prev_full, cross
+    static constexpr uint32_t oTmem = oBar + 48;
     static constexpr uint32_t oAbort = oTmem + 4;
     static constexpr uint32_t kTotal = oAbort + 4;
     static constexpr uint32_t kBytes = kTotal + 1024;
@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
     uint64_t* mma_bar = tile_full + 2;
     uint64_t* drain = tile_full + 3;
     uint64_t* prev_full = tile_full + 4;
+    uint64_t* cross_bar = tile_full + 5;      // the cross-chunk Gram product (and all before it) done
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::oTmem);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::oAbort);
 
@@ -86,6 +87,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
         mbar_init(mma_bar, 1);
         mbar_init(drain, 1);
         mbar_init(prev_full, 1);
+        mbar_init(cross_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -162,21 +164,16 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
                     const uint64_t o = sw128_ks_off(ks, 64);
                     mma_bf16(tmem, a + o, a + o, idG, ks > 0);
                 }
+                mma_commit(mma_bar);
                 if (prev) {
-                    // G' = [K; Q] K_prev^T
+                    // G' = [K; Q] K_prev^T, completes while the gates are applied
                     const uint64_t bp = sw128_desc(sbase + L::oPrev, 0, 32);
 #pragma unroll
                     for (int ks = 0; ks < DK / 16; ++ks)
                         mma_bf16(tmem + 32, a + sw128_ks_off(ks, 64), bp + sw128_ks_off(ks, 32), idG, ks > 0);
                 }
-                mma_commit(mma_bar);
+                mma_commit(cross_bar);
                 if (!mbar_wait(mma_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
-                // the buffers are free again: fetch the item after next, and the next item's
-                // previous-chunk keys
-                else {
-                    if (item + 2 * (int)gridDim.x < nitems) issue_tile(item + 2 * gridDim.x, b);
-                    if (item + (int)gridDim.x < nitems) issue_prev(item + gridDim.x);
-                }
             }
         }
         if (warp == 2) {
@@ -220,6 +217,14 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
                 asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + q * 16), "f"(vals[4 * q]),
                              "f"(vals[4 * q + 1]), "f"(vals[4 * q + 2]), "f"(vals[4 * q + 3]));
             GDN_PREP_TRACE(iter, 6);
+            // the tile buffers are free once G' has been formed: fetch the item after next and the
+            // next item's previous-chunk keys
+            if (!mbar_wait(cross_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
+            tc_fence_after();
+            if (tid == 0 && !*abort_flag) {
+                if (item + 2 * (int)gridDim.x < nitems) issue_tile(item + 2 * gridDim.x, b);
+                if (item + (int)gridDim.x < nitems) issue_prev(item + gridDim.x);
+            }
             if (prev) {
                 // row (32 w + r) of G' -> three bf16 parts, K-major 64-byte-swizzled A operand rows
                 float e[32];
