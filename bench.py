@@ -62,6 +62,7 @@ KERNELS = {
     "gdn_prep_bf16_kernel": dict(bound="tensor", flops_per_token_head=flops_prep(), split=3),
     "gdn_plan_kernel": dict(bound="latency"),
     "gdn_decode_step_kernel": dict(bound="hbm"),
+    "gdn_decode_verify_kernel": dict(bound="hbm"),
 }
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from the last ncu capture of that kernel
 # on the bench workload (None until captured, and reset whenever the kernel changes).  The decode
@@ -240,7 +241,7 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     from linear_attention_10_b200 import gdn
-    from linear_attention_10_b200.workloads import WORKLOADS, make_decode_inputs, workload_inputs
+    from linear_attention_10_b200.workloads import WORKLOADS, make_decode_inputs, make_verify_inputs, workload_inputs
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -368,6 +369,47 @@ def run_ours(args, rank, world, local_rank):
                                     traffic=TRAFFIC.get(name)))
         del dd, S
 
+    # ---- multi-token verify: B=64 sequences x 4 drafted tokens, every per-token state written ----
+    verify = None
+    if not args.no_verify:
+        w = WORKLOADS["verify_b64_k4"]
+        B_, Tk, H_, d_ = w.decode_batch, w.decode_steps, w.H, w.dk
+        vd = make_verify_inputs(B_, H_, d_, d_, Tk, dtype=w.dtype, gate=w.gate, seed=w.seed + rank,
+                                state_std=w.state_std, device=dev)
+        vst = torch.empty((B_, Tk, H_, d_, d_), dtype=torch.float32, device=dev)
+        vout = torch.empty((B_, Tk, H_, d_), dtype=torch.bfloat16, device=dev)
+        run_v = lambda: gdn.gdn_decode_verify(vd["q"], vd["k"], vd["v"], vd["g"], vd["beta"], vd["state"],
+                                              states_out=vst, out=vout)
+        for _ in range(3):
+            run_v()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        reps = 100
+        gdn.gdn_profile_start()
+        v0, v1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        v0.record(stream)
+        for _ in range(reps):
+            run_v()
+        v1.record(stream)
+        torch.cuda.synchronize()
+        vprof = gdn.gdn_profile_stop()
+        vms = max_over_ranks(v0.elapsed_time(v1), world, dev)
+        name = "gdn_decode_verify_kernel"
+        kms, kl = vprof.get(name, (vms, reps))
+        per_bh = (1 + Tk) * d_ * d_ * 4 + Tk * ((3 * d_) * 2 + 2 * 4 + d_ * 2)
+        bytes_per_launch = B_ * H_ * per_bh
+        ach = bytes_per_launch / (kms / kl / 1e3) / 1e9
+        pk, pu, pdesc = peak_for("hbm", peaks)
+        verify = dict(workload="verify_b64_k4: B=64 sequences x 4 drafted tokens, H=32, dk=dv=128, bf16 q/k/v, "
+                               "fp32 state read once, 4 per-token states written",
+                      value=job_throughput(B_ * Tk, reps, world, vms), unit="tokens/s",
+                      us_per_call=vms / reps * 1e3,
+                      roofline=dict(kernel=name, bound="hbm", achieved=ach, peak=pk, unit=pu, frac=ach / pk,
+                                    peak_source=pdesc, bytes_per_launch=bytes_per_launch,
+                                    traffic=TRAFFIC.get(name)))
+        del vd, vst, vout
+
     clk = clocks.stop()
 
     # ---- roofline of the dominant prefill kernel ----
@@ -411,7 +453,7 @@ def run_ours(args, rank, world, local_rank):
                 roofline=roofline, method_roofline=method_roofline, cpu_baseline=cpu,
                 e2e=dict(value=e2e_value, unit=UNIT, h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                          steps=e2e_steps),
-                gpu_launches=launches, clocks=clk, decode=decode)
+                gpu_launches=launches, clocks=clk, decode=decode, verify=verify)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -423,6 +465,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-verify", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()

@@ -140,6 +140,28 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
                     int dtype, void* stream);
 
 /*
+ * Multi-token recurrent verify (Ferrite project page, Design section 04: drafted tokens are checked
+ * by the big model in one pass): Tk speculative tokens per sequence run through the recurrence in
+ * order, as a linear chain, starting from the committed state, which is only read.  The state after
+ * every token is returned, so that the caller keeps the one after the last accepted token (or the
+ * committed state when none is accepted) and discards the rest.  Token t of sequence b gives exactly
+ * what the t-th of Tk chained gdn_decode_step calls from state_in would give.
+ *
+ *   q, k          device [B, Tk, H, dk], dtype `dtype`
+ *   v             device [B, Tk, H, dv], dtype `dtype`
+ *   g, beta       device fp32 [B, Tk, H]
+ *   state_in      device fp32 [B, H, dv, dk]; read only
+ *   states_out    device fp32 [B, Tk, H, dv, dk]: S after token t at [b, t]; or NULL
+ *   out           device [B, Tk, H, dv] in dtype `dtype`, or NULL (at least one of the two)
+ *   Tk >= 1.  Memory: states_out holds Tk states per (b, h) (64 KB each at dk = dv = 128).
+ *   Errors as gdn_decode_step; GDN_ERR_INVALID_ARG also for Tk < 1 or both outputs NULL.
+ *   states_out and out must not alias the inputs.
+ */
+int gdn_decode_verify(const void* q, const void* k, const void* v, const float* g,
+                      const float* beta, const float* state_in, float* states_out, void* out, int B,
+                      int Tk, int H, int dk, int dv, int dtype, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of the current device:
  * GDN_OK, or the first device-detected error (GDN_ERR_BAD_SEQLENS, GDN_ERR_TIMEOUT) recorded since
  * the last read.  Returns GDN_ERR_CUDA when the synchronisation itself fails.

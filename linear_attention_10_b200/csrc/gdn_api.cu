@@ -108,6 +108,28 @@ static int dispatch_decode(const void* q, const void* k, const void* v, const fl
     return launch_decode<T, 64, 64>(q, k, v, g, beta, state, out, B, H, st);
 }
 
+template <typename T, int DK, int DV>
+static int launch_verify(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                         const float* state_in, float* states_out, void* out, int B, int Tk, int H, cudaStream_t st)
+{
+    ProfScope prof("gdn_decode_verify_kernel", st);
+    gdn_decode_verify_kernel<T, DK, DV><<<(unsigned)B * H, 256, 0, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g, beta, state_in, states_out,
+        static_cast<T*>(out), H, Tk);
+    return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
+}
+
+template <typename T>
+static int dispatch_verify(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                           const float* state_in, float* states_out, void* out, int B, int Tk, int H, int dk, int dv,
+                           cudaStream_t st)
+{
+    if (dk == 128 && dv == 128) return launch_verify<T, 128, 128>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, st);
+    if (dk == 128 && dv == 64) return launch_verify<T, 128, 64>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, st);
+    if (dk == 64 && dv == 128) return launch_verify<T, 64, 128>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, st);
+    return launch_verify<T, 64, 64>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, st);
+}
+
 // ---- tensor maps (2-D tiled views of q/k/v) -------------------------------------------------------
 // cuTensorMapEncodeTiled is taken from the driver through the runtime's entry-point query, so the
 // library does not link libcuda directly.
@@ -388,6 +410,27 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dtype == GDN_F32) return dispatch_decode<float>(q, k, v, g, beta, state_inout, out, B, H, dk, dv, st);
     return dispatch_decode<__nv_bfloat16>(q, k, v, g, beta, state_inout, out, B, H, dk, dv, st);
+}
+
+int gdn_decode_verify(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                      const float* state_in, float* states_out, void* out, int B, int Tk, int H, int dk, int dv,
+                      int dtype, void* stream)
+{
+    if (B < 0 || Tk < 1 || H < 1) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!head_ok(dk) || !head_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    if (B == 0) return GDN_OK;
+    if (!q || !k || !v || !g || !beta || !state_in) return GDN_ERR_INVALID_ARG;
+    if (!states_out && !out) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, state_in, states_out, out};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    if (!aligned4(g) || !aligned4(beta)) return GDN_ERR_MISALIGNED;
+    if ((int64_t)B * H > INT32_MAX || (int64_t)B * Tk * H > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == GDN_F32)
+        return dispatch_verify<float>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, dk, dv, st);
+    return dispatch_verify<__nv_bfloat16>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, dk, dv, st);
 }
 
 int gdn_get_device_status(void* stream)

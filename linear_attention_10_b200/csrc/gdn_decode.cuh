@@ -20,6 +20,40 @@
 
 namespace gdn {
 
+// One row r of S for one token: the two dot products S_r.k and S_r.q are reduced over the LPR
+// lanes that hold the row (float4 each), then S_r <- alpha S_r + u k with u = beta (v_r - alpha S_r.k),
+// and o_r = scale (alpha S_r.q + u (k.q)).  Shared by the single-step and the multi-token kernels so
+// that both perform the same operations in the same order.
+template <int LPR>
+__device__ __forceinline__ float4 decode_row_step(const float4 s, const float4 k4, const float4 q4, float alpha,
+                                                  float b, float vr, float kq, float scale, float& o)
+{
+    float sk = s.x * k4.x + s.y * k4.y + s.z * k4.z + s.w * k4.w;
+    float sq = s.x * q4.x + s.y * q4.y + s.z * q4.z + s.w * q4.w;
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) {
+        sk += __shfl_xor_sync(0xffffffffu, sk, off);
+        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    }
+    const float uu = b * (vr - alpha * sk);
+    float4 n;
+    n.x = fmaf(alpha, s.x, uu * k4.x);
+    n.y = fmaf(alpha, s.y, uu * k4.y);
+    n.z = fmaf(alpha, s.z, uu * k4.z);
+    n.w = fmaf(alpha, s.w, uu * k4.w);
+    o = scale * fmaf(alpha, sq, uu * kq);
+    return n;
+}
+
+template <int LPR>
+__device__ __forceinline__ float row_dot(const float4 a, const float4 b)
+{
+    float d = a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+    return d;
+}
+
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(256) gdn_decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                           const T* __restrict__ v, const float* __restrict__ g,
@@ -45,10 +79,7 @@ __global__ void __launch_bounds__(256) gdn_decode_step_kernel(const T* __restric
     const float b = __ldg(beta + bh);
     const float scale = rsqrtf((float)DK);
 
-    // k . q over the row's lanes
-    float kq = k4.x * q4.x + k4.y * q4.y + k4.z * q4.z + k4.w * q4.w;
-#pragma unroll
-    for (int o = LPR / 2; o > 0; o >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, o);
+    const float kq = row_dot<LPR>(k4, q4);      // k . q over the row's lanes
 
     float* S = state + (size_t)bh * DV * DK;
     const int row0 = warp * ROWS_PER_WARP;
@@ -64,23 +95,67 @@ __global__ void __launch_bounds__(256) gdn_decode_step_kernel(const T* __restric
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            float sk = s[u].x * k4.x + s[u].y * k4.y + s[u].z * k4.z + s[u].w * k4.w;
-            float sq = s[u].x * q4.x + s[u].y * q4.y + s[u].z * q4.z + s[u].w * q4.w;
-#pragma unroll
-            for (int o = LPR / 2; o > 0; o >>= 1) {
-                sk += __shfl_xor_sync(0xffffffffu, sk, o);
-                sq += __shfl_xor_sync(0xffffffffu, sq, o);
-            }
-            const float uu = b * (vr[u] - alpha * sk);
-            float4 n;
-            n.x = fmaf(alpha, s[u].x, uu * k4.x);
-            n.y = fmaf(alpha, s[u].y, uu * k4.y);
-            n.z = fmaf(alpha, s[u].z, uu * k4.z);
-            n.w = fmaf(alpha, s[u].w, uu * k4.w);
+            float o;
+            const float4 n = decode_row_step<LPR>(s[u], k4, q4, alpha, b, vr[u], kq, scale, o);
             const int r = row0 + base + u * RPW + sub;
             *reinterpret_cast<float4*>(S + (size_t)r * DK + col) = n;
-            if (out != nullptr && (lane % LPR) == 0)
-                Elem<T>::st(out + (size_t)bh * DV + r, scale * fmaf(alpha, sq, uu * kq));
+            if (out != nullptr && (lane % LPR) == 0) Elem<T>::st(out + (size_t)bh * DV + r, o);
+        }
+    }
+}
+
+// Multi-token recurrent verify: Tk draft tokens of one sequence run through the recurrence in order
+// (a linear chain of speculative tokens, Ferrite project page, Design section 04), starting from the
+// committed state, which is only read.  The state after every token is written to states_out, so
+// that the caller keeps the one after the last accepted token and drops the rest.
+//
+// Mapping: one CTA (8 warps) per (b, h); the whole dv x dk state of the pair lives in registers for
+// the Tk tokens (each lane holds NR float4s of its rows), is read from HBM once and written Tk times.
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(256) gdn_decode_verify_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                            const T* __restrict__ v, const float* __restrict__ g,
+                                                            const float* __restrict__ beta,
+                                                            const float* __restrict__ state_in,
+                                                            float* __restrict__ states_out, T* __restrict__ out,
+                                                            int H, int Tk)
+{
+    constexpr int LPR = DK / 4;               // lanes per row
+    constexpr int RPW = 32 / LPR;             // rows handled by one warp at once
+    constexpr int ROWS_PER_WARP = DV / 8;
+    constexpr int NR = ROWS_PER_WARP / RPW;   // rows held by one lane
+    static_assert(ROWS_PER_WARP % RPW == 0, "row split");
+
+    const int bh = blockIdx.x;                // b * H + h
+    const int b = bh / H, h = bh - b * H;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane / LPR;
+    const int col = (lane % LPR) * 4;
+    const int row0 = warp * ROWS_PER_WARP + sub;
+    const float scale = rsqrtf((float)DK);
+
+    float4 s[NR];
+    const float* S0 = state_in + (size_t)bh * DV * DK;
+#pragma unroll
+    for (int u = 0; u < NR; ++u) s[u] = *reinterpret_cast<const float4*>(S0 + (size_t)(row0 + u * RPW) * DK + col);
+
+    for (int t = 0; t < Tk; ++t) {
+        const size_t tok = ((size_t)b * Tk + t) * H + h;      // index into [B, Tk, H]
+        const float4 k4 = Elem<T>::ld4(k + tok * DK + col);
+        const float4 q4 = Elem<T>::ld4(q + tok * DK + col);
+        const float alpha = expf(__ldg(g + tok));
+        const float bb = __ldg(beta + tok);
+        const float kq = row_dot<LPR>(k4, q4);
+        float vr[NR];
+#pragma unroll
+        for (int u = 0; u < NR; ++u) vr[u] = Elem<T>::ld(v + tok * DV + row0 + u * RPW);
+        float* St = states_out ? states_out + tok * DV * DK : nullptr;
+#pragma unroll
+        for (int u = 0; u < NR; ++u) {
+            const int r = row0 + u * RPW;
+            float o;
+            s[u] = decode_row_step<LPR>(s[u], k4, q4, alpha, bb, vr[u], kq, scale, o);
+            if (St) *reinterpret_cast<float4*>(St + (size_t)r * DK + col) = s[u];
+            if (out != nullptr && (lane % LPR) == 0) Elem<T>::st(out + tok * DV + r, o);
         }
     }
 }

@@ -27,6 +27,7 @@ EXPORTS = (
     "gdn_chunk_prefill",
     "gdn_chunk_prefill_noalloc",
     "gdn_decode_step",
+    "gdn_decode_verify",
     "gdn_get_device_status",
     "gdn_profile_start",
     "gdn_profile_stop",
@@ -64,6 +65,8 @@ def lib() -> ctypes.CDLL:
     L.gdn_chunk_prefill_noalloc.restype = i32
     L.gdn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
     L.gdn_decode_step.restype = i32
+    L.gdn_decode_verify.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
+    L.gdn_decode_verify.restype = i32
     L.gdn_get_device_status.argtypes = [vp]
     L.gdn_get_device_status.restype = i32
     L.gdn_profile_start.argtypes = []
@@ -174,6 +177,34 @@ def gdn_decode_step(q, k, v, g, beta, state, out=None, stream=None):
     if rc != 0:
         raise GdnError(rc, "gdn_decode_step")
     return out
+
+
+def gdn_decode_verify(q, k, v, g, beta, state_in, states_out=None, out=None, want_states=True, stream=None):
+    """Tk speculative tokens per sequence through the recurrence: q, k ``[B, Tk, H, dk]``, v
+    ``[B, Tk, H, dv]``, g, beta ``[B, Tk, H]``, state_in fp32 ``[B, H, dv, dk]`` (read only).
+    Returns ``(out [B, Tk, H, dv], states_out [B, Tk, H, dv, dk] or None)``."""
+    B, Tk, H, dk = q.shape
+    dv = v.shape[3]
+    dev, dt = q.device, q.dtype
+    _check(q, "q", (B, Tk, H, dk), dt, dev)
+    _check(k, "k", (B, Tk, H, dk), dt, dev)
+    _check(v, "v", (B, Tk, H, dv), dt, dev)
+    _check(g, "g", (B, Tk, H), torch.float32, dev)
+    _check(beta, "beta", (B, Tk, H), torch.float32, dev)
+    _check(state_in, "state_in", (B, H, dv, dk), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, Tk, H, dv), dtype=dt, device=dev)
+    _check(out, "out", (B, Tk, H, dv), dt, dev)
+    if states_out is None and want_states:
+        states_out = torch.empty((B, Tk, H, dv, dk), dtype=torch.float32, device=dev)
+    if states_out is not None:
+        _check(states_out, "states_out", (B, Tk, H, dv, dk), torch.float32, dev)
+    rc = lib().gdn_decode_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
+                                 None if states_out is None else _ptr(states_out), _ptr(out),
+                                 B, Tk, H, dk, dv, _dtype_code(q), _stream_ptr(stream))
+    if rc != 0:
+        raise GdnError(rc, "gdn_decode_verify")
+    return out, states_out
 
 
 def gdn_get_device_status(stream=None) -> int:

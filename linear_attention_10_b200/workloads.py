@@ -25,7 +25,8 @@ from typing import List, Optional
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_prefill_inputs", "make_decode_inputs", "cu_seqlens_of"]
+__all__ = ["Workload", "WORKLOADS", "make_prefill_inputs", "make_decode_inputs", "make_verify_inputs",
+           "cu_seqlens_of"]
 
 
 @dataclass(frozen=True)
@@ -55,6 +56,9 @@ WORKLOADS = {
     "long_128k": Workload("long_128k", [131072]),
     "decode_b64": Workload("decode_b64", [], dtype="bf16", gate="uniform", state_std=0.05,
                            decode_batch=64, decode_steps=1000),
+    # speculative verify: 4 drafted tokens for each of 64 sequences, the decode_b64 distributions
+    "verify_b64_k4": Workload("verify_b64_k4", [], dtype="bf16", gate="uniform", state_std=0.05,
+                              decode_batch=64, decode_steps=4),
 }
 
 
@@ -123,6 +127,15 @@ def make_decode_inputs(B, H, dk, dv, steps, dtype="bf16", gate="uniform", seed=0
     g = _gate(gen, (steps, B, H), gate, device)
     beta = torch.sigmoid(torch.randn((steps, B, H), generator=gen, device=device))
     return dict(q=q, k=k, v=v, g=g, beta=beta, state=state)
+
+
+def make_verify_inputs(B, H, dk, dv, Tk, dtype="bf16", gate="uniform", seed=0, state_std=0.05, device="cpu"):
+    """Inputs of one multi-token verify: ``Tk`` drafted tokens for each of ``B`` sequences, laid out
+    ``[B, Tk, H, d]`` / ``[B, Tk, H]``, drawn as ``make_decode_inputs`` draws a chain of Tk steps."""
+    d = make_decode_inputs(B, H, dk, dv, Tk, dtype=dtype, gate=gate, seed=seed, state_std=state_std, device=device)
+    out = {n: d[n].transpose(0, 1).contiguous() for n in ("q", "k", "v", "g", "beta")}
+    out["state"] = d["state"]
+    return out
 
 
 def workload_inputs(name: str, device="cpu", seed=None):

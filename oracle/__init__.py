@@ -144,6 +144,23 @@ def decode_step(q, k, v, g, beta, state):
     return recurrence(q, k, v, g, beta, cu_seqlens=np.arange(B + 1), state_in=state)
 
 
+def decode_verify(q, k, v, g, beta, state):
+    """Tk speculative tokens per sequence run in order from ``state`` (which is not modified):
+    inputs ``[B, Tk, H, d]`` / ``[B, Tk, H]``.  Returns ``(out [B, Tk, H, dv], states [B, Tk, H, dv,
+    dk])`` with the state after each token -- the decode step applied Tk times."""
+    q, k, v, g, beta = (_d(x) for x in (q, k, v, g, beta))
+    B, Tk, H, dk = q.shape
+    dv = v.shape[3]
+    out = np.zeros((B, Tk, H, dv))
+    states = np.zeros((B, Tk, H, dv, dk))
+    S = _d(state).copy()
+    for t in range(Tk):
+        o, S = decode_step(q[:, t], k[:, t], v[:, t], g[:, t], beta[:, t], S)
+        out[:, t] = o
+        states[:, t] = S
+    return out, states
+
+
 def brute_force(q, k, v, g, beta, state_in=None):
     """Unrolled recurrence with explicit matrices, one sequence, T <= 8 (numpy, fp64).
 

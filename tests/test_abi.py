@@ -108,6 +108,27 @@ def test_decode_rejects_bad_arguments(L):
     assert decode(L, B=0) == 0                          # nothing to do, nothing enqueued
 
 
+def verify(L, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, s=FAKE, st=FAKE, out=FAKE, B=4, Tk=3, H=2, dk=128, dv=128,
+             dtype=1, stream=None)
+    a.update(kw)
+    return L.gdn_decode_verify(a["q"], a["k"], a["v"], a["g"], a["beta"], a["s"], a["st"], a["out"], a["B"],
+                               a["Tk"], a["H"], a["dk"], a["dv"], a["dtype"], a["stream"])
+
+
+def test_verify_rejects_bad_arguments(L):
+    assert verify(L, s=None) == -1
+    assert verify(L, st=None, out=None) == -1           # nothing to return
+    assert verify(L, Tk=0) == -1
+    assert verify(L, H=0) == -1
+    assert verify(L, B=-1) == -1
+    assert verify(L, dtype=3) == -1
+    assert verify(L, dv=96) == -2
+    assert verify(L, st=FAKE + 4) == -3
+    assert verify(L, beta=FAKE + 1) == -3
+    assert verify(L, B=0) == 0                          # nothing to do, nothing enqueued
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(gdn, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(gdn, "_lib", None)

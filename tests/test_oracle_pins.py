@@ -278,6 +278,37 @@ def test_decode_step_is_length_one_recurrence():
             assert rel(o[i, h], Sn @ q[i, h] / np.sqrt(d)) < 1e-13
 
 
+def test_decode_verify_states_match_brute_force():
+    """The state after each drafted token equals the explicit-matrix expansion over that prefix, and
+    the outputs are S_t q_t / sqrt(dk); the committed state is left untouched."""
+    B, Tk, H, d = 2, 5, 2, 6
+    r = np.random.default_rng(21)
+    q, k, v, g, b, _ = rnd(B * Tk, H, d, d, 22)
+    q, k, v = (x.reshape(B, Tk, H, d) for x in (q, k, v))
+    g, b = g.reshape(B, Tk, H), b.reshape(B, Tk, H)
+    s0 = 0.05 * r.standard_normal((B, H, d, d))
+    keep = s0.copy()
+    o, st = oracle.decode_verify(q, k, v, g, b, s0)
+    assert np.array_equal(s0, keep)
+    for i in range(B):
+        for t in range(Tk):
+            ob, sb = oracle.brute_force(q[i, :t + 1], k[i, :t + 1], v[i, :t + 1], g[i, :t + 1], b[i, :t + 1],
+                                        state_in=s0[i][None])
+            assert rel(st[i, t], sb[0]) < 1e-12
+            assert rel(o[i, t], ob[t]) < 1e-12
+
+
+def test_decode_verify_equals_one_sequence_per_draft_chain():
+    """Tk drafted tokens of B sequences = the recurrence over B sequences of Tk tokens each."""
+    B, Tk, H, d = 3, 7, 2, 8
+    q, k, v, g, b, _ = rnd(B * Tk, H, d, d, 23)
+    s0 = 0.05 * np.random.default_rng(24).standard_normal((B, H, d, d))
+    o, st = oracle.decode_verify(*(x.reshape((B, Tk) + x.shape[1:]) for x in (q, k, v, g, b)), s0)
+    o2, s2 = oracle.recurrence(q, k, v, g, b, cu_seqlens=np.arange(0, B * Tk + 1, Tk), state_in=s0)
+    assert rel(o.reshape(B * Tk, H, d), o2) < 1e-13
+    assert rel(st[:, -1], s2) < 1e-13
+
+
 # ---------------------------------------------------------------------------------------------
 # planted mistakes: each variant below is one plausible error; at least one pin must reject it
 # ---------------------------------------------------------------------------------------------
