@@ -56,7 +56,8 @@ enum {
     GDN_ERR_MISALIGNED = -3,   /* a pointer breaks the alignment rule above                     */
     GDN_ERR_LAUNCH = -4,       /* a kernel launch failed (the CUDA error is left pending)        */
     GDN_ERR_WORKSPACE = -5,    /* workspace missing, misaligned (256 B) or smaller than needed   */
-    GDN_ERR_BAD_SEQLENS = -6,  /* device-detected: cu_seqlens not 0..T_total non-decreasing     */
+    GDN_ERR_BAD_SEQLENS = -6,  /* device-detected: cu_seqlens not 0..T_total non-decreasing, or
+                                  cut points not increasing and strictly inside a sequence      */
     GDN_ERR_TIMEOUT = -7,      /* device-detected: a bounded wait inside a kernel expired        */
     GDN_ERR_CUDA = -8          /* a CUDA runtime call made by the library failed                */
 };
@@ -100,6 +101,30 @@ int gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* 
                       int64_t total_tokens, const float* state_in, void* out, float* state_out,
                       int H, int dk, int dv, int dtype, void* workspace, size_t workspace_bytes,
                       void* stream);
+
+/*
+ * Chunked prefill with state snapshots at cut points (Ferrite project page, Design section 07:
+ * conversations are snapshotted at turn boundaries, and prompts are cut at the same points with or
+ * without a resume).  Same as gdn_chunk_prefill, plus: for every cut point c_i, snapshots[i]
+ * receives the state of the sequence that contains c_i after its tokens before c_i.  Chunks restart
+ * at every cut, so each snapshot, every output and each final state are bit for bit what a call
+ * that stops at c_i and a second call resumed from that state would give.
+ *
+ *   cuts        device int32 [num_cuts] token offsets into the packed batch, strictly increasing,
+ *               each strictly inside one sequence (start < c < end); checked on the device
+ *               (GDN_ERR_BAD_SEQLENS, nothing written)
+ *   num_cuts    >= 1 (GDN_ERR_INVALID_ARG otherwise; use gdn_chunk_prefill for none)
+ *   snapshots   device fp32 [num_cuts, H, dv, dk], 16-byte aligned
+ *   workspace   at least gdn_chunk_prefill_workspace_bytes(total_tokens, num_seqs + num_cuts, H,
+ *               dk, dv) bytes (a cut adds a segment)
+ * Every other argument, and the error behaviour, as gdn_chunk_prefill.
+ */
+int gdn_chunk_prefill_cuts(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, const int32_t* cu_seqlens, int num_seqs,
+                           int64_t total_tokens, const int32_t* cuts, int num_cuts,
+                           const float* state_in, void* out, float* state_out, float* snapshots,
+                           int H, int dk, int dv, int dtype, void* workspace,
+                           size_t workspace_bytes, void* stream);
 
 /*
  * gdn_chunk_prefill without a caller-provided workspace.  The pages have no counterpart to this

@@ -176,11 +176,18 @@ static bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uin
 
 static int g_num_sms = 0;
 
+// cut points of one prefill call and where their state snapshots go (n = 0: none)
+struct Cuts {
+    const int32_t* pos = nullptr;
+    int n = 0;
+    float* snaps = nullptr;
+};
+
 template <typename T, int DK, int DV>
 static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, const void* k, const void* v,
                           const float* g, const float* beta, const int32_t* cu, int N, int64_t T_total,
                           int fixed_len, const float* state_in, void* out, float* state_out, int H,
-                          cudaStream_t st)
+                          const Cuts& cuts, cudaStream_t st)
 {
     int* status = status_ptr();
     if (!status) return GDN_ERR_CUDA;
@@ -188,6 +195,7 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
     int* chunk_off = reinterpret_cast<int*>(ws + lay.off_chunk_off);
     int4* chunk_tab = reinterpret_cast<int4*>(ws + lay.off_chunk_tab);
     float* op = reinterpret_cast<float*>(ws + lay.off_op);
+    int* seg = reinterpret_cast<int*>(ws + lay.off_seg);
     if (g_num_sms == 0) {
         int dev = 0;
         cudaGetDevice(&dev);
@@ -196,7 +204,8 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
 
     {
         ProfScope prof("gdn_plan_kernel", st);
-        gdn_plan_kernel<<<1, 1024, 0, st>>>(cu, N, T_total, fixed_len, meta, chunk_off, chunk_tab, status);
+        gdn_plan_kernel<<<1, 1024, 0, st>>>(cu, N, T_total, fixed_len, cuts.pos, cuts.n, meta, chunk_off, chunk_tab,
+                                            seg, status);
     }
     if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
 
@@ -245,14 +254,14 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         using SB = ScanBf16Smem<DK, MSB, ST>;
         static_assert(SB3::kBytes <= 227 * 1024, "bf16 scan shared memory");
         static_assert(MSB == 32, "the V tensor map boxes 32 columns");
-        auto kb = gdn_scan_bf16_kernel<DK, DV, MSB, ST>;
+        auto kb = cuts.n > 0 ? gdn_scan_bf16_kernel<DK, DV, MSB, ST, true> : gdn_scan_bf16_kernel<DK, DV, MSB, ST, false>;
         if (cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SB::kBytes) != cudaSuccess)
             return GDN_ERR_LAUNCH;
         {
             ProfScope prof("gdn_scan_bf16_kernel", st);
             kb<<<dim3((unsigned)N, H, DV / MSB), kScanBf16Threads, SB::kBytes, st>>>(
                 tq, tk, tv, meta, chunk_off, chunk_tab, reinterpret_cast<const uint8_t*>(op), state_in,
-                static_cast<__nv_bfloat16*>(out), state_out, H, status);
+                static_cast<__nv_bfloat16*>(out), state_out, cuts.snaps, H, status);
         }
         return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
     }
@@ -271,7 +280,7 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         ProfScope prof("gdn_scan_tc_kernel", st);
         k2<<<dim3((unsigned)N, H, DV / MS), 256, SL::kBytes, st>>>(
             static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), meta, chunk_off,
-            chunk_tab, op, state_in, static_cast<T*>(out), state_out, H, status);
+            chunk_tab, op, state_in, static_cast<T*>(out), state_out, cuts.snaps, H, status);
     }
     return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
 }
@@ -280,12 +289,12 @@ template <typename T>
 static int dispatch_prefill(int dk, int dv, const PrefillLayout& lay, char* ws, const void* q, const void* k,
                             const void* v, const float* g, const float* beta, const int32_t* cu, int N,
                             int64_t T_total, int fixed_len, const float* state_in, void* out,
-                            float* state_out, int H, cudaStream_t st)
+                            float* state_out, int H, const Cuts& cuts, cudaStream_t st)
 {
 #define GDN_PF(DK_, DV_)                                                                                   \
     if (dk == DK_ && dv == DV_)                                                                            \
         return launch_prefill<T, DK_, DV_>(lay, ws, q, k, v, g, beta, cu, N, T_total, fixed_len, state_in, \
-                                           out, state_out, H, st);
+                                           out, state_out, H, cuts, st);
     GDN_PF(128, 128)
     GDN_PF(128, 64)
     GDN_PF(64, 128)
@@ -315,6 +324,40 @@ static void* noalloc_scratch_ptr()
         cache[dev] = p;
     }
     return cache[dev];
+}
+
+static int chunk_prefill(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                         const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens, const float* state_in,
+                         void* out, float* state_out, int H, int dk, int dv, int dtype, const Cuts& cuts,
+                         void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (num_seqs < 1 || H < 1 || total_tokens < 0 || total_tokens > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (cuts.n < 0 || (cuts.n > 0 && (!cuts.pos || !cuts.snaps))) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)num_seqs + cuts.n > INT32_MAX / 8) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!head_ok(dk) || !head_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return GDN_ERR_INVALID_ARG;
+    int fixed_len = 0;
+    if (!cu_seqlens) {
+        if (total_tokens % num_seqs != 0) return GDN_ERR_INVALID_ARG;
+        fixed_len = (int)(total_tokens / num_seqs);
+    }
+    const void* ptrs[] = {q, k, v, state_in, out, state_out, cuts.snaps};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    const void* small[] = {g, beta, cu_seqlens, cuts.pos};
+    for (const void* p : small)
+        if (p && !aligned4(p)) return GDN_ERR_MISALIGNED;
+    PrefillLayout lay(total_tokens, num_seqs + cuts.n, H, dk);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < lay.total)
+        return GDN_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    if (dtype == GDN_F32)
+        return dispatch_prefill<float>(dk, dv, lay, ws, q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
+                                       fixed_len, state_in, out, state_out, H, cuts, st);
+    return dispatch_prefill<__nv_bfloat16>(dk, dv, lay, ws, q, k, v, g, beta, cu_seqlens, num_seqs,
+                                           total_tokens, fixed_len, state_in, out, state_out, H, cuts, st);
 }
 
 }  // namespace gdn
@@ -352,31 +395,22 @@ int gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* 
                       void* out, float* state_out, int H, int dk, int dv, int dtype, void* workspace,
                       size_t workspace_bytes, void* stream)
 {
-    if (num_seqs < 1 || H < 1 || total_tokens < 0 || total_tokens > INT32_MAX) return GDN_ERR_INVALID_ARG;
-    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
-    if (!head_ok(dk) || !head_ok(dv)) return GDN_ERR_UNSUPPORTED;
-    if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return GDN_ERR_INVALID_ARG;
-    int fixed_len = 0;
-    if (!cu_seqlens) {
-        if (total_tokens % num_seqs != 0) return GDN_ERR_INVALID_ARG;
-        fixed_len = (int)(total_tokens / num_seqs);
-    }
-    const void* ptrs[] = {q, k, v, state_in, out, state_out};
-    for (const void* p : ptrs)
-        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
-    const void* small[] = {g, beta, cu_seqlens};
-    for (const void* p : small)
-        if (p && !aligned4(p)) return GDN_ERR_MISALIGNED;
-    PrefillLayout lay(total_tokens, num_seqs, H, dk);
-    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < lay.total)
-        return GDN_ERR_WORKSPACE;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    char* ws = static_cast<char*>(workspace);
-    if (dtype == GDN_F32)
-        return dispatch_prefill<float>(dk, dv, lay, ws, q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
-                                       fixed_len, state_in, out, state_out, H, st);
-    return dispatch_prefill<__nv_bfloat16>(dk, dv, lay, ws, q, k, v, g, beta, cu_seqlens, num_seqs,
-                                           total_tokens, fixed_len, state_in, out, state_out, H, st);
+    return chunk_prefill(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, state_in, out, state_out, H, dk, dv,
+                         dtype, Cuts{}, workspace, workspace_bytes, stream);
+}
+
+int gdn_chunk_prefill_cuts(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                           const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens, const int32_t* cuts,
+                           int num_cuts, const float* state_in, void* out, float* state_out, float* snapshots,
+                           int H, int dk, int dv, int dtype, void* workspace, size_t workspace_bytes, void* stream)
+{
+    Cuts c;
+    c.pos = cuts;
+    c.n = num_cuts;
+    c.snaps = snapshots;
+    if (num_cuts < 1) return GDN_ERR_INVALID_ARG;
+    return chunk_prefill(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, state_in, out, state_out, H, dk, dv,
+                         dtype, c, workspace, workspace_bytes, stream);
 }
 
 int gdn_chunk_prefill_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,

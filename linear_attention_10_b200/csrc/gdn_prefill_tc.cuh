@@ -493,7 +493,8 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                                                              const int4* __restrict__ chunk_tab,
                                                              const float* __restrict__ op,
                                                              const float* state_in, T* __restrict__ out,
-                                                             float* state_out, int H, int* status)
+                                                             float* state_out, float* __restrict__ snaps, int H,
+                                                             int* status)
 {
     using namespace sm100;
     using L = ScanSmem<T, DK, MS, STAGES>;
@@ -518,13 +519,6 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c_begin = chunk_off[n], c_end = chunk_off[n + 1];
     const int nch = c_end - c_begin;
-    // chunks of a sequence are consecutive 32-row blocks from its first token
-    int64_t seq_t0 = 0, seq_end = 0;
-    if (nch > 0) {
-        const int4 first = chunk_tab[c_begin], last = chunk_tab[c_end - 1];
-        seq_t0 = first.y;
-        seq_end = (int64_t)last.y + last.z;
-    }
 
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -561,8 +555,9 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
         };
         auto load_chunk = [&](Pre& p, int cl) {
             const int gc = c_begin + cl;
-            const int64_t t0 = seq_t0 + (int64_t)cl * kChunk;
-            const int Lr = (int)((seq_end - t0) < kChunk ? (seq_end - t0) : kChunk);
+            const int4 ctab = chunk_tab[gc];
+            const int64_t t0 = ctab.y;
+            const int Lr = ctab.z;
 #pragma unroll
             for (int u = 0; u < NB; ++u) {
                 const int b = ptid + 128 * u;
@@ -715,8 +710,9 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
             GDN_SCAN_TRACE(cl, 13);
             if (*abort_flag) { aborted = true; break; }
             tc_fence_after();
-            const int64_t t0 = seq_t0 + (int64_t)cl * kChunk;
-            const int Lr = (int)((seq_end - t0) < kChunk ? (seq_end - t0) : kChunk);
+            const int4 ctab = chunk_tab[c_begin + cl];
+            const int64_t t0 = ctab.y;
+            const int Lr = ctab.z;
             const float* gate = stf + L::oGate / 4;
             const float* Vs = stf + L::oV / 4;
             const float Gam = (lane < 16) ? gate[tok] : 0.f;
@@ -828,6 +824,12 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < MS; ++i) S[i] = fmaf(GamC, S[i], ds[i] + dl[i]);
+                // the state at a cut point the caller asked a snapshot of
+                const int snap = chunk_tab[c_begin + cl].w;
+                if (snap >= 0 && snaps != nullptr && owns) {
+#pragma unroll
+                    for (int i = 0; i < MS; ++i) snaps[(((size_t)snap * H + h) * DV + r0 + i) * DK + c_own] = S[i];
+                }
             }
             GDN_SCAN_TRACE(cl, 9);
             tc_fence_before();

@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
     auto issue_prev = [&](int item) {
         const int gc = item / H, h = item % H;
         const int t0 = chunk_tab[gc].y;
-        const int tp = has_prev(gc) ? t0 - kChunk : t0;
+        const int tp = has_prev(gc) ? chunk_tab[gc - 1].y : t0;    // the previous chunk may end at a cut
         mbar_arrive_expect_tx(prev_full, NP * 4096);
 #pragma unroll
         for (int p = 0; p < NP; ++p) tma_load_2d(sbase + L::oPrev + p * 4096, &tm_k, h * DK + p * 64, tp, prev_full);

@@ -54,7 +54,8 @@ struct ScanBf16Smem {
     // one stage
     static constexpr uint32_t oAKQ = 0;                               // [K;Q] bf16: NP panels x 64 rows x 128 B
     static constexpr uint32_t oOp = oAKQ + NP * 8192;                 // operator record: parts, G' parts, gates
-    static constexpr uint32_t oV = oOp + ((kOpBCopyBytes + 1023) & ~1023u);  // V tile: 32 rows x MS bf16
+    static constexpr uint32_t oCt = oOp + ((kOpBCopyBytes + 15) & ~15u);    // the chunk's table entry (int4)
+    static constexpr uint32_t oV = oOp + ((kOpBCopyBytes + 16 + 1023) & ~1023u);  // V tile: 32 rows x MS bf16
     static constexpr uint32_t kStage = ((oV + 32 * MS * 2) + 1023) & ~1023u;
     static constexpr uint32_t kStageTx = NP * 2 * 4096 + kOpBCopyBytes + 32 * MS * 2;
     // shared by all stages
@@ -95,13 +96,15 @@ __device__ __forceinline__ void put_parts(uint32_t tile, uint32_t lbo, int k, in
     }
 }
 
-template <int DK, int DV, int MS, int STAGES>
+// CUTS: the call has cut points (segments, snapshots); without them chunk c of a sequence starts at
+// its token 32 c and only chunk 0 starts a segment.
+template <int DK, int DV, int MS, int STAGES, bool CUTS>
 __global__ void __launch_bounds__(kScanBf16Threads, 1)
     gdn_scan_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const int* __restrict__ meta,
                          const int* __restrict__ chunk_off, const int4* __restrict__ chunk_tab,
                          const uint8_t* __restrict__ op, const float* state_in, __nv_bfloat16* __restrict__ out,
-                         float* state_out, int H, int* status)
+                         float* state_out, float* __restrict__ snaps, int H, int* status)
 {
     using namespace sm100;
     using L = ScanBf16Smem<DK, MS, STAGES>;
@@ -131,7 +134,7 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
     const int c_begin = chunk_off[n], c_end = chunk_off[n + 1];
     const int nch = c_end - c_begin;
     int64_t seq_t0 = 0, seq_end = 0;
-    if (nch > 0) {
+    if (!CUTS && nch > 0) {
         const int4 first = chunk_tab[c_begin], last = chunk_tab[c_end - 1];
         seq_t0 = first.y;
         seq_end = (int64_t)last.y + last.z;
@@ -169,6 +172,10 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
     auto stage_of = [](int c) { return c % STAGES; };
     auto phase_of = [](int c) { return (uint32_t)(c / STAGES) & 1u; };
 
+    // a chunk that starts a segment (its sequence's first, or the first after a cut point) takes its
+    // [X; Z] from the exact state before it, as a call resumed at the cut would
+    auto seg_first = [&](int c) { return c == 0 || (CUTS && chunk_tab[c_begin + c - 1].w >= 0); };
+
     const bool chain = warp < 8 && (warp & 3) < 2;
     const bool sgrp = (warp < 8) ? ((warp & 3) >= 2) : (warp == 8 || warp == 9 || warp == 12 || warp == 13);
 
@@ -183,7 +190,13 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
                     break;
                 }
                 const uint32_t st = sbase + s * L::kStage;
-                const int t0 = (int)(seq_t0 + (int64_t)cl * kChunk);
+                int t0 = (int)(seq_t0 + (int64_t)cl * kChunk);
+                if constexpr (CUTS) {
+                    const int4 ct = chunk_tab[c_begin + cl];
+                    t0 = ct.y;
+                    // the entry travels with the stage (published by the arrive below)
+                    *reinterpret_cast<int4*>(sm + s * L::kStage + L::oCt) = ct;
+                }
                 const int gc = c_begin + cl;
                 mbar_arrive_expect_tx(&full[s], L::kStageTx);
 #pragma unroll
@@ -207,7 +220,11 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
         const uint32_t lane_q = (uint32_t)(q4 * 32) << 16;
         const float scale = rsqrtf((float)DK);
         float GamPrev = 1.f;
+        int nx = 0;                           // MMA_x products waited for so far
+        // chunk-table entries travel in registers, the next one loaded a chunk ahead
+        int prev_w = -1;
         for (int c = 0; c < nch; ++c) {
+            const bool first = (c == 0) || (CUTS && prev_w >= 0);
             const int s = stage_of(c);
             const uint32_t st = sbase + s * L::kStage;
             const uint8_t* stp = sm + s * L::kStage;
@@ -215,12 +232,29 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
             bool ok = mbar_wait(&full[s], phase_of(c), abort_flag) &&
                       mbar_wait(&bar_w[c & 1], (uint32_t)(c >> 1) & 1u, abort_flag);
             GDN_SCAN_TRACE(c, 1);
-            if (ok && c > 0) ok = mbar_wait(bar_x, (uint32_t)(c - 1) & 1u, abort_flag);
+            // MMA_x of this chunk (which also covers MMA_c of the last one) or, at a segment start,
+            // MMA_c of the last chunk alone
+            if constexpr (CUTS) {
+                if (ok && c > 0) ok = first ? mbar_wait(bar_c, (uint32_t)(c - 1) & 1u, abort_flag)
+                                            : mbar_wait(bar_x, (uint32_t)nx & 1u, abort_flag);
+                if (c > 0 && !first) ++nx;
+            } else {
+                if (ok && c > 0) ok = mbar_wait(bar_x, (uint32_t)(c - 1) & 1u, abort_flag);
+            }
             if (!ok) tc_abort(status, abort_flag);
             GDN_SCAN_TRACE(c, 2);
             tc_fence_after();
-            const int64_t t0 = seq_t0 + (int64_t)c * kChunk;
-            const int Lr = (int)((seq_end - t0) < kChunk ? (seq_end - t0) : kChunk);
+            int64_t t0;
+            int Lr, ctab_w = -1;
+            if constexpr (CUTS) {
+                const int4 ctab = *reinterpret_cast<const int4*>(stp + L::oCt);
+                t0 = ctab.y;
+                Lr = ctab.z;
+                ctab_w = ctab.w;
+            } else {
+                t0 = seq_t0 + (int64_t)c * kChunk;
+                Lr = (int)((seq_end - t0) < kChunk ? (seq_end - t0) : kChunk);
+            }
             const float* gate = reinterpret_cast<const float*>(stp + L::oOp + kOpBGate);
             const float Gam = gate[lane];
             const float del = gate[32 + lane];
@@ -233,7 +267,7 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
                 tmem_ld<MH>(tw, w1);
                 tmem_ld<MH>(tw + MS, w2);
                 tmem_ld<MH>(tw + 2 * MS, w3);
-                if (c > 0) {
+                if (!first) {
                     float x1[MH], x2[MH], x3[MH];
                     const uint32_t tx = tD1 + lane_q + hf * MH;
                     tmem_ld<MH>(tx, x1);
@@ -329,7 +363,7 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
                     mma_commit(bar_c);
                     GDN_SCAN_TRACE(c, 9);
                     // ---- MMA_x of the next chunk: D1 = G'_{c+1} U~_c
-                    if (c + 1 < nch) {
+                    if (c + 1 < nch && (!CUTS || ctab_w < 0)) {
                         const int s1 = stage_of(c + 1);
                         ok2 = mbar_wait(&full[s1], phase_of(c + 1), abort_flag);
                         GDN_SCAN_TRACE(c, 10);
@@ -351,6 +385,7 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
                 GDN_SCAN_TRACE(c, 7);
             }
             GamPrev = GamC;
+            prev_w = ctab_w;
         }
     } else if (sgrp) {
         // ------------------------------------------------------------------ state warps
@@ -380,22 +415,35 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
             return true;
         };
 
+        int last_w = 0;                       // the last W issued (it reads the state's parts)
         bool aborted = false;
         if (nch > 0) {
-            // the initial state serves both W_0 and W_1
+            // the initial state serves W_0 and (unless a cut follows chunk 0) W_1
             if (owns) put_parts<MS, MH>(sbase + L::oBS, L::kLboS, c_own, hf, S);
             fence_async_smem();
             tc_fence_before();
             named_bar(3, 256);
             if (lead) {
                 tc_fence_after();
-                if (!issue_w(0) || (nch > 1 && !issue_w(1))) tc_abort(status, abort_flag);
+                if (!issue_w(0) || (nch > 1 && !seg_first(1) && !issue_w(1))) tc_abort(status, abort_flag);
             }
+            last_w = (nch > 1 && !seg_first(1)) ? 1 : 0;
         }
         for (int j = 0; j < nch; ++j) {
             const int s = stage_of(j);
-            if (!mbar_wait(&full[s], phase_of(j), abort_flag) || !mbar_wait(bar_c, (uint32_t)j & 1u, abort_flag))
-                tc_abort(status, abort_flag);
+            // snapshot indices of chunks j and j + 1 (a segment ends after a chunk with one), from
+            // the chunk-table entries that travel with the stages
+            int w_cur = -1, w_next = -1;
+            if constexpr (CUTS) {
+                const bool okw = mbar_wait(&full[s], phase_of(j), abort_flag) &&
+                                 (j + 1 >= nch || mbar_wait(&full[stage_of(j + 1)], phase_of(j + 1), abort_flag));
+                if (!okw || !mbar_wait(bar_c, (uint32_t)j & 1u, abort_flag)) tc_abort(status, abort_flag);
+                w_cur = reinterpret_cast<const int4*>(sm + s * L::kStage + L::oCt)->w;
+                if (j + 1 < nch) w_next = reinterpret_cast<const int4*>(sm + stage_of(j + 1) * L::kStage + L::oCt)->w;
+            } else {
+                if (!mbar_wait(&full[s], phase_of(j), abort_flag) || !mbar_wait(bar_c, (uint32_t)j & 1u, abort_flag))
+                    tc_abort(status, abort_flag);
+            }
             if (lead) GDN_SCAN_TRACE(j, 12);
             tc_fence_after();
             {
@@ -409,6 +457,13 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < MH; ++i) S[i] = fmaf(GamC, S[i], (d1[i] + d2[i]) + d3[i]);
+                // the state at a cut point the caller asked a snapshot of
+                const int snap = w_cur;
+                if (CUTS && snap >= 0 && snaps != nullptr && owns) {
+#pragma unroll
+                    for (int ii = 0; ii < MH; ++ii)
+                        snaps[(((size_t)snap * H + h) * DV + r0 + hf * MH + ii) * DK + c_own] = S[ii];
+                }
             }
             tc_fence_before();
             if (named_bar_any(3, 256, *abort_flag)) { aborted = true; break; }
@@ -418,7 +473,26 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
                 mbar_arrive(&empty[s]);
                 GDN_SCAN_TRACE(j, 13);
             }
-            if (j + 2 < nch) {
+            if constexpr (CUTS) {
+                // W_{j+1} when chunk j+1 starts a segment (from the exact state S_j), and W_{j+2} one
+                // chunk ahead unless chunk j+2 starts a segment (then it waits for S_{j+1})
+                const bool wa = (j + 1 < nch) && w_cur >= 0;
+                const bool wb = (j + 2 < nch) && w_next < 0;
+                if (wa || wb) {
+                    // once the last W issued has finished reading the previous state's parts
+                    if (!mbar_wait(&bar_w[last_w & 1], (uint32_t)(last_w >> 1) & 1u, abort_flag))
+                        tc_abort(status, abort_flag);
+                    if (owns) put_parts<MS, MH>(sbase + L::oBS, L::kLboS, c_own, hf, S);
+                    fence_async_smem();
+                    tc_fence_before();
+                    if (named_bar_any(3, 256, *abort_flag)) { aborted = true; break; }
+                    if (lead) {
+                        tc_fence_after();
+                        if ((wa && !issue_w(j + 1)) || (wb && !issue_w(j + 2))) tc_abort(status, abort_flag);
+                    }
+                    last_w = wb ? j + 2 : j + 1;
+                }
+            } else if (j + 2 < nch) {
                 // once W_{j+1} has finished reading the previous state's parts
                 if (!mbar_wait(&bar_w[(j + 1) & 1], (uint32_t)((j + 1) >> 1) & 1u, abort_flag))
                     tc_abort(status, abort_flag);

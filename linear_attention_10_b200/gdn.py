@@ -25,6 +25,7 @@ EXPORTS = (
     "gdn_version",
     "gdn_chunk_prefill_workspace_bytes",
     "gdn_chunk_prefill",
+    "gdn_chunk_prefill_cuts",
     "gdn_chunk_prefill_noalloc",
     "gdn_decode_step",
     "gdn_decode_verify",
@@ -61,6 +62,9 @@ def lib() -> ctypes.CDLL:
     L.gdn_chunk_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, i32, i32,
                                     vp, sz, vp]
     L.gdn_chunk_prefill.restype = i32
+    L.gdn_chunk_prefill_cuts.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, i32, vp, vp, vp, vp, i32, i32, i32,
+                                         i32, vp, sz, vp]
+    L.gdn_chunk_prefill_cuts.restype = i32
     L.gdn_chunk_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, i32, i32, vp]
     L.gdn_chunk_prefill_noalloc.restype = i32
     L.gdn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
@@ -155,6 +159,50 @@ def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens=None, state_in=None, out=None
     if rc != 0:
         raise GdnError(rc, "gdn_chunk_prefill")
     return out, state_out
+
+
+def gdn_chunk_prefill_cuts(q, k, v, g, beta, cuts, cu_seqlens=None, state_in=None, out=None, state_out=None,
+                           snapshots=None, workspace=None, num_seqs: Optional[int] = None, stream=None,
+                           output_final_state=True):
+    """``gdn_chunk_prefill`` that also returns the state at each cut point: ``cuts`` int32 ``[n]`` on
+    the device (strictly increasing token offsets, each strictly inside a sequence).  Returns
+    ``(out, state_out, snapshots [n, H, dv, dk])``."""
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    dev = q.device
+    dt = q.dtype
+    N = (cu_seqlens.numel() - 1) if cu_seqlens is not None else int(num_seqs or 1)
+    nc = int(cuts.numel())
+    _check(q, "q", (T, H, dk), dt, dev)
+    _check(k, "k", (T, H, dk), dt, dev)
+    _check(v, "v", (T, H, dv), dt, dev)
+    _check(g, "g", (T, H), torch.float32, dev)
+    _check(beta, "beta", (T, H), torch.float32, dev)
+    _check(cuts, "cuts", (nc,), torch.int32, dev)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", (N + 1,), torch.int32, dev)
+    if state_in is not None:
+        _check(state_in, "state_in", (N, H, dv, dk), torch.float32, dev)
+    if out is None:
+        out = torch.empty((T, H, dv), dtype=dt, device=dev)
+    _check(out, "out", (T, H, dv), dt, dev)
+    if state_out is None and output_final_state:
+        state_out = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+    if state_out is not None:
+        _check(state_out, "state_out", (N, H, dv, dk), torch.float32, dev)
+    if snapshots is None:
+        snapshots = torch.empty((max(nc, 1), H, dv, dk), dtype=torch.float32, device=dev)[:nc]
+    _check(snapshots, "snapshots", (nc, H, dv, dk), torch.float32, dev)
+    need = workspace_bytes(T, N + nc, H, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    rc = lib().gdn_chunk_prefill_cuts(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, T,
+                                      _ptr(cuts), nc, _ptr(state_in), _ptr(out), _ptr(state_out), _ptr(snapshots),
+                                      H, dk, dv, _dtype_code(q), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if rc != 0:
+        raise GdnError(rc, "gdn_chunk_prefill_cuts")
+    return out, state_out, snapshots
 
 
 def gdn_decode_step(q, k, v, g, beta, state, out=None, stream=None):

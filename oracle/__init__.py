@@ -144,6 +144,35 @@ def decode_step(q, k, v, g, beta, state):
     return recurrence(q, k, v, g, beta, cu_seqlens=np.arange(B + 1), state_in=state)
 
 
+def states_at(q, k, v, g, beta, cuts, cu_seqlens=None, state_in=None):
+    """The recurrence with the state captured at token offsets ``cuts`` (each strictly inside a
+    sequence; Ferrite project page, Design section 07, turn-boundary snapshots).  Each sequence is
+    run segment by segment between its cuts, carrying the state.  Returns ``(o, state,
+    snapshots [len(cuts), H, dv, dk])``."""
+    q, k, v, g, beta = (_d(x) for x in (q, k, v, g, beta))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    cu = _cu(cu_seqlens, T)
+    N = len(cu) - 1
+    cuts = [int(c) for c in np.asarray(cuts).reshape(-1)]
+    out = np.zeros((T, H, dv))
+    st = np.zeros((N, H, dv, dk))
+    snaps = np.zeros((len(cuts), H, dv, dk))
+    for n in range(N):
+        a, b = int(cu[n]), int(cu[n + 1])
+        inner = [(i, c) for i, c in enumerate(cuts) if a < c < b]
+        s = np.zeros((1, H, dv, dk)) if state_in is None else _d(state_in)[n:n + 1].copy()
+        bounds = [a] + [c for _, c in inner] + [b]
+        for j in range(len(bounds) - 1):
+            lo, hi = bounds[j], bounds[j + 1]
+            o, s = recurrence(q[lo:hi], k[lo:hi], v[lo:hi], g[lo:hi], beta[lo:hi], state_in=s)
+            out[lo:hi] = o
+            if j < len(inner):
+                snaps[inner[j][0]] = s[0]
+        st[n] = s[0]
+    return out, st, snaps
+
+
 def decode_verify(q, k, v, g, beta, state):
     """Tk speculative tokens per sequence run in order from ``state`` (which is not modified):
     inputs ``[B, Tk, H, d]`` / ``[B, Tk, H]``.  Returns ``(out [B, Tk, H, dv], states [B, Tk, H, dv,

@@ -129,6 +129,29 @@ def test_verify_rejects_bad_arguments(L):
     assert verify(L, B=0) == 0                          # nothing to do, nothing enqueued
 
 
+def prefill_cuts(L, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu=FAKE, N=2, T=64, cuts=FAKE, nc=2, s_in=None, out=FAKE,
+             s_out=FAKE, snaps=FAKE, H=2, dk=128, dv=128, dtype=1, ws=FAKE, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return L.gdn_chunk_prefill_cuts(a["q"], a["k"], a["v"], a["g"], a["beta"], a["cu"], a["N"], a["T"], a["cuts"],
+                                    a["nc"], a["s_in"], a["out"], a["s_out"], a["snaps"], a["H"], a["dk"], a["dv"],
+                                    a["dtype"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def test_prefill_cuts_rejects_bad_arguments(L):
+    assert prefill_cuts(L, nc=0) == -1
+    assert prefill_cuts(L, cuts=None) == -1
+    assert prefill_cuts(L, snaps=None) == -1
+    assert prefill_cuts(L, snaps=FAKE + 8) == -3
+    assert prefill_cuts(L, cuts=FAKE + 2) == -3
+    assert prefill_cuts(L, dk=96) == -2
+    # the workspace must cover num_seqs + num_cuts segments
+    need_plain = L.gdn_chunk_prefill_workspace_bytes(64, 2, 2, 128, 128)
+    need_cuts = L.gdn_chunk_prefill_workspace_bytes(64, 2 + 2, 2, 128, 128)
+    assert need_cuts > need_plain
+    assert prefill_cuts(L, ws_bytes=need_cuts - 1) == -5
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(gdn, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(gdn, "_lib", None)

@@ -278,6 +278,21 @@ def test_decode_step_is_length_one_recurrence():
             assert rel(o[i, h], Sn @ q[i, h] / np.sqrt(d)) < 1e-13
 
 
+def test_states_at_cuts_equal_prefix_runs():
+    """A snapshot at cut c equals the final state of the recurrence over the sequence's tokens
+    before c, and cutting changes neither the outputs nor the final states."""
+    q, k, v, g, b, s0 = rnd(90, 2, 6, 5, 31, N=3)
+    cu = np.array([0, 40, 40, 90])
+    cuts = [1, 17, 39, 41, 77]
+    o, st, sn = oracle.states_at(q, k, v, g, b, cuts, cu_seqlens=cu, state_in=s0)
+    o1, st1 = oracle.recurrence(q, k, v, g, b, cu_seqlens=cu, state_in=s0)
+    assert rel(o, o1) < 1e-13 and rel(st, st1) < 1e-13
+    for i, c in enumerate(cuts):
+        n = int(np.searchsorted(cu, c, side="right")) - 1
+        _, sp = oracle.recurrence(q[cu[n]:c], k[cu[n]:c], v[cu[n]:c], g[cu[n]:c], b[cu[n]:c], state_in=s0[n:n + 1])
+        assert rel(sn[i], sp[0]) < 1e-13
+
+
 def test_decode_verify_states_match_brute_force():
     """The state after each drafted token equals the explicit-matrix expansion over that prefix, and
     the outputs are S_t q_t / sqrt(dk); the committed state is left untouched."""
