@@ -369,6 +369,34 @@ def run_ours(args, rank, world, local_rank):
                                     traffic=TRAFFIC.get(name)))
         del dd, S
 
+    # ---- prefill_4k with state snapshots at 7 cut points (turn boundaries, not chunk-aligned) ----
+    cuts_line = None
+    if not args.no_cuts:
+        cut_pos = torch.tensor([517, 1000, 1531, 2048, 2600, 3071, 3500], dtype=torch.int32, device=dev)
+        ci = sets[0]
+        snaps = torch.empty((cut_pos.numel(), H, D, D), dtype=torch.float32, device=dev)
+        ws_c = torch.empty(gdn.workspace_bytes(T_PREFILL, N + cut_pos.numel(), H, D, D), dtype=torch.uint8,
+                           device=dev)
+        run_c = lambda: gdn.gdn_chunk_prefill_cuts(ci["q"], ci["k"], ci["v"], ci["g"], ci["beta"], cut_pos,
+                                                   cu_seqlens=ci["cu_seqlens"], state_in=ci["state_in"],
+                                                   snapshots=snaps, workspace=ws_c)
+        for _ in range(3):
+            run_c()
+        torch.cuda.synchronize()
+        reps = 20
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(reps):
+            run_c()
+        c1.record(stream)
+        torch.cuda.synchronize()
+        cms = max_over_ranks(c0.elapsed_time(c1), world, dev)
+        cuts_line = dict(workload="prefill_4k with 7 cut points (517, 1000, 1531, 2048, 2600, 3071, 3500): "
+                                  "chunks restart at each cut, 7 state snapshots written",
+                         value=job_throughput(T_PREFILL, reps, world, cms), unit="tokens/s",
+                         us_per_call=cms / reps * 1e3, inputs="first of the rotating input sets (L2-warm)")
+        del snaps, ws_c
+
     # ---- multi-token verify: B=64 sequences x 4 drafted tokens, every per-token state written ----
     verify = None
     if not args.no_verify:
@@ -453,7 +481,8 @@ def run_ours(args, rank, world, local_rank):
                 roofline=roofline, method_roofline=method_roofline, cpu_baseline=cpu,
                 e2e=dict(value=e2e_value, unit=UNIT, h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                          steps=e2e_steps),
-                gpu_launches=launches, clocks=clk, decode=decode, verify=verify)
+                gpu_launches=launches, clocks=clk, decode=decode, verify=verify,
+                cuts=cuts_line)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -466,6 +495,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-verify", action="store_true")
+    ap.add_argument("--no-cuts", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
