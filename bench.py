@@ -63,6 +63,7 @@ KERNELS = {
     "gdn_plan_kernel": dict(bound="latency"),
     "gdn_decode_step_kernel": dict(bound="hbm"),
     "gdn_decode_verify_kernel": dict(bound="hbm"),
+    "gdn_l2norm_kernel": dict(bound="hbm"),
 }
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from the last ncu capture of that kernel
 # on the bench workload (None until captured, and reset whenever the kernel changes).  The decode
@@ -397,6 +398,45 @@ def run_ours(args, rank, world, local_rank):
                          us_per_call=cms / reps * 1e3, inputs="first of the rotating input sets (L2-warm)")
         del snaps, ws_c
 
+    # ---- prefill_4k with raw q/k: the library L2-normalises them (pre-pass into the workspace) ----
+    norm_line = None
+    if not args.no_norm:
+        ni = sets[0]
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(77)
+        sc = torch.exp(torch.empty((T_PREFILL, H, 1), device=dev).uniform_(-3.0, 3.0, generator=gen))
+        qr, kr = (ni["q"].float() * sc).to(ni["q"].dtype), (ni["k"].float() * sc.flip(0)).to(ni["k"].dtype)
+        ws_n = torch.empty(gdn.workspace_bytes(T_PREFILL, N, H, D, D, gdn.GDN_BF16 | gdn.GDN_QK_L2NORM),
+                           dtype=torch.uint8, device=dev)
+        run_n = lambda: gdn.gdn_chunk_prefill(qr, kr, ni["v"], ni["g"], ni["beta"], cu_seqlens=ni["cu_seqlens"],
+                                              workspace=ws_n, normalize_qk=True)
+        for _ in range(3):
+            run_n()
+        torch.cuda.synchronize()
+        reps = 20
+        gdn.gdn_profile_start()
+        n0, n1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n0.record(stream)
+        for _ in range(reps):
+            run_n()
+        n1.record(stream)
+        torch.cuda.synchronize()
+        nprof = gdn.gdn_profile_stop()
+        nms = max_over_ranks(n0.elapsed_time(n1), world, dev)
+        name = "gdn_l2norm_kernel"
+        kms, kl = nprof.get(name, (nms, reps))
+        bytes_per_launch = 4 * T_PREFILL * H * D * 2          # q, k read and their normalised copies written
+        ach = bytes_per_launch / (kms / kl / 1e3) / 1e9
+        pk, pu, pdesc = peak_for("hbm", peaks)
+        norm_line = dict(workload="prefill_4k with raw q/k (vectors scaled by e^U[-3,3]); the library L2-normalises "
+                                  "them in a pre-pass",
+                         value=job_throughput(T_PREFILL, reps, world, nms), unit="tokens/s",
+                         us_per_call=nms / reps * 1e3, inputs="first of the rotating input sets (L2-warm)",
+                         roofline=dict(kernel=name, bound="hbm", achieved=ach, peak=pk, unit=pu, frac=ach / pk,
+                                       peak_source=pdesc, bytes_per_launch=bytes_per_launch,
+                                       avg_launch_us=kms / kl * 1e3, traffic=TRAFFIC.get(name)))
+        del qr, kr, ws_n
+
     # ---- multi-token verify: B=64 sequences x 4 drafted tokens, every per-token state written ----
     verify = None
     if not args.no_verify:
@@ -482,7 +522,7 @@ def run_ours(args, rank, world, local_rank):
                 e2e=dict(value=e2e_value, unit=UNIT, h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                          steps=e2e_steps),
                 gpu_launches=launches, clocks=clk, decode=decode, verify=verify,
-                cuts=cuts_line)
+                cuts=cuts_line, norm=norm_line)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -496,6 +536,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-verify", action="store_true")
     ap.add_argument("--no-cuts", action="store_true")
+    ap.add_argument("--no-norm", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()

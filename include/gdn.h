@@ -48,6 +48,16 @@ extern "C" {
 /* Storage type of q, k, v and out. */
 typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
 
+/*
+ * Flag that may be OR'ed into the `dtype` argument of every call that takes q and k: they are
+ * passed raw and the library L2-normalises each (token, head) vector, x / max(||x||_2, 1e-12) with
+ * the norm summed in fp32, and rounds the result to the storage dtype before use.  The prefill
+ * writes the normalised copies into its workspace (see gdn_chunk_prefill_workspace_bytes_ex);
+ * decode and verify normalise in registers.  Without the flag q and k must arrive normalised
+ * (the method's definition) and are used as given.
+ */
+#define GDN_QK_L2NORM 0x100
+
 /* Status codes. */
 enum {
     GDN_OK = 0,
@@ -76,6 +86,14 @@ int gdn_version(void);
 size_t gdn_chunk_prefill_workspace_bytes(int64_t total_tokens, int num_seqs, int H, int dk, int dv);
 
 /*
+ * Workspace for any prefill call: num_segments = num_seqs (+ num_cuts for gdn_chunk_prefill_cuts),
+ * dtype as passed to the call (with GDN_QK_L2NORM the normalised q and k copies are included).
+ * Returns 0 for arguments the calls would reject.
+ */
+size_t gdn_chunk_prefill_workspace_bytes_ex(int64_t total_tokens, int num_segments, int H, int dk,
+                                            int dv, int dtype);
+
+/*
  * Chunked prefill (Ferrite project page, Design section 03): runs the gated delta rule over every
  * token of N packed sequences, chunk size C = 32 with chunk boundaries relative to each sequence's
  * start, and writes every output o_t and each sequence's final state.
@@ -90,7 +108,9 @@ size_t gdn_chunk_prefill_workspace_bytes(int64_t total_tokens, int num_seqs, int
  *   out           device [T_total, H, dv], dtype `dtype`; must not overlap any input
  *   state_out     device fp32 [N, H, dv, dk] final states, or NULL (not written).  May equal
  *                 state_in (in-place resume); must not overlap any other buffer otherwise.
- *   workspace     device scratch of at least gdn_chunk_prefill_workspace_bytes(...) bytes,
+ *   dtype         GDN_F32 or GDN_BF16, optionally | GDN_QK_L2NORM (raw q, k)
+ *   workspace     device scratch of at least gdn_chunk_prefill_workspace_bytes(...) bytes (with
+ *                 GDN_QK_L2NORM: gdn_chunk_prefill_workspace_bytes_ex(..., dtype)),
  *                 256-byte aligned; its contents on entry do not matter and are clobbered.  The
  *                 workspace must not be used by another call that runs concurrently.
  *

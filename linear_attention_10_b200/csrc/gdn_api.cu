@@ -14,6 +14,7 @@
 
 #include "gdn_common.cuh"
 #include "gdn_decode.cuh"
+#include "gdn_norm.cuh"
 #include "gdn_plan.cuh"
 #include "gdn_prefill_tc.cuh"
 #include "gdn_prep_bf16.cuh"
@@ -89,45 +90,50 @@ static bool head_ok(int d) { return d == 64 || d == 128; }
 
 template <typename T, int DK, int DV>
 static int launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                         float* state, void* out, int B, int H, cudaStream_t st)
+                         float* state, void* out, int B, int H, bool norm, cudaStream_t st)
 {
     ProfScope prof("gdn_decode_step_kernel", st);
-    gdn_decode_step_kernel<T, DK, DV><<<(unsigned)B * H, 256, 0, st>>>(
-        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g, beta, state,
-        static_cast<T*>(out), H);
+    auto kern = norm ? gdn_decode_step_kernel<T, DK, DV, true> : gdn_decode_step_kernel<T, DK, DV, false>;
+    kern<<<(unsigned)B * H, 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
+                                          g, beta, state, static_cast<T*>(out), H);
     return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
 }
 
 template <typename T>
 static int dispatch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                           float* state, void* out, int B, int H, int dk, int dv, cudaStream_t st)
+                           float* state, void* out, int B, int H, int dk, int dv, bool norm, cudaStream_t st)
 {
-    if (dk == 128 && dv == 128) return launch_decode<T, 128, 128>(q, k, v, g, beta, state, out, B, H, st);
-    if (dk == 128 && dv == 64) return launch_decode<T, 128, 64>(q, k, v, g, beta, state, out, B, H, st);
-    if (dk == 64 && dv == 128) return launch_decode<T, 64, 128>(q, k, v, g, beta, state, out, B, H, st);
-    return launch_decode<T, 64, 64>(q, k, v, g, beta, state, out, B, H, st);
+    if (dk == 128 && dv == 128) return launch_decode<T, 128, 128>(q, k, v, g, beta, state, out, B, H, norm, st);
+    if (dk == 128 && dv == 64) return launch_decode<T, 128, 64>(q, k, v, g, beta, state, out, B, H, norm, st);
+    if (dk == 64 && dv == 128) return launch_decode<T, 64, 128>(q, k, v, g, beta, state, out, B, H, norm, st);
+    return launch_decode<T, 64, 64>(q, k, v, g, beta, state, out, B, H, norm, st);
 }
 
 template <typename T, int DK, int DV>
 static int launch_verify(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                         const float* state_in, float* states_out, void* out, int B, int Tk, int H, cudaStream_t st)
+                         const float* state_in, float* states_out, void* out, int B, int Tk, int H, bool norm,
+                         cudaStream_t st)
 {
     ProfScope prof("gdn_decode_verify_kernel", st);
-    gdn_decode_verify_kernel<T, DK, DV><<<(unsigned)B * H, 256, 0, st>>>(
-        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g, beta, state_in, states_out,
-        static_cast<T*>(out), H, Tk);
+    auto kern = norm ? gdn_decode_verify_kernel<T, DK, DV, true> : gdn_decode_verify_kernel<T, DK, DV, false>;
+    kern<<<(unsigned)B * H, 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
+                                          g, beta, state_in, states_out, static_cast<T*>(out), H, Tk);
     return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
 }
 
 template <typename T>
 static int dispatch_verify(const void* q, const void* k, const void* v, const float* g, const float* beta,
                            const float* state_in, float* states_out, void* out, int B, int Tk, int H, int dk, int dv,
-                           cudaStream_t st)
+                           bool norm, cudaStream_t st)
 {
-    if (dk == 128 && dv == 128) return launch_verify<T, 128, 128>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, st);
-    if (dk == 128 && dv == 64) return launch_verify<T, 128, 64>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, st);
-    if (dk == 64 && dv == 128) return launch_verify<T, 64, 128>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, st);
-    return launch_verify<T, 64, 64>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, st);
+#define GDN_VF(DK_, DV_)                                                                                   \
+    if (dk == DK_ && dv == DV_)                                                                            \
+        return launch_verify<T, DK_, DV_>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, norm, st);
+    GDN_VF(128, 128)
+    GDN_VF(128, 64)
+    GDN_VF(64, 128)
+#undef GDN_VF
+    return launch_verify<T, 64, 64>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, norm, st);
 }
 
 // ---- tensor maps (2-D tiled views of q/k/v) -------------------------------------------------------
@@ -326,6 +332,37 @@ static void* noalloc_scratch_ptr()
     return cache[dev];
 }
 
+// dtype argument: GDN_F32 or GDN_BF16, optionally with the GDN_QK_L2NORM flag
+static bool split_dtype(int code, int& dtype, bool& norm)
+{
+    if (code & ~(0xff | GDN_QK_L2NORM)) return false;
+    dtype = code & 0xff;
+    norm = (code & GDN_QK_L2NORM) != 0;
+    return dtype == GDN_F32 || dtype == GDN_BF16;
+}
+
+// bytes of the normalised q and k copies that the prefill's pre-pass writes after the layout
+static size_t norm_bytes(int64_t T, int H, int dk, int dtype)
+{
+    return PrefillLayout::align((size_t)T * H * dk * (dtype == GDN_F32 ? 4 : 2)) * 2;
+}
+
+template <typename T>
+static int launch_l2norm(const void* q, const void* k, void* qn, void* kn, int64_t nvec, int dk, cudaStream_t st)
+{
+    ProfScope prof("gdn_l2norm_kernel", st);
+    const int64_t vpw = (dk == 128 ? 1 : 2) * kNormU;          // vectors per warp
+    const int64_t warps = (nvec + vpw - 1) / vpw;
+    const unsigned grid = (unsigned)((warps + 7) / 8);
+    if (dk == 128)
+        gdn_l2norm_kernel<T, 128><<<grid, 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                                        static_cast<T*>(qn), static_cast<T*>(kn), nvec);
+    else
+        gdn_l2norm_kernel<T, 64><<<grid, 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                                       static_cast<T*>(qn), static_cast<T*>(kn), nvec);
+    return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
+}
+
 static int chunk_prefill(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens, const float* state_in,
                          void* out, float* state_out, int H, int dk, int dv, int dtype, const Cuts& cuts,
@@ -334,7 +371,8 @@ static int chunk_prefill(const void* q, const void* k, const void* v, const floa
     if (num_seqs < 1 || H < 1 || total_tokens < 0 || total_tokens > INT32_MAX) return GDN_ERR_INVALID_ARG;
     if (cuts.n < 0 || (cuts.n > 0 && (!cuts.pos || !cuts.snaps))) return GDN_ERR_INVALID_ARG;
     if ((int64_t)num_seqs + cuts.n > INT32_MAX / 8) return GDN_ERR_INVALID_ARG;
-    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    bool norm = false;
+    if (!split_dtype(dtype, dtype, norm)) return GDN_ERR_INVALID_ARG;
     if (!head_ok(dk) || !head_ok(dv)) return GDN_ERR_UNSUPPORTED;
     if (total_tokens > 0 && (!q || !k || !v || !g || !beta || !out)) return GDN_ERR_INVALID_ARG;
     int fixed_len = 0;
@@ -349,10 +387,21 @@ static int chunk_prefill(const void* q, const void* k, const void* v, const floa
     for (const void* p : small)
         if (p && !aligned4(p)) return GDN_ERR_MISALIGNED;
     PrefillLayout lay(total_tokens, num_seqs + cuts.n, H, dk);
-    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < lay.total)
+    const size_t need = lay.total + (norm ? norm_bytes(total_tokens, H, dk, dtype) : 0);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
         return GDN_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char* ws = static_cast<char*>(workspace);
+    if (norm && total_tokens > 0) {
+        // raw q and k: normalised copies in the workspace replace them for the rest of the call
+        char* qn = ws + lay.total;
+        char* kn = qn + norm_bytes(total_tokens, H, dk, dtype) / 2;
+        const int rc = dtype == GDN_F32 ? launch_l2norm<float>(q, k, qn, kn, total_tokens * H, dk, st)
+                                        : launch_l2norm<__nv_bfloat16>(q, k, qn, kn, total_tokens * H, dk, st);
+        if (rc != GDN_OK) return rc;
+        q = qn;
+        k = kn;
+    }
     if (dtype == GDN_F32)
         return dispatch_prefill<float>(dk, dv, lay, ws, q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
                                        fixed_len, state_in, out, state_out, H, cuts, st);
@@ -390,6 +439,15 @@ size_t gdn_chunk_prefill_workspace_bytes(int64_t total_tokens, int num_seqs, int
     return PrefillLayout(total_tokens, num_seqs, H, dk).total;
 }
 
+size_t gdn_chunk_prefill_workspace_bytes_ex(int64_t total_tokens, int num_segments, int H, int dk, int dv, int dtype)
+{
+    bool norm = false;
+    if (!split_dtype(dtype, dtype, norm)) return 0;
+    const size_t base = gdn_chunk_prefill_workspace_bytes(total_tokens, num_segments, H, dk, dv);
+    if (base == 0) return 0;
+    return base + (norm ? norm_bytes(total_tokens, H, dk, dtype) : 0);
+}
+
 int gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* g, const float* beta,
                       const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens, const float* state_in,
                       void* out, float* state_out, int H, int dk, int dv, int dtype, void* workspace,
@@ -419,7 +477,7 @@ int gdn_chunk_prefill_noalloc(const void* q, const void* k, const void* v, const
                               int dtype, void* stream)
 {
     // the scratch must hold the whole workspace of this call; refuse before touching the device
-    const size_t need = gdn_chunk_prefill_workspace_bytes(total_tokens, num_seqs, H, dk, dv);
+    const size_t need = gdn_chunk_prefill_workspace_bytes_ex(total_tokens, num_seqs, H, dk, dv, dtype);
     if (need > kNoallocScratchBytes) return GDN_ERR_WORKSPACE;
     void* scratch = noalloc_scratch_ptr();
     if (!scratch) return GDN_ERR_CUDA;
@@ -432,7 +490,8 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
                     float* state_inout, void* out, int B, int H, int dk, int dv, int dtype, void* stream)
 {
     if (B < 0 || H < 1) return GDN_ERR_INVALID_ARG;
-    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    bool norm = false;
+    if (!split_dtype(dtype, dtype, norm)) return GDN_ERR_INVALID_ARG;
     if (!head_ok(dk) || !head_ok(dv)) return GDN_ERR_UNSUPPORTED;
     if (B == 0) return GDN_OK;
     if (!q || !k || !v || !g || !beta || !state_inout) return GDN_ERR_INVALID_ARG;
@@ -442,8 +501,8 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
     if (!aligned4(g) || !aligned4(beta)) return GDN_ERR_MISALIGNED;
     if ((int64_t)B * H > INT32_MAX) return GDN_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (dtype == GDN_F32) return dispatch_decode<float>(q, k, v, g, beta, state_inout, out, B, H, dk, dv, st);
-    return dispatch_decode<__nv_bfloat16>(q, k, v, g, beta, state_inout, out, B, H, dk, dv, st);
+    if (dtype == GDN_F32) return dispatch_decode<float>(q, k, v, g, beta, state_inout, out, B, H, dk, dv, norm, st);
+    return dispatch_decode<__nv_bfloat16>(q, k, v, g, beta, state_inout, out, B, H, dk, dv, norm, st);
 }
 
 int gdn_decode_verify(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -451,7 +510,8 @@ int gdn_decode_verify(const void* q, const void* k, const void* v, const float* 
                       int dtype, void* stream)
 {
     if (B < 0 || Tk < 1 || H < 1) return GDN_ERR_INVALID_ARG;
-    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    bool norm = false;
+    if (!split_dtype(dtype, dtype, norm)) return GDN_ERR_INVALID_ARG;
     if (!head_ok(dk) || !head_ok(dv)) return GDN_ERR_UNSUPPORTED;
     if (B == 0) return GDN_OK;
     if (!q || !k || !v || !g || !beta || !state_in) return GDN_ERR_INVALID_ARG;
@@ -463,8 +523,8 @@ int gdn_decode_verify(const void* q, const void* k, const void* v, const float* 
     if ((int64_t)B * H > INT32_MAX || (int64_t)B * Tk * H > INT32_MAX) return GDN_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dtype == GDN_F32)
-        return dispatch_verify<float>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, dk, dv, st);
-    return dispatch_verify<__nv_bfloat16>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, dk, dv, st);
+        return dispatch_verify<float>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, dk, dv, norm, st);
+    return dispatch_verify<__nv_bfloat16>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, dk, dv, norm, st);
 }
 
 int gdn_get_device_status(void* stream)

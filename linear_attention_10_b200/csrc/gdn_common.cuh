@@ -32,6 +32,7 @@ struct Elem<float> {
     {
         return __ldg(reinterpret_cast<const float4*>(p));
     }
+    static __device__ __forceinline__ void st4(float* p, float4 x) { *reinterpret_cast<float4*>(p) = x; }
 };
 
 template <>
@@ -49,6 +50,14 @@ struct Elem<__nv_bfloat16> {
         __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&raw.y);
         float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
         return make_float4(fa.x, fa.y, fb.x, fb.y);
+    }
+    static __device__ __forceinline__ void st4(__nv_bfloat16* p, float4 x)
+    {
+        __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y), b = __floats2bfloat162_rn(x.z, x.w);
+        uint2 raw;
+        raw.x = *reinterpret_cast<uint32_t*>(&a);
+        raw.y = *reinterpret_cast<uint32_t*>(&b);
+        *reinterpret_cast<uint2*>(p) = raw;
     }
 };
 

@@ -17,6 +17,7 @@
 #pragma once
 
 #include "gdn_common.cuh"
+#include "gdn_norm.cuh"
 
 namespace gdn {
 
@@ -54,7 +55,7 @@ __device__ __forceinline__ float row_dot(const float4 a, const float4 b)
     return d;
 }
 
-template <typename T, int DK, int DV>
+template <typename T, int DK, int DV, bool NORM>
 __global__ void __launch_bounds__(256) gdn_decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                           const T* __restrict__ v, const float* __restrict__ g,
                                                           const float* __restrict__ beta, float* state,
@@ -73,8 +74,13 @@ __global__ void __launch_bounds__(256) gdn_decode_step_kernel(const T* __restric
     const int sub = lane / LPR;               // which of the RPW rows this lane serves
     const int col = (lane % LPR) * 4;
 
-    const float4 k4 = Elem<T>::ld4(k + (size_t)bh * DK + col);
-    const float4 q4 = Elem<T>::ld4(q + (size_t)bh * DK + col);
+    float4 k4 = Elem<T>::ld4(k + (size_t)bh * DK + col);
+    float4 q4 = Elem<T>::ld4(q + (size_t)bh * DK + col);
+    if constexpr (NORM) {
+        // raw q and k: normalised here exactly as the prefill's pre-pass does
+        k4 = scale_round<T>(k4, l2_inv_norm(row_dot<LPR>(k4, k4)));
+        q4 = scale_round<T>(q4, l2_inv_norm(row_dot<LPR>(q4, q4)));
+    }
     const float alpha = expf(__ldg(g + bh));
     const float b = __ldg(beta + bh);
     const float scale = rsqrtf((float)DK);
@@ -111,7 +117,7 @@ __global__ void __launch_bounds__(256) gdn_decode_step_kernel(const T* __restric
 //
 // Mapping: one CTA (8 warps) per (b, h); the whole dv x dk state of the pair lives in registers for
 // the Tk tokens (each lane holds NR float4s of its rows), is read from HBM once and written Tk times.
-template <typename T, int DK, int DV>
+template <typename T, int DK, int DV, bool NORM>
 __global__ void __launch_bounds__(256) gdn_decode_verify_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                             const T* __restrict__ v, const float* __restrict__ g,
                                                             const float* __restrict__ beta,
@@ -140,8 +146,12 @@ __global__ void __launch_bounds__(256) gdn_decode_verify_kernel(const T* __restr
 
     for (int t = 0; t < Tk; ++t) {
         const size_t tok = ((size_t)b * Tk + t) * H + h;      // index into [B, Tk, H]
-        const float4 k4 = Elem<T>::ld4(k + tok * DK + col);
-        const float4 q4 = Elem<T>::ld4(q + tok * DK + col);
+        float4 k4 = Elem<T>::ld4(k + tok * DK + col);
+        float4 q4 = Elem<T>::ld4(q + tok * DK + col);
+        if constexpr (NORM) {
+            k4 = scale_round<T>(k4, l2_inv_norm(row_dot<LPR>(k4, k4)));
+            q4 = scale_round<T>(q4, l2_inv_norm(row_dot<LPR>(q4, q4)));
+        }
         const float alpha = expf(__ldg(g + tok));
         const float bb = __ldg(beta + tok);
         const float kq = row_dot<LPR>(k4, q4);

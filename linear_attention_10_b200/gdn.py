@@ -17,6 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdn.so")
 
 GDN_F32, GDN_BF16 = 0, 1
+GDN_QK_L2NORM = 0x100           # flag in the dtype argument: q, k raw, normalised by the library
 CHUNK = 32
 
 # symbols declared in include/gdn.h
@@ -24,6 +25,7 @@ EXPORTS = (
     "gdn_status_string",
     "gdn_version",
     "gdn_chunk_prefill_workspace_bytes",
+    "gdn_chunk_prefill_workspace_bytes_ex",
     "gdn_chunk_prefill",
     "gdn_chunk_prefill_cuts",
     "gdn_chunk_prefill_noalloc",
@@ -59,6 +61,8 @@ def lib() -> ctypes.CDLL:
     L.gdn_version.restype = i32
     L.gdn_chunk_prefill_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
     L.gdn_chunk_prefill_workspace_bytes.restype = sz
+    L.gdn_chunk_prefill_workspace_bytes_ex.argtypes = [i64, i32, i32, i32, i32, i32]
+    L.gdn_chunk_prefill_workspace_bytes_ex.restype = sz
     L.gdn_chunk_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, i32, i32,
                                     vp, sz, vp]
     L.gdn_chunk_prefill.restype = i32
@@ -115,12 +119,19 @@ def _check(t, name, shape, dtype, dev):
         raise ValueError("%s must be contiguous" % name)
 
 
-def workspace_bytes(total_tokens: int, num_seqs: int, H: int, dk: int, dv: int) -> int:
-    return int(lib().gdn_chunk_prefill_workspace_bytes(int(total_tokens), int(num_seqs), int(H), int(dk), int(dv)))
+def workspace_bytes(total_tokens: int, num_seqs: int, H: int, dk: int, dv: int, dtype_code: Optional[int] = None) -> int:
+    """Workspace of a prefill call (num_seqs counts segments: sequences plus cut points); with a
+    dtype code carrying GDN_QK_L2NORM the normalised q/k copies are included."""
+    if dtype_code is None:
+        return int(lib().gdn_chunk_prefill_workspace_bytes(int(total_tokens), int(num_seqs), int(H), int(dk),
+                                                            int(dv)))
+    return int(lib().gdn_chunk_prefill_workspace_bytes_ex(int(total_tokens), int(num_seqs), int(H), int(dk), int(dv),
+                                                           int(dtype_code)))
 
 
 def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens=None, state_in=None, out=None, state_out=None,
-                      workspace=None, num_seqs: Optional[int] = None, stream=None, output_final_state=True):
+                      workspace=None, num_seqs: Optional[int] = None, stream=None, output_final_state=True,
+                      normalize_qk=False):
     """Chunked gated-delta-rule prefill over packed sequences.
 
     q, k ``[T, H, dk]``; v ``[T, H, dv]`` (fp32 or bf16, same dtype); g, beta ``[T, H]`` fp32;
@@ -149,11 +160,12 @@ def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens=None, state_in=None, out=None
         state_out = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
     if state_out is not None:
         _check(state_out, "state_out", (N, H, dv, dk), torch.float32, dev)
-    need = workspace_bytes(T, N, H, dk, dv)
+    code = _dtype_code(q) | (GDN_QK_L2NORM if normalize_qk else 0)
+    need = workspace_bytes(T, N, H, dk, dv, code)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     rc = lib().gdn_chunk_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, T,
-                                 _ptr(state_in), _ptr(out), _ptr(state_out), H, dk, dv, _dtype_code(q),
+                                 _ptr(state_in), _ptr(out), _ptr(state_out), H, dk, dv, code,
                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
                                  _stream_ptr(stream))
     if rc != 0:
@@ -163,7 +175,7 @@ def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens=None, state_in=None, out=None
 
 def gdn_chunk_prefill_cuts(q, k, v, g, beta, cuts, cu_seqlens=None, state_in=None, out=None, state_out=None,
                            snapshots=None, workspace=None, num_seqs: Optional[int] = None, stream=None,
-                           output_final_state=True):
+                           output_final_state=True, normalize_qk=False):
     """``gdn_chunk_prefill`` that also returns the state at each cut point: ``cuts`` int32 ``[n]`` on
     the device (strictly increasing token offsets, each strictly inside a sequence).  Returns
     ``(out, state_out, snapshots [n, H, dv, dk])``."""
@@ -193,19 +205,20 @@ def gdn_chunk_prefill_cuts(q, k, v, g, beta, cuts, cu_seqlens=None, state_in=Non
     if snapshots is None:
         snapshots = torch.empty((max(nc, 1), H, dv, dk), dtype=torch.float32, device=dev)[:nc]
     _check(snapshots, "snapshots", (nc, H, dv, dk), torch.float32, dev)
-    need = workspace_bytes(T, N + nc, H, dk, dv)
+    code = _dtype_code(q) | (GDN_QK_L2NORM if normalize_qk else 0)
+    need = workspace_bytes(T, N + nc, H, dk, dv, code)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     rc = lib().gdn_chunk_prefill_cuts(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, T,
                                       _ptr(cuts), nc, _ptr(state_in), _ptr(out), _ptr(state_out), _ptr(snapshots),
-                                      H, dk, dv, _dtype_code(q), _ptr(workspace),
+                                      H, dk, dv, code, _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     if rc != 0:
         raise GdnError(rc, "gdn_chunk_prefill_cuts")
     return out, state_out, snapshots
 
 
-def gdn_decode_step(q, k, v, g, beta, state, out=None, stream=None):
+def gdn_decode_step(q, k, v, g, beta, state, out=None, stream=None, normalize_qk=False):
     """One recurrent step for B sequences: q, k ``[B, H, dk]``, v ``[B, H, dv]``, g, beta ``[B, H]``,
     state fp32 ``[B, H, dv, dk]`` updated in place.  Returns ``out [B, H, dv]``."""
     B, H, dk = q.shape
@@ -220,14 +233,16 @@ def gdn_decode_step(q, k, v, g, beta, state, out=None, stream=None):
     if out is None:
         out = torch.empty((B, H, dv), dtype=dt, device=dev)
     _check(out, "out", (B, H, dv), dt, dev)
+    code = _dtype_code(q) | (GDN_QK_L2NORM if normalize_qk else 0)
     rc = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(out),
-                               B, H, dk, dv, _dtype_code(q), _stream_ptr(stream))
+                               B, H, dk, dv, code, _stream_ptr(stream))
     if rc != 0:
         raise GdnError(rc, "gdn_decode_step")
     return out
 
 
-def gdn_decode_verify(q, k, v, g, beta, state_in, states_out=None, out=None, want_states=True, stream=None):
+def gdn_decode_verify(q, k, v, g, beta, state_in, states_out=None, out=None, want_states=True, stream=None,
+                      normalize_qk=False):
     """Tk speculative tokens per sequence through the recurrence: q, k ``[B, Tk, H, dk]``, v
     ``[B, Tk, H, dv]``, g, beta ``[B, Tk, H]``, state_in fp32 ``[B, H, dv, dk]`` (read only).
     Returns ``(out [B, Tk, H, dv], states_out [B, Tk, H, dv, dk] or None)``."""
@@ -249,7 +264,8 @@ def gdn_decode_verify(q, k, v, g, beta, state_in, states_out=None, out=None, wan
         _check(states_out, "states_out", (B, Tk, H, dv, dk), torch.float32, dev)
     rc = lib().gdn_decode_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
                                  None if states_out is None else _ptr(states_out), _ptr(out),
-                                 B, Tk, H, dk, dv, _dtype_code(q), _stream_ptr(stream))
+                                 B, Tk, H, dk, dv, _dtype_code(q) | (GDN_QK_L2NORM if normalize_qk else 0),
+                                 _stream_ptr(stream))
     if rc != 0:
         raise GdnError(rc, "gdn_decode_verify")
     return out, states_out

@@ -144,6 +144,15 @@ def decode_step(q, k, v, g, beta, state):
     return recurrence(q, k, v, g, beta, cu_seqlens=np.arange(B + 1), state_in=state)
 
 
+def l2norm(x, eps=1e-12):
+    """L2 normalisation of every vector along the last axis in fp64, x / max(||x||_2, eps): the
+    step that makes q_t and k_t the unit vectors the recurrence is defined on (inputs of the
+    method are L2-normalised per token and head)."""
+    x = _d(x)
+    n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+    return x / np.maximum(n, eps)
+
+
 def states_at(q, k, v, g, beta, cuts, cu_seqlens=None, state_in=None):
     """The recurrence with the state captured at token offsets ``cuts`` (each strictly inside a
     sequence; Ferrite project page, Design section 07, turn-boundary snapshots).  Each sequence is

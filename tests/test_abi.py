@@ -152,6 +152,24 @@ def test_prefill_cuts_rejects_bad_arguments(L):
     assert prefill_cuts(L, ws_bytes=need_cuts - 1) == -5
 
 
+def test_normalisation_flag(L):
+    assert L.gdn_chunk_prefill_workspace_bytes_ex(4096, 1, 32, 128, 128, 1) == \
+        L.gdn_chunk_prefill_workspace_bytes(4096, 1, 32, 128, 128)
+    plain = L.gdn_chunk_prefill_workspace_bytes(4096, 1, 32, 128, 128)
+    assert L.gdn_chunk_prefill_workspace_bytes_ex(4096, 1, 32, 128, 128, 1 | gdn.GDN_QK_L2NORM) >= plain + 2 * 4096 * 32 * 128 * 2
+    assert L.gdn_chunk_prefill_workspace_bytes_ex(4096, 1, 32, 128, 128, 0x200) == 0      # unknown flag bit
+    assert prefill(L, dtype=1 | 0x200) == -1
+    assert decode(L, dtype=1 | 0x200) == -1
+    assert verify(L, dtype=1 | 0x200) == -1
+    # the normalised copies need room: the plain workspace size of the same call is refused (the
+    # sizes here are prefill()'s defaults: T=64, N=1, H=2, dk=dv=64)
+    need = L.gdn_chunk_prefill_workspace_bytes(64, 1, 2, 64, 64)
+    need_ex = L.gdn_chunk_prefill_workspace_bytes_ex(64, 1, 2, 64, 64, 1 | gdn.GDN_QK_L2NORM)
+    assert need_ex > need
+    assert prefill(L, dtype=1 | gdn.GDN_QK_L2NORM, ws_bytes=need) == -5
+    assert prefill(L, dtype=1 | gdn.GDN_QK_L2NORM, ws_bytes=need_ex - 1) == -5
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(gdn, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(gdn, "_lib", None)

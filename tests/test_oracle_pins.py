@@ -278,6 +278,22 @@ def test_decode_step_is_length_one_recurrence():
             assert rel(o[i, h], Sn @ q[i, h] / np.sqrt(d)) < 1e-13
 
 
+def test_l2norm_unit_length_direction_and_degenerate_vectors():
+    r = np.random.default_rng(51)
+    x = r.standard_normal((7, 3, 16)) * r.uniform(0.01, 100.0, (7, 3, 1))
+    y = oracle.l2norm(x)
+    assert np.max(np.abs(np.linalg.norm(y, axis=-1) - 1.0)) < 1e-14
+    # same direction: y is a positive multiple of x
+    cos = np.sum(x * y, axis=-1) / np.linalg.norm(x, axis=-1)
+    assert np.max(np.abs(cos - 1.0)) < 1e-14
+    assert rel(oracle.l2norm(3.5 * x), y) < 1e-15               # scale invariance
+    assert rel(oracle.l2norm(y), y) < 1e-15                     # idempotent
+    z = np.zeros((2, 5))
+    assert np.array_equal(oracle.l2norm(z), z)                  # zero vector stays zero
+    tiny = np.full((1, 4), 1e-14)                               # norm below eps: divided by eps
+    assert rel(oracle.l2norm(tiny), tiny / 1e-12) < 1e-15
+
+
 def test_states_at_cuts_equal_prefix_runs():
     """A snapshot at cut c equals the final state of the recurrence over the sequence's tokens
     before c, and cutting changes neither the outputs nor the final states."""
