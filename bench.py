@@ -70,7 +70,6 @@ KERNELS = {
 # figure undercounts writes: ncu starts each replay from a clean L2, and about 57 MB of the written
 # state is still resident (dirty) in L2 when the launch ends.
 TRAFFIC = {
-    "gdn_decode_step_kernel": 135.90e6 + 77.22e6,
     "gdn_scan_bf16_kernel": 203.15e6 + 27.64e6,
     "gdn_prep_bf16_kernel": 68.22e6 + 48.88e6,
 }

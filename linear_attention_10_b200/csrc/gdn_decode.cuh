@@ -11,9 +11,10 @@
 // hold it, and the updated row is stored once.  The kernel is bound by HBM bandwidth: per (b, h)
 // it moves 2 * dv * dk * 4 bytes of state and a few hundred bytes of q, k, v, o.
 //
-// Mapping: one CTA (8 warps) per (b, h).  A row of dk fp32 is held by dk/4 lanes as float4s
-// (a full warp for dk = 128, half a warp for dk = 64).  Each warp owns dv/8 consecutive rows and
-// loads UNROLL row-groups before reducing, to keep enough bytes in flight.
+// Mapping: the state of one (b, h) is split into row blocks of 32 rows, one CTA (8 warps) per block;
+// a row of dk fp32 is held by dk/4 lanes as float4s (a full warp for dk = 128, half a warp for
+// dk = 64).  Each warp owns 4 consecutive rows and loads them all before reducing.  Small CTAs keep
+// the last wave short (2048 (b, h) pairs would leave a 0.3-full third wave at 256-row granularity).
 #pragma once
 
 #include "gdn_common.cuh"
@@ -55,21 +56,34 @@ __device__ __forceinline__ float row_dot(const float4 a, const float4 b)
     return d;
 }
 
+// Rows of one (sequence, head) state per CTA and threads per CTA of the decode step (rows evolve
+// independently, so a state may be split across CTAs; smaller CTAs leave a smaller last wave).
+#ifndef GDN_DECODE_RB
+#define GDN_DECODE_RB 32
+#endif
+#ifndef GDN_DECODE_NT
+#define GDN_DECODE_NT 256
+#endif
+
 template <typename T, int DK, int DV, bool NORM>
-__global__ void __launch_bounds__(256) gdn_decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(GDN_DECODE_NT) gdn_decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                           const T* __restrict__ v, const float* __restrict__ g,
                                                           const float* __restrict__ beta, float* state,
                                                           T* __restrict__ out, int H)
 {
     constexpr int LPR = DK / 4;               // lanes per row
     constexpr int RPW = 32 / LPR;             // rows handled by one warp at once
-    constexpr int ROWS_PER_WARP = DV / 8;
+    constexpr int RB = (GDN_DECODE_RB < DV) ? GDN_DECODE_RB : DV;   // rows of the state per CTA
+    constexpr int NW = GDN_DECODE_NT / 32;
+    constexpr int ROWS_PER_WARP = RB / NW;
     constexpr int UNROLL = 4;
+    static_assert(ROWS_PER_WARP >= RPW && ROWS_PER_WARP % RPW == 0, "row split");
     static_assert(ROWS_PER_WARP % (RPW * UNROLL) == 0 || ROWS_PER_WARP < RPW * UNROLL, "row split");
     constexpr int STEP = (ROWS_PER_WARP < RPW * UNROLL) ? ROWS_PER_WARP : RPW * UNROLL;
     constexpr int U = STEP / RPW;             // row groups per iteration
 
-    const int bh = blockIdx.x;                // b * H + h
+    const int bh = blockIdx.x / (DV / RB);    // b * H + h
+    const int rblk = blockIdx.x % (DV / RB);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int sub = lane / LPR;               // which of the RPW rows this lane serves
     const int col = (lane % LPR) * 4;
@@ -88,7 +102,7 @@ __global__ void __launch_bounds__(256) gdn_decode_step_kernel(const T* __restric
     const float kq = row_dot<LPR>(k4, q4);      // k . q over the row's lanes
 
     float* S = state + (size_t)bh * DV * DK;
-    const int row0 = warp * ROWS_PER_WARP;
+    const int row0 = rblk * RB + warp * ROWS_PER_WARP;
 #pragma unroll
     for (int base = 0; base < ROWS_PER_WARP; base += STEP) {
         float4 s[U];
@@ -115,8 +129,9 @@ __global__ void __launch_bounds__(256) gdn_decode_step_kernel(const T* __restric
 // committed state, which is only read.  The state after every token is written to states_out, so
 // that the caller keeps the one after the last accepted token and drops the rest.
 //
-// Mapping: one CTA (8 warps) per (b, h); the whole dv x dk state of the pair lives in registers for
-// the Tk tokens (each lane holds NR float4s of its rows), is read from HBM once and written Tk times.
+// Mapping: one CTA (8 warps) per block of GDN_DECODE_RB rows of one (b, h) state; the block lives in
+// registers for the Tk tokens (each lane holds NR float4s of its rows), is read from HBM once and
+// written Tk times.
 template <typename T, int DK, int DV, bool NORM>
 __global__ void __launch_bounds__(256) gdn_decode_verify_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                             const T* __restrict__ v, const float* __restrict__ g,
@@ -127,16 +142,18 @@ __global__ void __launch_bounds__(256) gdn_decode_verify_kernel(const T* __restr
 {
     constexpr int LPR = DK / 4;               // lanes per row
     constexpr int RPW = 32 / LPR;             // rows handled by one warp at once
-    constexpr int ROWS_PER_WARP = DV / 8;
+    constexpr int RB = (GDN_DECODE_RB < DV) ? GDN_DECODE_RB : DV;   // rows of the state per CTA
+    constexpr int ROWS_PER_WARP = RB / 8;
     constexpr int NR = ROWS_PER_WARP / RPW;   // rows held by one lane
-    static_assert(ROWS_PER_WARP % RPW == 0, "row split");
+    static_assert(ROWS_PER_WARP >= RPW && ROWS_PER_WARP % RPW == 0, "row split");
 
-    const int bh = blockIdx.x;                // b * H + h
+    const int bh = blockIdx.x / (DV / RB);    // b * H + h
+    const int rblk = blockIdx.x % (DV / RB);
     const int b = bh / H, h = bh - b * H;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int sub = lane / LPR;
     const int col = (lane % LPR) * 4;
-    const int row0 = warp * ROWS_PER_WARP + sub;
+    const int row0 = rblk * RB + warp * ROWS_PER_WARP + sub;
     const float scale = rsqrtf((float)DK);
 
     float4 s[NR];
