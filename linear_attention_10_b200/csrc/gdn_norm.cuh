@@ -1,10 +1,11 @@
 // gdn_norm.cuh -- L2 normalisation of raw q and k inside the library (sm_100a).
 //
 // The method takes L2-normalised q_t and k_t per (token, head).  With the GDN_QK_L2NORM flag the
-// caller passes them raw and the library normalises: x / max(||x||_2, 1e-12), the norm summed in
-// fp32, and the result rounded to the storage dtype -- the same steps, in the same order, in the
-// prefill's pre-pass and inside the decode and verify kernels, so that every path sees the same
-// normalised values.  A row of DK elements is held by DK/4 lanes as four consecutive elements each
+// caller passes them raw and the library normalises: x / max(||x||_2, 1e-12), taken as
+// x * rsqrt(max(sum x^2, 1e-24)) with the sum in fp32 (one reciprocal square root per vector instead
+// of a square root and a divide), and the result rounded to the storage dtype -- the same steps, in
+// the same order, in the prefill's pre-pass and inside the decode and verify kernels, so that every
+// path sees the same normalised values.  A row of DK elements is held by DK/4 lanes as four consecutive elements each
 // and its sum of squares is reduced over those lanes with xor shuffles, as row_dot does.
 #pragma once
 
@@ -14,7 +15,7 @@
 
 namespace gdn {
 
-__device__ __forceinline__ float l2_inv_norm(float sum_sq) { return 1.f / fmaxf(sqrtf(sum_sq), 1e-12f); }
+__device__ __forceinline__ float l2_inv_norm(float sum_sq) { return rsqrtf(fmaxf(sum_sq, 1e-24f)); }
 
 // x -> x * inv, rounded to T and widened back (the value the tensor cores or the decode step use)
 template <typename T>
@@ -67,7 +68,9 @@ __global__ void __launch_bounds__(256) gdn_l2norm_kernel(const T* __restrict__ q
             float ss = a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
 #pragma unroll
             for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-            const float4 y = scale_round<T>(a, l2_inv_norm(ss));
+            // the store rounds to T once (scale_round's round-and-widen would only repeat it)
+            const float inv = l2_inv_norm(ss);
+            const float4 y = make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
             if (v < nvec) Elem<T>::st4(dst + v * DK + col, y);
         }
     }
