@@ -67,11 +67,13 @@ KERNELS = {
 }
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from the last ncu capture of that kernel
 # on the bench workload (None until captured, and reset whenever the kernel changes).  The decode
-# figure undercounts writes: ncu starts each replay from a clean L2, and about 57 MB of the written
-# state is still resident (dirty) in L2 when the launch ends.
+# and verify figures undercount writes: ncu starts each replay from a clean L2, and 56-58 MB of the
+# written states are still resident (dirty) in L2 when the launch ends.
 TRAFFIC = {
     "gdn_scan_bf16_kernel": 203.15e6 + 27.64e6,
     "gdn_prep_bf16_kernel": 68.22e6 + 48.88e6,
+    "gdn_decode_step_kernel": 135.83e6 + 77.84e6,
+    "gdn_decode_verify_kernel": 140.59e6 + 479.75e6,
 }
 
 
