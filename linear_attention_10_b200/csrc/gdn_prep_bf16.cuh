@@ -16,6 +16,11 @@
 //   T21 = -T22 (A21 T11),
 //
 // which shortens the dependent chain of the substitution from 31 steps to 15.
+//
+// The cross-chunk Gram G' = [K; Q] K_prev^T (the scan's MMA_x operand) is issued by a second thread
+// with the A descriptor started 64 rows before the tile, so its rows land in tensor-memory lanes
+// 64..127: warps 2 and 3, which only those lanes are visible to, split and store it while warps 0
+// and 1 gate the chunk's own Gram rows in lanes 0..63.
 #pragma once
 
 #include <cuda.h>
@@ -29,22 +34,29 @@ namespace gdn {
 template <int DK>
 struct PrepBf16Smem {
     static constexpr int NP = DK / 64;
+    // The tensor cores read 128 rows of an A operand.  The chunk's Gram reads the tile's 64 rows and
+    // the 64 rows after them; G' reads 64 rows before the tile and the tile.  Each tile therefore has
+    // at least 8 KB of this CTA's shared memory on both sides.
     static constexpr uint32_t kTile = NP * 8192;                      // [K;Q] bf16: NP panels x 64 rows x 128 B
-    static constexpr uint32_t oTile = 0;                              // two buffers
-    static constexpr uint32_t oPrev = 2 * kTile;                      // previous chunk's K: NP x 32 rows x 128 B
+    static constexpr uint32_t oPrev = 0;                              // previous chunk's K: NP x 32 rows x 128 B
+    static constexpr uint32_t oTile = 8192;                           // two buffers
     static constexpr int LD = 36;                                     // row pitch: 16-byte rows, no bank conflicts
-    static constexpr uint32_t oG = oPrev + NP * 4096;                 // [32][LD] A
+    static constexpr uint32_t oG = oTile + 2 * kTile;                 // [32][LD] A
     static constexpr uint32_t oP = oG + 32 * LD * 4;                  // [32][LD] P
     static constexpr uint32_t oT = oP + 32 * LD * 4;                  // [32][LD] T
-    static constexpr uint32_t oM = oT + 32 * LD * 4;                  // [16][17] A21 T11
-    static constexpr uint32_t oGam = oM + 16 * 17 * 4;
+    static constexpr int LM = 16;                                     // pitch of M (2-way write conflicts)
+    static constexpr uint32_t oM = oT + 32 * LD * 4;                  // [16][LM] A21 T11
+    static constexpr uint32_t oGam = oM + 16 * LM * 4;
     static constexpr uint32_t oBet = oGam + 128;
     static constexpr uint32_t oAlph = oBet + 128;                     // per-token decays exp(g), one spare
-    static constexpr uint32_t oBar = oAlph + 136;                      // tile_full[2], mma, drain, prev_full, cross
-    static constexpr uint32_t oTmem = oBar + 48;
+    static constexpr uint32_t oBar = oAlph + 136;   // tile_full[2], mma, drain[2], prev_full, cross
+    static constexpr uint32_t oTmem = oBar + 56;
     static constexpr uint32_t oAbort = oTmem + 4;
     static constexpr uint32_t kTotal = oAbort + 4;
     static constexpr uint32_t kBytes = kTotal + 1024;
+    static_assert(NP * 4096 <= oTile, "previous-K buffer; 8 KB before the first tile");
+    static_assert(kTotal >= oG + 8192, "rows read after the last tile's last panel");
+    static_assert(kBytes <= 57344, "four CTAs per SM");
 };
 
 template <int DK>
@@ -72,10 +84,10 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
     float* bet = reinterpret_cast<float*>(sm + L::oBet);
     float* alph = reinterpret_cast<float*>(sm + L::oAlph);
     uint64_t* tile_full = reinterpret_cast<uint64_t*>(sm + L::oBar);
-    uint64_t* mma_bar = tile_full + 2;
-    uint64_t* drain = tile_full + 3;
-    uint64_t* prev_full = tile_full + 4;
-    uint64_t* cross_bar = tile_full + 5;      // the cross-chunk Gram product (and all before it) done
+    uint64_t* mma_bar = tile_full + 2;        // the chunk's Gram product done
+    uint64_t* drain = tile_full + 3;          // [2]: after an abort, the products of threads 0 / 96
+    uint64_t* prev_full = tile_full + 5;
+    uint64_t* cross_bar = tile_full + 6;      // the cross-chunk Gram product (thread 96's) done
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::oTmem);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::oAbort);
 
@@ -85,7 +97,8 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
         mbar_init(&tile_full[0], 1);
         mbar_init(&tile_full[1], 1);
         mbar_init(mma_bar, 1);
-        mbar_init(drain, 1);
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
         mbar_init(prev_full, 1);
         mbar_init(cross_bar, 1);
         *abort_flag = 0;
@@ -102,7 +115,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
 
     // whether chunk gc has a previous chunk in its sequence (then the cross-chunk Gram is built)
     auto has_prev = [&](int gc) { return gc > chunk_off[chunk_tab[gc].x]; };
-    // copies the [K; Q] rows of one item into tile buffer `b` (thread 0 only)
+    // copies the [K; Q] rows of one item into tile buffer `b` (one thread per fill)
     auto issue_tile = [&](int item, int b) {
         const int gc = item / H, h = item % H;
         const int t0 = chunk_tab[gc].y;
@@ -114,8 +127,8 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
             tma_load_2d(dst + p * 8192 + 4096, &tm_q, h * DK + p * 64, t0, &tile_full[b]);
         }
     };
-    // copies the previous chunk's K rows of one item into the single previous-K buffer (thread 0
-    // only; issued once the buffer's last reader has completed).  An item that starts its sequence
+    // copies the previous chunk's K rows of one item into the single previous-K buffer (one thread;
+    // issued once the buffer's last reader has completed).  An item that starts its sequence
     // loads its own K rows instead, so that the buffer's barrier completes once per item.
     auto issue_prev = [&](int item) {
         const int gc = item / H, h = item % H;
@@ -151,10 +164,9 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
         const int Lr = chunk_tab[gc].z;
         const bool prev = has_prev(gc);
 
-        // Gram products D[r][n] = [K; Q]_r . K_n on the tensor cores (rows 64..127 unused)
+        // Gram products D[r][n] = [K; Q]_r . K_n on the tensor cores, rows in lanes 0..63 (thread 0)
         if (tid == 0) {
-            if (!mbar_wait(&tile_full[b], (iter >> 1) & 1u, abort_flag) ||
-                !mbar_wait(prev_full, iter & 1u, abort_flag)) {
+            if (!mbar_wait(&tile_full[b], (iter >> 1) & 1u, abort_flag)) {
                 tc_abort(status, abort_flag);
             } else {
                 tc_fence_after();
@@ -165,15 +177,25 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
                     mma_bf16(tmem, a + o, a + o, idG, ks > 0);
                 }
                 mma_commit(mma_bar);
+                if (!mbar_wait(mma_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
+            }
+        } else if (tid == 96) {
+            // G' = [K; Q] K_prev^T (thread 96), completes while the gates are applied.  A starts 64
+            // rows (8 KB) before the tile, so row r of [K; Q] is row 64 + r of the product: lanes
+            // 64..127, and its columns 32..63
+            if (!mbar_wait(&tile_full[b], (iter >> 1) & 1u, abort_flag) ||
+                !mbar_wait(prev_full, iter & 1u, abort_flag)) {
+                tc_abort(status, abort_flag);
+            } else {
+                tc_fence_after();
                 if (prev) {
-                    // G' = [K; Q] K_prev^T, completes while the gates are applied
+                    const uint64_t a = sw128_desc(sbase + L::oTile + b * L::kTile - 8192, 0, 64);
                     const uint64_t bp = sw128_desc(sbase + L::oPrev, 0, 32);
 #pragma unroll
                     for (int ks = 0; ks < DK / 16; ++ks)
                         mma_bf16(tmem + 32, a + sw128_ks_off(ks, 64), bp + sw128_ks_off(ks, 32), idG, ks > 0);
                 }
                 mma_commit(cross_bar);
-                if (!mbar_wait(mma_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
             }
         }
         if (warp == 2) {
@@ -217,21 +239,25 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
                 asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + q * 16), "f"(vals[4 * q]),
                              "f"(vals[4 * q + 1]), "f"(vals[4 * q + 2]), "f"(vals[4 * q + 3]));
             GDN_PREP_TRACE(iter, 6);
-            // the tile buffers are free once G' has been formed: fetch the item after next and the
-            // next item's previous-chunk keys
-            if (!mbar_wait(cross_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
+        } else {
+            // warps 2 and 3: the tile buffers are free once G' has been formed (the chunk's own Gram
+            // was waited for before the barrier above): fetch the item after next and the next item's
+            // previous-chunk keys, then split G'
+            if (tid == 64 && !mbar_wait(cross_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
+            named_bar(1, 64);
             tc_fence_after();
-            if (tid == 0 && !*abort_flag) {
+            if (tid == 64 && !*abort_flag) {
                 if (item + 2 * (int)gridDim.x < nitems) issue_tile(item + 2 * gridDim.x, b);
                 if (item + (int)gridDim.x < nitems) issue_prev(item + gridDim.x);
             }
             if (prev) {
-                // row (32 w + r) of G' -> three bf16 parts, K-major 64-byte-swizzled A operand rows
+                // row (32 (w - 2) + lane) of G', in lane 32 w + lane -> three bf16 parts, K-major
+                // 64-byte-swizzled A operand rows
                 float e[32];
                 tmem_ld32(tmem + 32 + ((uint32_t)(warp * 32) << 16), e);
                 tmem_ld_wait();
                 uint8_t* rec = op + ((size_t)gc * H + h) * kOpBytesB + kOpBCross;
-                const int row = warp * 32 + r;
+                const int row = (warp - 2) * 32 + lane;
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8) {
                     uint32_t w1[4], w2[4], w3[4];
@@ -277,8 +303,8 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
                 a0 = fmaf(am, Tm[m * LD + c], a0);
                 a1 = fmaf(am, Tm[m * LD + c + 1], a1);
             }
-            M1[r * 17 + c] = a0;
-            M1[r * 17 + c + 1] = a1;
+            M1[r * L::LM + c] = a0;
+            M1[r * L::LM + c + 1] = a1;
         }
         __syncthreads();
         {
@@ -288,8 +314,8 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
                 const float tm = Tm[(16 + r) * LD + 16 + m];
-                a0 = fmaf(tm, M1[m * 17 + c], a0);
-                a1 = fmaf(tm, M1[m * 17 + c + 1], a1);
+                a0 = fmaf(tm, M1[m * L::LM + c], a0);
+                a1 = fmaf(tm, M1[m * L::LM + c + 1], a1);
             }
             Tm[(16 + r) * LD + c] = -a0;
             Tm[(16 + r) * LD + c + 1] = -a1;
@@ -297,45 +323,53 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
         __syncthreads();
         GDN_PREP_TRACE(iter, 3);
 
-        // operator record: rows i of T'' = T diag(beta) and of P T'', TF32 hi/lo, swizzled image
+        // operator record: thread (i, cb) forms columns 8 cb .. 8 cb + 7 of row i of T'' = T diag(beta)
+        // and of P T'' = (P T) diag(beta), and writes each as three bf16 parts of 16 bytes into the
+        // 64-byte-swizzled A-operand image (rows 0..31: T'', rows 32..63: P T'')
         uint8_t* dst = op + ((size_t)gc * H + h) * kOpBytesB;
         {
-            const int j = lane, rg = warp;
-            const float bj = bet[j];
-            float tc[32];
+            const int i = tid >> 2, c0 = (tid & 3) * 8;
+            const float4 b0 = *reinterpret_cast<const float4*>(bet + c0);
+            const float4 b1 = *reinterpret_cast<const float4*>(bet + c0 + 4);
+            const float bc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            float acc[8];
 #pragma unroll
-            for (int m = 0; m < 32; ++m) tc[m] = Tm[m * LD + j] * bj;
+            for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+            const float4* prow = reinterpret_cast<const float4*>(P + i * LD);
 #pragma unroll
-            for (int rr = 0; rr < 8; ++rr) {
-                const int i = rg * 8 + rr;
-                float acc = 0.f;
-                const float4* prow = reinterpret_cast<const float4*>(P + i * LD);
+            for (int q = 0; q < 8; ++q) {
+                const float4 pv = prow[q];
+                const float pm[4] = {pv.x, pv.y, pv.z, pv.w};
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 pv = prow[q];
-                    acc = fmaf(pv.x, tc[4 * q], acc);
-                    acc = fmaf(pv.y, tc[4 * q + 1], acc);
-                    acc = fmaf(pv.z, tc[4 * q + 2], acc);
-                    acc = fmaf(pv.w, tc[4 * q + 3], acc);
-                }
-                // three bf16 parts, lanes j and j+1 packed into one 32-bit store by the even lane
-                const float tv = Tm[i * LD + j] * bj;
-                const float tn = __shfl_xor_sync(0xffffffffu, tv, 1);
-                const float an = __shfl_xor_sync(0xffffffffu, acc, 1);
-                if ((j & 1) == 0) {
-                    uint32_t w1, w2, w3;
-                    bf16x2_split3(tv, tn, w1, w2, w3);
-                    uint32_t o = sw64_off_h(i, j);
-                    stg32(dst + o, w1);
-                    stg32(dst + kOpBPart + o, w2);
-                    stg32(dst + 2 * kOpBPart + o, w3);
-                    bf16x2_split3(acc, an, w1, w2, w3);
-                    o = sw64_off_h(32 + i, j);
-                    stg32(dst + o, w1);
-                    stg32(dst + kOpBPart + o, w2);
-                    stg32(dst + 2 * kOpBPart + o, w3);
+                for (int e = 0; e < 4; ++e) {
+                    const float4* trow = reinterpret_cast<const float4*>(Tm + (4 * q + e) * LD + c0);
+                    const float4 t0 = trow[0], t1 = trow[1];
+                    acc[0] = fmaf(pm[e], t0.x, acc[0]);
+                    acc[1] = fmaf(pm[e], t0.y, acc[1]);
+                    acc[2] = fmaf(pm[e], t0.z, acc[2]);
+                    acc[3] = fmaf(pm[e], t0.w, acc[3]);
+                    acc[4] = fmaf(pm[e], t1.x, acc[4]);
+                    acc[5] = fmaf(pm[e], t1.y, acc[5]);
+                    acc[6] = fmaf(pm[e], t1.z, acc[6]);
+                    acc[7] = fmaf(pm[e], t1.w, acc[7]);
                 }
             }
+            const float4* tri = reinterpret_cast<const float4*>(Tm + i * LD + c0);
+            const float4 ti0 = tri[0], ti1 = tri[1];
+            const float tv[8] = {ti0.x, ti0.y, ti0.z, ti0.w, ti1.x, ti1.y, ti1.z, ti1.w};
+            uint32_t w1[4], w2[4], w3[4], x1[4], x2[4], x3[4];
+#pragma unroll
+            for (int c = 0; c < 8; c += 2) {
+                bf16x2_split3(tv[c] * bc[c], tv[c + 1] * bc[c + 1], w1[c / 2], w2[c / 2], w3[c / 2]);
+                bf16x2_split3(acc[c] * bc[c], acc[c + 1] * bc[c + 1], x1[c / 2], x2[c / 2], x3[c / 2]);
+            }
+            const uint32_t ot = sw64_off_h(i, c0), op2 = sw64_off_h(32 + i, c0);
+            stg128(dst + ot, w1);
+            stg128(dst + kOpBPart + ot, w2);
+            stg128(dst + 2 * kOpBPart + ot, w3);
+            stg128(dst + op2, x1);
+            stg128(dst + kOpBPart + op2, x2);
+            stg128(dst + 2 * kOpBPart + op2, x3);
         }
         if (tid < 80) {
             float* gt = reinterpret_cast<float*>(dst + kOpBGate);
@@ -352,11 +386,12 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
     }
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && *abort_flag) {
-        // after a timeout, give copies and an MMA still in flight a bounded time to finish
-        mma_commit(drain);
+    if ((tid == 0 || tid == 96) && *abort_flag) {
+        // after a timeout, give the products this thread issued a bounded time to finish
+        uint64_t* d = &drain[tid == 0 ? 0 : 1];
+        mma_commit(d);
         volatile int never = 0;
-        mbar_wait(drain, 0, &never, 100000000ull);
+        mbar_wait(d, 0, &never, 100000000ull);
     }
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 64);
