@@ -113,6 +113,30 @@ def max_over_ranks(x, world, device=None):
     return float(t.item())
 
 
+def timed_passes(fn, n, world, dev, stream):
+    """Times n calls of fn(i) on `stream` with CUDA events (max over ranks), then runs them again with
+    an event pair around every library launch; returns (ms of the first pass, per-kernel profile of
+    the second).  The first pass has no events between launches, which would serialise them."""
+    import torch
+    import torch.distributed as dist
+    from linear_attention_10_b200 import gdn
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    gdn.gdn_profile_start()
+    for i in range(n):
+        fn(i)
+    torch.cuda.synchronize()
+    return ms, gdn.gdn_profile_stop()
+
+
 def job_throughput(units_per_rank_step, steps, world, max_ms):
     """Whole-job units per second: all ranks' units over the slowest rank's time."""
     return units_per_rank_step * world * steps / (max_ms / 1e3)
@@ -282,23 +306,35 @@ def run_ours(args, rank, world, local_rank):
     clocks.start()
     time.sleep(0.3)
 
-    # ---- timed region: K prefill steps ----
+    # ---- timed region: K prefill steps, as a caller runs them.  No event is recorded between the
+    # three launches of a step here: an event there serialises them (the prep and scan kernels are
+    # launched as programmatic dependents of their predecessors) and costs ~20 us per step ----
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    gdn.gdn_profile_start()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for i in range(args.steps):
         step(i)
     ev1.record(stream)
     torch.cuda.synchronize()
-    prof = gdn.gdn_profile_stop()
     if world > 1:
         dist.barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     if gdn.gdn_get_device_status() != 0:
         raise RuntimeError("device status error in the timed region")
+    # ---- per-kernel durations: the same K steps again, with an event pair around every launch on the
+    # launching stream (the roofline of the dominant kernel and the launch count come from here) ----
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    gdn.gdn_profile_start()
+    for i in range(args.steps):
+        step(i)
+    torch.cuda.synchronize()
+    prof = gdn.gdn_profile_stop()
+    if gdn.gdn_get_device_status() != 0:
+        raise RuntimeError("device status error in the profiled pass")
     ms_per_step = ms / args.steps
     value = job_throughput(T_PREFILL, args.steps, world, ms)
 
@@ -377,18 +413,9 @@ def run_ours(args, rank, world, local_rank):
         for s in range(3):
             gdn.gdn_decode_step(dd["q"][s], dd["k"][s], dd["v"][s], dd["g"][s], dd["beta"][s], S, out=dout)
         S.copy_(dd["state"])
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        gdn.gdn_profile_start()
-        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        d0.record(stream)
-        for s in range(w.decode_steps):
-            gdn.gdn_decode_step(dd["q"][s], dd["k"][s], dd["v"][s], dd["g"][s], dd["beta"][s], S, out=dout)
-        d1.record(stream)
-        torch.cuda.synchronize()
-        dprof = gdn.gdn_profile_stop()
-        dms = max_over_ranks(d0.elapsed_time(d1), world, dev)
+        dms, dprof = timed_passes(lambda s: gdn.gdn_decode_step(dd["q"][s], dd["k"][s], dd["v"][s], dd["g"][s],
+                                                                dd["beta"][s], S, out=dout),
+                                  w.decode_steps, world, dev, stream)
         name = "gdn_decode_step_kernel"
         kms, kl = dprof.get(name, (dms, w.decode_steps))
         B_, H_, d_ = w.decode_batch, w.H, w.dk
@@ -448,15 +475,7 @@ def run_ours(args, rank, world, local_rank):
             run_n()
         torch.cuda.synchronize()
         reps = 20
-        gdn.gdn_profile_start()
-        n0, n1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n0.record(stream)
-        for _ in range(reps):
-            run_n()
-        n1.record(stream)
-        torch.cuda.synchronize()
-        nprof = gdn.gdn_profile_stop()
-        nms = max_over_ranks(n0.elapsed_time(n1), world, dev)
+        nms, nprof = timed_passes(lambda i: run_n(), reps, world, dev, stream)
         name = "gdn_l2norm_kernel"
         kms, kl = nprof.get(name, (nms, reps))
         bytes_per_launch = 4 * T_PREFILL * H * D * 2          # q, k read and their normalised copies written
@@ -484,19 +503,8 @@ def run_ours(args, rank, world, local_rank):
                                               states_out=vst, out=vout)
         for _ in range(3):
             run_v()
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
         reps = 100
-        gdn.gdn_profile_start()
-        v0, v1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        v0.record(stream)
-        for _ in range(reps):
-            run_v()
-        v1.record(stream)
-        torch.cuda.synchronize()
-        vprof = gdn.gdn_profile_stop()
-        vms = max_over_ranks(v0.elapsed_time(v1), world, dev)
+        vms, vprof = timed_passes(lambda i: run_v(), reps, world, dev, stream)
         name = "gdn_decode_verify_kernel"
         kms, kl = vprof.get(name, (vms, reps))
         per_bh = (1 + Tk) * d_ * d_ * 4 + Tk * ((3 * d_) * 2 + 2 * 4 + d_ * 2)
@@ -526,6 +534,7 @@ def run_ours(args, rank, world, local_rank):
     roofline = dict(kernel=dom, bound=spec["bound"], achieved=ach, peak=pk, unit=pu, frac=ach / pk,
                     peak_source=pdesc, flops_per_launch=flops, avg_launch_us=kms / kl * 1e3,
                     traffic=TRAFFIC.get(dom),
+                    timing="CUDA events around each launch, in a second pass over the same K steps",
                     kernels={n: dict(avg_us=v[0] / v[1] * 1e3, launches=v[1], share=v[0] / total_prof_ms)
                              for n, v in prof.items()})
     # whole-call roofline of the method (TF32 3x split vs HBM), as the metric defines "% of roofline"

@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <mutex>
 #include <type_traits>
+#include <utility>
 #include <string>
 #include <vector>
 
@@ -83,6 +84,25 @@ struct ProfScope {
         g_prof_recs.push_back(rec);
     }
 };
+
+// Launches `kernel` as a programmatic dependent of the previous kernel in the stream: it may become
+// resident before that kernel ends and waits for it (grid_dep_wait) before reading its results.
+template <typename... Params, typename... Args>
+static cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                    Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -236,9 +256,9 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         const int64_t cap = (int64_t)g_num_sms * 4;
         const unsigned grid = (unsigned)(items < cap ? items : cap);
         ProfScope prof("gdn_prep_bf16_kernel", st);
-        k1<<<grid, 128, PL::kBytes, st>>>(tq, tk, g, beta, meta, chunk_off, chunk_tab, reinterpret_cast<uint8_t*>(op),
-                                          H, status);
-        if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
+        if (launch_dependent(k1, dim3(grid), dim3(128), PL::kBytes, st, tq, tk, g, beta, meta, chunk_off, chunk_tab,
+                             reinterpret_cast<uint8_t*>(op), H, status) != cudaSuccess)
+            return GDN_ERR_LAUNCH;
       }
     } else if (lay.nc_max > 0 && T_total > 0) {
         using PL = PrepSmem<T, DK>;
@@ -249,9 +269,10 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         const int64_t cap = (int64_t)g_num_sms * 4;
         const unsigned grid = (unsigned)(items < cap ? items : cap);
         ProfScope prof("gdn_prep_kernel", st);
-        k1<<<grid, 128, PL::kBytes, st>>>(static_cast<const T*>(q), static_cast<const T*>(k), g, beta, meta,
-                                          chunk_tab, op, H, status);
-        if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
+        if (launch_dependent(k1, dim3(grid), dim3(128), PL::kBytes, st, static_cast<const T*>(q),
+                             static_cast<const T*>(k), g, beta, (const int*)meta, (const int4*)chunk_tab, op, H,
+                             status) != cudaSuccess)
+            return GDN_ERR_LAUNCH;
     }
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         // bf16 inputs: operands staged by tensor maps, bf16 tensor-core products for K and Q
@@ -267,11 +288,13 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
             return GDN_ERR_LAUNCH;
         {
             ProfScope prof("gdn_scan_bf16_kernel", st);
-            kb<<<dim3((unsigned)N, H, DV / MSB), kScanBf16Threads, SB::kBytes, st>>>(
-                tq, tk, tv, meta, chunk_off, chunk_tab, reinterpret_cast<const uint8_t*>(op), state_in,
-                static_cast<__nv_bfloat16*>(out), state_out, cuts.snaps, H, status);
+            if (launch_dependent(kb, dim3((unsigned)N, H, DV / MSB), dim3(kScanBf16Threads), SB::kBytes, st, tq, tk,
+                                 tv, (const int*)meta, (const int*)chunk_off, (const int4*)chunk_tab,
+                                 reinterpret_cast<const uint8_t*>(op), state_in, static_cast<__nv_bfloat16*>(out),
+                                 state_out, cuts.snaps, H, status) != cudaSuccess)
+                return GDN_ERR_LAUNCH;
         }
-        return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
+        return GDN_OK;
     }
     // state rows per CTA and CTAs per SM of the scan (compile-time tuning knobs)
     constexpr int MS = GDN_SCAN_MS;
@@ -286,11 +309,13 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         return GDN_ERR_LAUNCH;
     {
         ProfScope prof("gdn_scan_tc_kernel", st);
-        k2<<<dim3((unsigned)N, H, DV / MS), 256, SL::kBytes, st>>>(
-            static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), meta, chunk_off,
-            chunk_tab, op, state_in, static_cast<T*>(out), state_out, cuts.snaps, H, status);
+        if (launch_dependent(k2, dim3((unsigned)N, H, DV / MS), dim3(256), SL::kBytes, st, static_cast<const T*>(q),
+                             static_cast<const T*>(k), static_cast<const T*>(v), (const int*)meta,
+                             (const int*)chunk_off, (const int4*)chunk_tab, (const float*)op, state_in,
+                             static_cast<T*>(out), state_out, cuts.snaps, H, status) != cudaSuccess)
+            return GDN_ERR_LAUNCH;
     }
-    return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
+    return GDN_OK;
 }
 
 template <typename T>

@@ -12,6 +12,7 @@
 #pragma once
 
 #include "gdn_common.cuh"
+#include "gdn_sm100.cuh"
 
 namespace gdn {
 
@@ -91,6 +92,9 @@ __global__ void __launch_bounds__(1024) gdn_plan_kernel(const int32_t* __restric
     __shared__ int warp_tot[32];
     __shared__ int s_err;
     __shared__ int s_running;
+    // the prep kernel is launched as a dependent: let it become resident while this runs (it waits
+    // for this kernel's writes before reading them)
+    sm100::grid_dep_launch();
     if (threadIdx.x == 0) { s_err = 0; s_running = 0; }
     __syncthreads();
     auto start_of = [&](int n) -> int64_t { return cu ? (int64_t)cu[n] : (int64_t)n * fixed_len; };

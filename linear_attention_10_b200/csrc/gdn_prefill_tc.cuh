@@ -247,6 +247,9 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const T* __restrict__ 
     using L = PrepSmem<T, DK>;
     constexpr bool EXACT = L::EXACT;
     constexpr int C = kChunk;
+    // launched as a dependent of the plan kernel: its chunk table is read below
+    grid_dep_wait();
+    grid_dep_launch();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -499,6 +502,8 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
     using namespace sm100;
     using L = ScanSmem<T, DK, MS, STAGES>;
     constexpr bool EXACT = L::EXACT;
+    // launched as a dependent of the prep kernel: its records (and the plan's table) are read below
+    grid_dep_wait();
     static_assert(MS == 16 || MS == 32, "MS");
     static_assert(DK == 64 || DK == 128, "DK");
     static_assert(DV % MS == 0, "DV");

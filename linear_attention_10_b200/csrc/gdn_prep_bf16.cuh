@@ -73,6 +73,9 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
     using L = PrepBf16Smem<DK>;
     constexpr int NP = L::NP;
     constexpr int LD = L::LD;
+    // launched as a dependent of the plan kernel: its chunk table is read below
+    grid_dep_wait();
+    grid_dep_launch();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);

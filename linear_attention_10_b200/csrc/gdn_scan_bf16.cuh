@@ -108,6 +108,8 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
 {
     using namespace sm100;
     using L = ScanBf16Smem<DK, MS, STAGES>;
+    // launched as a dependent of the prep kernel: its records (and the plan's table) are read below
+    grid_dep_wait();
     static_assert(MS == 32, "bf16 scan: 32 state rows per CTA");
     static_assert(DK == 64 || DK == 128, "DK");
     static_assert(DV % MS == 0, "DV");

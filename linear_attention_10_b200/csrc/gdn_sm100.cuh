@@ -103,6 +103,14 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 // ------------------------------------------------------------------------------------------------
 // fences and named barriers
 // ------------------------------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched as a dependent of the previous kernel in its
+// stream may become resident before that kernel ends; grid_dep_wait() returns once the previous
+// kernel has completed and its memory writes are visible (at once when there is no such
+// dependency).  grid_dep_launch() lets the next kernel, if it is launched as a dependent, be
+// scheduled now; it does not relax that kernel's own wait.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // generic-proxy shared-memory writes -> visible to the async proxy (tensor-core operand reads)
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
