@@ -181,8 +181,9 @@ static EncodeTiledFn encode_tiled()
 
 // [rows, inner] bf16 matrix with row stride `row_elems`, tiles of box_rows x box_inner elements;
 // rows past the end read as zeros.
+// swizzle: 128 or 64 (bytes of the swizzle span), 0 for none
 static bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_elems,
-                           uint32_t box_inner, uint32_t box_rows, bool swizzle128)
+                           uint32_t box_inner, uint32_t box_rows, int swizzle)
 {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
@@ -191,7 +192,9 @@ static bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uin
     cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_INTERLEAVE_NONE,
+              swizzle == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                             : (swizzle == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE),
               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -241,9 +244,9 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
     CUtensorMap tq{}, tk{}, tv{};
     if constexpr (kBf16) {
         const uint64_t Tn = (uint64_t)(T_total > 0 ? T_total : 1);
-        if (!make_tmap_bf16(&tq, q, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, true) ||
-            !make_tmap_bf16(&tk, k, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, true) ||
-            !make_tmap_bf16(&tv, v, (uint64_t)H * DV, Tn, (uint64_t)H * DV, 32, 32, false))
+        if (!make_tmap_bf16(&tq, q, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, 128) ||
+            !make_tmap_bf16(&tk, k, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, 128) ||
+            !make_tmap_bf16(&tv, v, (uint64_t)H * DV, Tn, (uint64_t)H * DV, 32, 32, 64))
             return GDN_ERR_CUDA;
     }
     if constexpr (kBf16) {

@@ -55,7 +55,8 @@ struct ScanBf16Smem {
     static constexpr uint32_t oAKQ = 0;                               // [K;Q] bf16: NP panels x 64 rows x 128 B
     static constexpr uint32_t oOp = oAKQ + NP * 8192;                 // operator record: parts, G' parts, gates
     static constexpr uint32_t oCt = oOp + ((kOpBCopyBytes + 15) & ~15u);    // the chunk's table entry (int4)
-    static constexpr uint32_t oV = oOp + ((kOpBCopyBytes + 16 + 1023) & ~1023u);  // V tile: 32 rows x MS bf16
+    // V tile: 32 rows x MS bf16 (64-byte rows, 64-byte swizzle: 16-byte chunk j of row r at j ^ ((r / 2) % 4))
+    static constexpr uint32_t oV = oOp + ((kOpBCopyBytes + 16 + 1023) & ~1023u);
     static constexpr uint32_t kStage = ((oV + 32 * MS * 2) + 1023) & ~1023u;
     static constexpr uint32_t kStageTx = NP * 2 * 4096 + kOpBCopyBytes + 32 * MS * 2;
     // shared by all stages
@@ -234,6 +235,19 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
             bool ok = mbar_wait(&full[s], phase_of(c), abort_flag) &&
                       mbar_wait(&bar_w[c & 1], (uint32_t)(c >> 1) & 1u, abort_flag);
             GDN_SCAN_TRACE(c, 1);
+            // W_c is ready well before MMA_x: read and sum its three parts while MMA_x still runs
+            tc_fence_after();
+            float wsum[MH];
+            {
+                float w1[MH], w2[MH], w3[MH];
+                const uint32_t tw = ((c & 1) ? tDW1 : tDW0) + lane_q + hf * MH;
+                tmem_ld<MH>(tw, w1);
+                tmem_ld<MH>(tw + MS, w2);
+                tmem_ld<MH>(tw + 2 * MS, w3);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < MH; ++i) wsum[i] = (w1[i] + w2[i]) + w3[i];
+            }
             // MMA_x of this chunk (which also covers MMA_c of the last one) or, at a segment start,
             // MMA_c of the last chunk alone
             if constexpr (CUTS) {
@@ -263,35 +277,30 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
             const float GamC = gate[64];
             // [X; Z] rows: Gamma_{c-1} W_c + G'_c U~_{c-1}  (chunk 0: W_0 = [K; Q] S_-1^T alone)
             float za[MH];
-            {
-                float w1[MH], w2[MH], w3[MH];
-                const uint32_t tw = ((c & 1) ? tDW1 : tDW0) + lane_q + hf * MH;
-                tmem_ld<MH>(tw, w1);
-                tmem_ld<MH>(tw + MS, w2);
-                tmem_ld<MH>(tw + 2 * MS, w3);
-                if (!first) {
-                    float x1[MH], x2[MH], x3[MH];
-                    const uint32_t tx = tD1 + lane_q + hf * MH;
-                    tmem_ld<MH>(tx, x1);
-                    tmem_ld<MH>(tx + MS, x2);
-                    tmem_ld<MH>(tx + 2 * MS, x3);
-                    tmem_ld_wait();
+            if (!first) {
+                float x1[MH], x2[MH], x3[MH];
+                const uint32_t tx = tD1 + lane_q + hf * MH;
+                tmem_ld<MH>(tx, x1);
+                tmem_ld<MH>(tx + MS, x2);
+                tmem_ld<MH>(tx + 2 * MS, x3);
+                tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < MH; ++i) za[i] = fmaf(GamPrev, (w1[i] + w2[i]) + w3[i], (x1[i] + x2[i]) + x3[i]);
-                } else {
-                    tmem_ld_wait();
+                for (int i = 0; i < MH; ++i) za[i] = fmaf(GamPrev, wsum[i], (x1[i] + x2[i]) + x3[i]);
+            } else {
 #pragma unroll
-                    for (int i = 0; i < MH; ++i) za[i] = (w1[i] + w2[i]) + w3[i];
-                }
+                for (int i = 0; i < MH; ++i) za[i] = wsum[i];
             }
             GDN_SCAN_TRACE(c, 3);
             if (q4 == 0) {
                 // Y = V - diag(Gamma) X (zero past the sequence end) -> bf16 parts of MMA_b's B
                 float vt[MH];
-                const uint4* vrow = reinterpret_cast<const uint4*>(stp + L::oV + lane * MS * 2 + hf * MH * 2);
+                const uint8_t* vrow = stp + L::oV + lane * MS * 2;
 #pragma unroll
                 for (int q8 = 0; q8 < MH / 8; ++q8) {
-                    const uint4 u = vrow[q8];
+                    // the swizzled position of 16-byte chunk (hf * MH / 8 + q8) of row `lane`: the 32
+                    // lanes of a warp then read distinct banks
+                    const int j = (hf * (MH / 8) + q8) ^ ((lane >> 1) & 3);
+                    const uint4 u = *reinterpret_cast<const uint4*>(vrow + j * 16);
                     const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
