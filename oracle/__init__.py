@@ -13,6 +13,13 @@ What is computed and why (each function cites its source):
                      (Ferrite project page, Design section 03 "Chunked Gated DeltaNet": chunks of
                      32 rows, WY/UT form).
 * ``brute_force`` -- explicit d x d matrix products of the unrolled recurrence, numpy, for T <= 8.
+* ``decode_step``, ``decode_verify``, ``decode_verify_tree`` -- the recurrence one token at a time
+                     from a given state: one step, a chain of drafted tokens, and a tree of drafted
+                     tokens where each node continues from its parent's state (Ferrite project page,
+                     Design section 04, drafts verified as best-first trees); ``tree_path`` lists the
+                     nodes from the root to a node.
+* ``states_at``   -- the recurrence with the state captured at cut points (Design section 07).
+* ``l2norm``      -- the L2 normalisation the method's q and k carry.
 
 The recurrence (published gated delta rule, Yang, Kautz and Hatamizadeh, "Gated Delta Networks"):
 ``S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T``, ``o_t = S_t q_t / sqrt(dk)``.
@@ -197,6 +204,43 @@ def decode_verify(q, k, v, g, beta, state):
         out[:, t] = o
         states[:, t] = S
     return out, states
+
+
+def decode_verify_tree(q, k, v, g, beta, parents, state):
+    """Tk drafted tokens per sequence arranged as a tree (Ferrite project page, Design section 04:
+    drafts are verified as best-first trees in one pass of the model).  Node t of sequence b follows
+    node ``parents[b, t]`` (an earlier node, < t) or, when that is -1, the committed ``state`` (not
+    modified): its state is the decode step of its token applied to its parent's state.  Inputs as
+    ``decode_verify`` plus ``parents`` int ``[B, Tk]``.  Returns ``(out [B, Tk, H, dv], states
+    [B, Tk, H, dv, dk])``; a chain (parents[b, t] = t - 1) gives exactly ``decode_verify``."""
+    q, k, v, g, beta = (_d(x) for x in (q, k, v, g, beta))
+    par = np.asarray(parents, dtype=np.int64)
+    B, Tk, H, dk = q.shape
+    dv = v.shape[3]
+    if par.shape != (B, Tk):
+        raise ValueError("parents must be [B, Tk]")
+    s0 = _d(state)
+    out = np.zeros((B, Tk, H, dv))
+    states = np.zeros((B, Tk, H, dv, dk))
+    for b in range(B):
+        for t in range(Tk):
+            p = int(par[b, t])
+            if not -1 <= p < t:
+                raise ValueError("node %d of sequence %d has parent %d: it must be -1 or an earlier node" % (t, b, p))
+            before = s0[b:b + 1] if p < 0 else states[b:b + 1, p]
+            o, S = decode_step(q[b:b + 1, t], k[b:b + 1, t], v[b:b + 1, t], g[b:b + 1, t], beta[b:b + 1, t], before)
+            out[b, t] = o[0]
+            states[b, t] = S[0]
+    return out, states
+
+
+def tree_path(parents_row, t):
+    """The nodes from the root down to node t (inclusive) of one sequence's tree, in order."""
+    path = []
+    while t >= 0:
+        path.append(int(t))
+        t = int(parents_row[t])
+    return path[::-1]
 
 
 def brute_force(q, k, v, g, beta, state_in=None):

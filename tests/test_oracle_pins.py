@@ -340,6 +340,92 @@ def test_decode_verify_equals_one_sequence_per_draft_chain():
     assert rel(st[:, -1], s2) < 1e-13
 
 
+# a best-first draft tree of 8 nodes per sequence: a main chain with side branches, and a root
+# sibling (parent -1); every parent precedes its child
+TREE8 = [[-1, 0, 1, 1, 3, 0, -1, 6],
+         [-1, 0, 0, 2, 2, 4, 1, 6]]
+
+
+def _tree_inputs(B, Tk, H, d, seed):
+    q, k, v, g, b, _ = rnd(B * Tk, H, d, d, seed)
+    s0 = 0.05 * np.random.default_rng(seed + 1).standard_normal((B, H, d, d))
+    return tuple(x.reshape((B, Tk) + x.shape[1:]) for x in (q, k, v, g, b)) + (s0,)
+
+
+def test_decode_verify_tree_nodes_match_brute_force_along_their_path():
+    """Every node's state and output equal the explicit-matrix expansion over the tokens on the path
+    from the root to that node, starting from the committed state (left untouched)."""
+    B, Tk, H, d = 2, 8, 2, 6
+    q, k, v, g, b, s0 = _tree_inputs(B, Tk, H, d, 41)
+    keep = s0.copy()
+    o, st = oracle.decode_verify_tree(q, k, v, g, b, TREE8, s0)
+    assert np.array_equal(s0, keep)
+    for i in range(B):
+        for t in range(Tk):
+            path = oracle.tree_path(TREE8[i], t)
+            assert len(path) <= 8 and path[-1] == t
+            ob, sb = oracle.brute_force(q[i, path], k[i, path], v[i, path], g[i, path], b[i, path],
+                                        state_in=s0[i][None])
+            assert rel(st[i, t], sb[0]) < 1e-12
+            assert rel(o[i, t], ob[-1]) < 1e-12
+
+
+def test_decode_verify_tree_nodes_equal_the_recurrence_on_their_path():
+    """Deeper random trees (up to 24 nodes): each node = the plain recurrence over its root path."""
+    B, Tk, H, d = 3, 24, 2, 8
+    q, k, v, g, b, s0 = _tree_inputs(B, Tk, H, d, 43)
+    r = np.random.default_rng(44)
+    par = np.array([[-1] + [int(r.integers(-1, t)) for t in range(1, Tk)] for _ in range(B)])
+    o, st = oracle.decode_verify_tree(q, k, v, g, b, par, s0)
+    for i in range(B):
+        for t in range(Tk):
+            path = oracle.tree_path(par[i], t)
+            o2, s2 = oracle.recurrence(q[i, path], k[i, path], v[i, path], g[i, path], b[i, path],
+                                       state_in=s0[i][None])
+            assert rel(st[i, t], s2[0]) < 1e-13
+            assert rel(o[i, t], o2[-1]) < 1e-13
+
+
+def test_decode_verify_tree_special_shapes():
+    """A chain tree is the linear verify; a star (every node on the committed state) is Tk
+    independent single steps from that state."""
+    B, Tk, H, d = 2, 5, 2, 8
+    q, k, v, g, b, s0 = _tree_inputs(B, Tk, H, d, 45)
+    chain = [[t - 1 for t in range(Tk)]] * B
+    o1, s1 = oracle.decode_verify_tree(q, k, v, g, b, chain, s0)
+    o2, s2 = oracle.decode_verify(q, k, v, g, b, s0)
+    assert np.array_equal(o1, o2) and np.array_equal(s1, s2)
+    star = [[-1] * Tk] * B
+    o3, s3 = oracle.decode_verify_tree(q, k, v, g, b, star, s0)
+    for t in range(Tk):
+        o4, s4 = oracle.decode_step(q[:, t], k[:, t], v[:, t], g[:, t], b[:, t], s0)
+        assert rel(o3[:, t], o4) < 1e-14 and rel(s3[:, t], s4) < 1e-14
+
+
+def test_decode_verify_tree_rejects_forward_or_out_of_range_parents():
+    B, Tk, H, d = 1, 4, 1, 4
+    q, k, v, g, b, s0 = _tree_inputs(B, Tk, H, d, 47)
+    for bad in ([[-1, 0, 2, 1]], [[-1, 0, -2, 1]], [[0, 0, 1, 2]]):
+        with pytest.raises(ValueError):
+            oracle.decode_verify_tree(q, k, v, g, b, bad, s0)
+
+
+def test_tree_planted_mistake_is_caught():
+    """A verify that ignores the tree and continues from the previous node (a chain) must fail the
+    path pin on a tree that branches."""
+    B, Tk, H, d = 2, 8, 2, 6
+    q, k, v, g, b, s0 = _tree_inputs(B, Tk, H, d, 49)
+    o_wrong, s_wrong = oracle.decode_verify(q, k, v, g, b, s0)       # the mistake: previous node
+    bad = 0
+    for i in range(B):
+        for t in range(Tk):
+            path = oracle.tree_path(TREE8[i], t)
+            o2, s2 = oracle.recurrence(q[i, path], k[i, path], v[i, path], g[i, path], b[i, path],
+                                       state_in=s0[i][None])
+            bad += rel(s_wrong[i, t], s2[0]) > 1e-6
+    assert bad > 0
+
+
 # ---------------------------------------------------------------------------------------------
 # planted mistakes: each variant below is one plausible error; at least one pin must reject it
 # ---------------------------------------------------------------------------------------------
