@@ -307,7 +307,8 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     from linear_attention_10_b200 import gdn
-    from linear_attention_10_b200.workloads import WORKLOADS, make_decode_inputs, make_verify_inputs, workload_inputs
+    from linear_attention_10_b200.workloads import (WORKLOADS, best_first_parents, make_decode_inputs,
+                                                    make_verify_inputs, workload_inputs)
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -560,6 +561,42 @@ def run_ours(args, rank, world, local_rank):
                                     traffic=TRAFFIC.get(name)))
         del vd, vst, vout
 
+    # ---- tree verify: B=64 sequences x 8 drafted tokens in a best-first tree ----
+    verify_tree = None
+    if not args.no_verify:
+        w = WORKLOADS["verify_tree_b64_k8"]
+        B_, Tk, H_, d_ = w.decode_batch, w.decode_steps, w.H, w.dk
+        vd = make_verify_inputs(B_, H_, d_, d_, Tk, dtype=w.dtype, gate=w.gate, seed=w.seed + rank,
+                                state_std=w.state_std, device=dev)
+        tree = best_first_parents(Tk)
+        par = torch.tensor([tree] * B_, dtype=torch.int32, device=dev)
+        vst = torch.empty((B_, Tk, H_, d_, d_), dtype=torch.float32, device=dev)
+        vout = torch.empty((B_, Tk, H_, d_), dtype=torch.bfloat16, device=dev)
+        run_t = lambda: gdn.gdn_decode_verify_tree(vd["q"], vd["k"], vd["v"], vd["g"], vd["beta"], par, vd["state"],
+                                                   states_out=vst, out=vout)
+        for _ in range(3):
+            run_t()
+        reps = 50
+        tms, tprof = timed_passes(lambda i: run_t(), reps, world, dev, stream)
+        name = "gdn_decode_verify_kernel"
+        kms, kl = tprof.get(name, (tms, reps))
+        per_bh = (1 + Tk) * d_ * d_ * 4 + Tk * ((3 * d_) * 2 + 2 * 4 + d_ * 2)   # API bytes, as for the chain
+        rereads = sum(1 for t in range(Tk) if tree[t] != t - 1 and tree[t] >= 0)
+        bytes_per_launch = B_ * H_ * per_bh
+        ach = bytes_per_launch / (kms / kl / 1e3) / 1e9
+        pk, pu, pdesc = peak_for("hbm", peaks)
+        verify_tree = dict(workload="verify_tree_b64_k8: B=64 sequences x 8 drafted tokens in the best-first tree "
+                                    "%s (parent of each token, -1 = committed state), decode_b64 distributions"
+                                    % tree,
+                           value=job_throughput(B_ * Tk, reps, world, tms), unit="tokens/s",
+                           us_per_call=tms / reps * 1e3,
+                           roofline=dict(kernel=name, bound="hbm", achieved=ach, peak=pk, unit=pu, frac=ach / pk,
+                                         peak_source=pdesc, bytes_per_launch=bytes_per_launch,
+                                         note="API bytes only; %d tokens re-read their parent's state "
+                                              "(%d x 64 KB per sequence-head more)" % (rereads, rereads),
+                                         traffic=None))
+        del vd, vst, vout, par
+
     clk = clocks.stop()
 
     # ---- roofline of the dominant prefill kernel ----
@@ -615,7 +652,7 @@ def run_ours(args, rank, world, local_rank):
                          ms_per_step=e2e_ms / e2e_steps,
                          pipelining="copy-in, compute and copy-out on three streams, double-buffered",
                          steps=e2e_steps),
-                gpu_launches=launches, clocks=clk, decode=decode, verify=verify,
+                gpu_launches=launches, clocks=clk, decode=decode, verify=verify, verify_tree=verify_tree,
                 cuts=cuts_line, norm=norm_line)
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -69,7 +69,9 @@ enum {
     GDN_ERR_BAD_SEQLENS = -6,  /* device-detected: cu_seqlens not 0..T_total non-decreasing, or
                                   cut points not increasing and strictly inside a sequence      */
     GDN_ERR_TIMEOUT = -7,      /* device-detected: a bounded wait inside a kernel expired        */
-    GDN_ERR_CUDA = -8          /* a CUDA runtime call made by the library failed                */
+    GDN_ERR_CUDA = -8,         /* a CUDA runtime call made by the library failed                */
+    GDN_ERR_BAD_PARENTS = -9   /* device-detected: a draft-tree parent index is not -1 or an
+                                  earlier node of the same sequence                              */
 };
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -207,8 +209,29 @@ int gdn_decode_verify(const void* q, const void* k, const void* v, const float* 
                       int Tk, int H, int dk, int dv, int dtype, void* stream);
 
 /*
+ * Tree verify (Ferrite project page, Design section 04: drafted tokens are verified as best-first
+ * trees in one pass of the model).  As gdn_decode_verify, but the Tk drafted tokens of a sequence
+ * form a tree: token t continues from the state after token parents[b * Tk + t], which must be an
+ * earlier token (< t), or from the committed state when the parent is -1.  A linear chain
+ * (parents[b * Tk + t] = t - 1) gives exactly gdn_decode_verify.
+ *
+ *   parents       device int32 [B, Tk], 4-byte aligned
+ *   states_out    device fp32 [B, Tk, H, dv, dk]: S after token t at [b, t] -- required (the tree
+ *                 reads a parent's state back from it)
+ *   out           device [B, Tk, H, dv] in dtype `dtype`, or NULL
+ *   Other arguments and errors as gdn_decode_verify; GDN_ERR_INVALID_ARG also for parents or
+ *   states_out NULL.  A parent that is neither -1 nor an earlier token is device-detected: the
+ *   token starts from the committed state and gdn_get_device_status reports GDN_ERR_BAD_PARENTS.
+ */
+int gdn_decode_verify_tree(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, const int32_t* parents, const float* state_in,
+                           float* states_out, void* out, int B, int Tk, int H, int dk, int dv, int dtype,
+                           void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of the current device:
- * GDN_OK, or the first device-detected error (GDN_ERR_BAD_SEQLENS, GDN_ERR_TIMEOUT) recorded since
+ * GDN_OK, or the first device-detected error (GDN_ERR_BAD_SEQLENS, GDN_ERR_TIMEOUT,
+ * GDN_ERR_BAD_PARENTS) recorded since
  * the last read.  Returns GDN_ERR_CUDA when the synchronisation itself fails.
  */
 int gdn_get_device_status(void* stream);

@@ -132,30 +132,36 @@ static int dispatch_decode(const void* q, const void* k, const void* v, const fl
 
 template <typename T, int DK, int DV>
 static int launch_verify(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                         const float* state_in, float* states_out, void* out, int B, int Tk, int H, bool norm,
-                         cudaStream_t st)
+                         const float* state_in, float* states_out, void* out, const int32_t* parents, int B,
+                         int Tk, int H, bool norm, cudaStream_t st)
 {
+    int* status = status_ptr();
+    if (!status) return GDN_ERR_CUDA;
     ProfScope prof("gdn_decode_verify_kernel", st);
-    auto kern = norm ? gdn_decode_verify_kernel<T, DK, DV, true> : gdn_decode_verify_kernel<T, DK, DV, false>;
+    auto kern = parents ? (norm ? gdn_decode_verify_kernel<T, DK, DV, true, true>
+                                : gdn_decode_verify_kernel<T, DK, DV, false, true>)
+                        : (norm ? gdn_decode_verify_kernel<T, DK, DV, true, false>
+                                : gdn_decode_verify_kernel<T, DK, DV, false, false>);
     constexpr int RB = (GDN_DECODE_RB < DV) ? GDN_DECODE_RB : DV;
     kern<<<(unsigned)B * H * (DV / RB), 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
-                                          g, beta, state_in, states_out, static_cast<T*>(out), H, Tk);
+                                          g, beta, state_in, states_out, static_cast<T*>(out), parents, status,
+                                          H, Tk);
     return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
 }
 
 template <typename T>
 static int dispatch_verify(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                           const float* state_in, float* states_out, void* out, int B, int Tk, int H, int dk, int dv,
-                           bool norm, cudaStream_t st)
+                           const float* state_in, float* states_out, void* out, const int32_t* parents, int B,
+                           int Tk, int H, int dk, int dv, bool norm, cudaStream_t st)
 {
 #define GDN_VF(DK_, DV_)                                                                                   \
     if (dk == DK_ && dv == DV_)                                                                            \
-        return launch_verify<T, DK_, DV_>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, norm, st);
+        return launch_verify<T, DK_, DV_>(q, k, v, g, beta, state_in, states_out, out, parents, B, Tk, H, norm, st);
     GDN_VF(128, 128)
     GDN_VF(128, 64)
     GDN_VF(64, 128)
 #undef GDN_VF
-    return launch_verify<T, 64, 64>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, norm, st);
+    return launch_verify<T, 64, 64>(q, k, v, g, beta, state_in, states_out, out, parents, B, Tk, H, norm, st);
 }
 
 // ---- tensor maps (2-D tiled views of q/k/v) -------------------------------------------------------
@@ -457,6 +463,7 @@ const char* gdn_status_string(int s)
     case GDN_ERR_BAD_SEQLENS: return "GDN_ERR_BAD_SEQLENS: cu_seqlens is not 0..T_total non-decreasing";
     case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT: a bounded wait inside a kernel expired";
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA: a CUDA runtime call failed";
+    case GDN_ERR_BAD_PARENTS: return "GDN_ERR_BAD_PARENTS: a draft-tree parent is not -1 or an earlier token";
     default: return "unknown gdn status";
     }
 }
@@ -535,9 +542,10 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
     return dispatch_decode<__nv_bfloat16>(q, k, v, g, beta, state_inout, out, B, H, dk, dv, norm, st);
 }
 
-int gdn_decode_verify(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                      const float* state_in, float* states_out, void* out, int B, int Tk, int H, int dk, int dv,
-                      int dtype, void* stream)
+// Checks and dispatch shared by the chain and tree verify (parents == nullptr: a chain).
+static int verify_entry(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                        const int32_t* parents, const float* state_in, float* states_out, void* out, int B, int Tk,
+                        int H, int dk, int dv, int dtype, void* stream)
 {
     if (B < 0 || Tk < 1 || H < 1) return GDN_ERR_INVALID_ARG;
     bool norm = false;
@@ -550,11 +558,29 @@ int gdn_decode_verify(const void* q, const void* k, const void* v, const float* 
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
     if (!aligned4(g) || !aligned4(beta)) return GDN_ERR_MISALIGNED;
+    if (parents && !aligned4(parents)) return GDN_ERR_MISALIGNED;
     if ((int64_t)B * H > INT32_MAX || (int64_t)B * Tk * H > INT32_MAX) return GDN_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dtype == GDN_F32)
-        return dispatch_verify<float>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, dk, dv, norm, st);
-    return dispatch_verify<__nv_bfloat16>(q, k, v, g, beta, state_in, states_out, out, B, Tk, H, dk, dv, norm, st);
+        return dispatch_verify<float>(q, k, v, g, beta, state_in, states_out, out, parents, B, Tk, H, dk, dv, norm,
+                                      st);
+    return dispatch_verify<__nv_bfloat16>(q, k, v, g, beta, state_in, states_out, out, parents, B, Tk, H, dk, dv,
+                                          norm, st);
+}
+
+int gdn_decode_verify(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                      const float* state_in, float* states_out, void* out, int B, int Tk, int H, int dk, int dv,
+                      int dtype, void* stream)
+{
+    return verify_entry(q, k, v, g, beta, nullptr, state_in, states_out, out, B, Tk, H, dk, dv, dtype, stream);
+}
+
+int gdn_decode_verify_tree(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                           const int32_t* parents, const float* state_in, float* states_out, void* out, int B,
+                           int Tk, int H, int dk, int dv, int dtype, void* stream)
+{
+    if (B > 0 && (!parents || !states_out)) return GDN_ERR_INVALID_ARG;
+    return verify_entry(q, k, v, g, beta, parents, state_in, states_out, out, B, Tk, H, dk, dv, dtype, stream);
 }
 
 int gdn_get_device_status(void* stream)

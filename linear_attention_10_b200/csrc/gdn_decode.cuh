@@ -124,20 +124,23 @@ __global__ void __launch_bounds__(GDN_DECODE_NT) gdn_decode_step_kernel(const T*
     }
 }
 
-// Multi-token recurrent verify: Tk draft tokens of one sequence run through the recurrence in order
-// (a linear chain of speculative tokens, Ferrite project page, Design section 04), starting from the
-// committed state, which is only read.  The state after every token is written to states_out, so
-// that the caller keeps the one after the last accepted token and drops the rest.
+// Multi-token recurrent verify: Tk draft tokens of one sequence run through the recurrence, starting
+// from the committed state, which is only read (Ferrite project page, Design section 04: drafts are
+// verified in one pass, as best-first trees).  Without TREE the tokens form a linear chain; with
+// TREE token t continues from the state after token parents[b, t] (< t), or from the committed state
+// when that is -1.  (The chain is its own instantiation, so its code is not burdened by the tree's.)  The state after every token is written to states_out, so that
+// the caller keeps the one after the last accepted token and drops the rest.
 //
 // Mapping: one CTA (8 warps) per block of GDN_DECODE_RB rows of one (b, h) state; the block lives in
 // registers for the Tk tokens (each lane holds NR float4s of its rows), is read from HBM once and
 // written Tk times.
-template <typename T, int DK, int DV, bool NORM>
+template <typename T, int DK, int DV, bool NORM, bool TREE>
 __global__ void __launch_bounds__(256) gdn_decode_verify_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                             const T* __restrict__ v, const float* __restrict__ g,
                                                             const float* __restrict__ beta,
                                                             const float* __restrict__ state_in,
                                                             float* __restrict__ states_out, T* __restrict__ out,
+                                                            const int32_t* __restrict__ parents, int* status,
                                                             int H, int Tk)
 {
     constexpr int LPR = DK / 4;               // lanes per row
@@ -163,6 +166,28 @@ __global__ void __launch_bounds__(256) gdn_decode_verify_kernel(const T* __restr
 
     for (int t = 0; t < Tk; ++t) {
         const size_t tok = ((size_t)b * Tk + t) * H + h;      // index into [B, Tk, H]
+        if constexpr (TREE) {
+            int p = __ldg(parents + (size_t)b * Tk + t);
+            if (p < -1 || p >= t) {
+                // not -1 or an earlier node: reported, and the node starts from the committed state
+                if (threadIdx.x == 0) report(status, GDN_ERR_BAD_PARENTS);
+                p = -1;
+            }
+            if (p != t - 1) {
+                // the parent's state: the committed one, or the rows this thread wrote for node p
+                // (read back through L2, never the read-only path: this kernel wrote them)
+                if (p < 0) {
+#pragma unroll
+                    for (int u = 0; u < NR; ++u)
+                        s[u] = *reinterpret_cast<const float4*>(S0 + (size_t)(row0 + u * RPW) * DK + col);
+                } else {
+                    const float* Sp = states_out + (((size_t)b * Tk + p) * H + h) * DV * DK;
+#pragma unroll
+                    for (int u = 0; u < NR; ++u)
+                        s[u] = __ldcg(reinterpret_cast<const float4*>(Sp + (size_t)(row0 + u * RPW) * DK + col));
+                }
+            }
+        }
         float4 k4 = Elem<T>::ld4(k + tok * DK + col);
         float4 q4 = Elem<T>::ld4(q + tok * DK + col);
         if constexpr (NORM) {

@@ -31,6 +31,7 @@ EXPORTS = (
     "gdn_chunk_prefill_noalloc",
     "gdn_decode_step",
     "gdn_decode_verify",
+    "gdn_decode_verify_tree",
     "gdn_get_device_status",
     "gdn_profile_start",
     "gdn_profile_stop",
@@ -75,6 +76,8 @@ def lib() -> ctypes.CDLL:
     L.gdn_decode_step.restype = i32
     L.gdn_decode_verify.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
     L.gdn_decode_verify.restype = i32
+    L.gdn_decode_verify_tree.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
+    L.gdn_decode_verify_tree.restype = i32
     L.gdn_get_device_status.argtypes = [vp]
     L.gdn_get_device_status.restype = i32
     L.gdn_profile_start.argtypes = []
@@ -268,6 +271,37 @@ def gdn_decode_verify(q, k, v, g, beta, state_in, states_out=None, out=None, wan
                                  _stream_ptr(stream))
     if rc != 0:
         raise GdnError(rc, "gdn_decode_verify")
+    return out, states_out
+
+
+def gdn_decode_verify_tree(q, k, v, g, beta, parents, state_in, states_out=None, out=None, stream=None,
+                           normalize_qk=False):
+    """Tk drafted tokens per sequence verified as a tree: token t continues from the state after token
+    ``parents[b, t]`` (an earlier token) or from state_in when that is -1.  Shapes as
+    ``gdn_decode_verify`` plus parents int32 ``[B, Tk]`` on the device.  Returns ``(out [B, Tk, H,
+    dv], states_out [B, Tk, H, dv, dk])``; a parent that is not -1 or an earlier token is reported by
+    ``gdn_get_device_status`` as GDN_ERR_BAD_PARENTS."""
+    B, Tk, H, dk = q.shape
+    dv = v.shape[3]
+    dev, dt = q.device, q.dtype
+    _check(q, "q", (B, Tk, H, dk), dt, dev)
+    _check(k, "k", (B, Tk, H, dk), dt, dev)
+    _check(v, "v", (B, Tk, H, dv), dt, dev)
+    _check(g, "g", (B, Tk, H), torch.float32, dev)
+    _check(beta, "beta", (B, Tk, H), torch.float32, dev)
+    _check(parents, "parents", (B, Tk), torch.int32, dev)
+    _check(state_in, "state_in", (B, H, dv, dk), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, Tk, H, dv), dtype=dt, device=dev)
+    _check(out, "out", (B, Tk, H, dv), dt, dev)
+    if states_out is None:
+        states_out = torch.empty((B, Tk, H, dv, dk), dtype=torch.float32, device=dev)
+    _check(states_out, "states_out", (B, Tk, H, dv, dk), torch.float32, dev)
+    rc = lib().gdn_decode_verify_tree(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(parents),
+                                      _ptr(state_in), _ptr(states_out), _ptr(out), B, Tk, H, dk, dv,
+                                      _dtype_code(q) | (GDN_QK_L2NORM if normalize_qk else 0), _stream_ptr(stream))
+    if rc != 0:
+        raise GdnError(rc, "gdn_decode_verify_tree")
     return out, states_out
 
 

@@ -59,7 +59,27 @@ WORKLOADS = {
     # speculative verify: 4 drafted tokens for each of 64 sequences, the decode_b64 distributions
     "verify_b64_k4": Workload("verify_b64_k4", [], dtype="bf16", gate="uniform", state_std=0.05,
                               decode_batch=64, decode_steps=4),
+    # tree verify: 8 drafted tokens per sequence in the best-first tree of best_first_parents(8)
+    "verify_tree_b64_k8": Workload("verify_tree_b64_k8", [], dtype="bf16", gate="uniform", state_std=0.05,
+                                   decode_batch=64, decode_steps=8),
 }
+
+
+def best_first_parents(Tk):
+    """Parent of each of Tk drafted tokens in a best-first draft tree: a main chain through the first
+    half of the tokens, the rest branching off main-chain tokens (token t under main token
+    (7 t) mod (Tk / 2)), and the last token a second child of the committed state (-1) when Tk > 2.
+    Every parent precedes its child."""
+    main = max(1, Tk // 2)
+    row = []
+    for t in range(Tk):
+        if t == 0 or (t == Tk - 1 and Tk > 2):
+            row.append(-1)
+        elif t < main:
+            row.append(t - 1)
+        else:
+            row.append((7 * t) % main)
+    return row
 
 
 def _torch_dtype(name: str) -> torch.dtype:

@@ -129,6 +129,31 @@ def test_verify_rejects_bad_arguments(L):
     assert verify(L, B=0) == 0                          # nothing to do, nothing enqueued
 
 
+def verify_tree(L, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, par=FAKE, s=FAKE, st=FAKE, out=FAKE, B=4, Tk=3, H=2,
+             dk=128, dv=128, dtype=1, stream=None)
+    a.update(kw)
+    return L.gdn_decode_verify_tree(a["q"], a["k"], a["v"], a["g"], a["beta"], a["par"], a["s"], a["st"], a["out"],
+                                    a["B"], a["Tk"], a["H"], a["dk"], a["dv"], a["dtype"], a["stream"])
+
+
+def test_verify_tree_rejects_bad_arguments(L):
+    """Every case returns before any launch (the pointers are not real device memory)."""
+    assert verify_tree(L, par=None) == -1
+    assert verify_tree(L, st=None) == -1                # the tree reads parents' states back from it
+    assert verify_tree(L, s=None) == -1
+    assert verify_tree(L, Tk=0) == -1
+    assert verify_tree(L, dtype=3) == -1
+    assert verify_tree(L, dv=96) == -2
+    assert verify_tree(L, par=FAKE + 2) == -3
+    assert verify_tree(L, st=FAKE + 4) == -3
+    assert verify_tree(L, B=0) == 0                     # nothing to do, nothing enqueued
+
+
+def test_status_string_names_bad_parents(L):
+    assert b"BAD_PARENTS" in L.gdn_status_string(-9)
+
+
 def prefill_cuts(L, **kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu=FAKE, N=2, T=64, cuts=FAKE, nc=2, s_in=None, out=FAKE,
              s_out=FAKE, snaps=FAKE, H=2, dk=128, dv=128, dtype=1, ws=FAKE, ws_bytes=1 << 30, stream=None)
