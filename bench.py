@@ -75,6 +75,7 @@ TRAFFIC = {
     "gdn_l2norm_kernel": 67.12e6 + 21.02e6,
     "gdn_decode_step_kernel": 135.83e6 + 77.84e6,
     "gdn_decode_verify_kernel": 140.59e6 + 479.75e6,
+    "gdn_decode_verify_kernel (tree, verify_tree_b64_k8)": 147.02e6 + 1019.77e6,
 }
 
 
@@ -594,7 +595,7 @@ def run_ours(args, rank, world, local_rank):
                                          peak_source=pdesc, bytes_per_launch=bytes_per_launch,
                                          note="API bytes only; %d tokens re-read their parent's state "
                                               "(%d x 64 KB per sequence-head more)" % (rereads, rereads),
-                                         traffic=None))
+                                         traffic=TRAFFIC.get("gdn_decode_verify_kernel (tree, verify_tree_b64_k8)")))
         del vd, vst, vout, par
 
     clk = clocks.stop()
