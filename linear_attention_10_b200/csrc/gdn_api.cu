@@ -115,9 +115,11 @@ static int launch_decode(const void* q, const void* k, const void* v, const floa
     ProfScope prof("gdn_decode_step_kernel", st);
     auto kern = norm ? gdn_decode_step_kernel<T, DK, DV, true> : gdn_decode_step_kernel<T, DK, DV, false>;
     constexpr int RB = (GDN_DECODE_RB < DV) ? GDN_DECODE_RB : DV;
-    kern<<<(unsigned)B * H * (DV / RB), GDN_DECODE_NT, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
-                                          g, beta, state, static_cast<T*>(out), H);
-    return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
+    if (launch_dependent(kern, dim3((unsigned)B * H * (DV / RB)), dim3(GDN_DECODE_NT), 0, st, static_cast<const T*>(q),
+                         static_cast<const T*>(k), static_cast<const T*>(v), g, beta, state, static_cast<T*>(out),
+                         H) != cudaSuccess)
+        return GDN_ERR_LAUNCH;
+    return GDN_OK;
 }
 
 template <typename T>
@@ -143,10 +145,11 @@ static int launch_verify(const void* q, const void* k, const void* v, const floa
                         : (norm ? gdn_decode_verify_kernel<T, DK, DV, true, false>
                                 : gdn_decode_verify_kernel<T, DK, DV, false, false>);
     constexpr int RB = (GDN_DECODE_RB < DV) ? GDN_DECODE_RB : DV;
-    kern<<<(unsigned)B * H * (DV / RB), 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
-                                          g, beta, state_in, states_out, static_cast<T*>(out), parents, status,
-                                          H, Tk);
-    return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
+    if (launch_dependent(kern, dim3((unsigned)B * H * (DV / RB)), dim3(256), 0, st, static_cast<const T*>(q),
+                         static_cast<const T*>(k), static_cast<const T*>(v), g, beta, state_in, states_out,
+                         static_cast<T*>(out), parents, status, H, Tk) != cudaSuccess)
+        return GDN_ERR_LAUNCH;
+    return GDN_OK;
 }
 
 template <typename T>

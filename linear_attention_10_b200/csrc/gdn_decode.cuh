@@ -19,6 +19,7 @@
 
 #include "gdn_common.cuh"
 #include "gdn_norm.cuh"
+#include "gdn_sm100.cuh"
 
 namespace gdn {
 
@@ -81,6 +82,11 @@ __global__ void __launch_bounds__(GDN_DECODE_NT) gdn_decode_step_kernel(const T*
     static_assert(ROWS_PER_WARP % (RPW * UNROLL) == 0 || ROWS_PER_WARP < RPW * UNROLL, "row split");
     constexpr int STEP = (ROWS_PER_WARP < RPW * UNROLL) ? ROWS_PER_WARP : RPW * UNROLL;
     constexpr int U = STEP / RPW;             // row groups per iteration
+
+    // launched as a programmatic dependent: the previous kernel in the stream (typically the last
+    // decode step, which wrote this state) has completed before anything is read here
+    sm100::grid_dep_wait();
+    sm100::grid_dep_launch();
 
     const int bh = blockIdx.x / (DV / RB);    // b * H + h
     const int rblk = blockIdx.x % (DV / RB);
@@ -149,6 +155,10 @@ __global__ void __launch_bounds__(256) gdn_decode_verify_kernel(const T* __restr
     constexpr int ROWS_PER_WARP = RB / 8;
     constexpr int NR = ROWS_PER_WARP / RPW;   // rows held by one lane
     static_assert(ROWS_PER_WARP >= RPW && ROWS_PER_WARP % RPW == 0, "row split");
+
+    // launched as a programmatic dependent, as the decode step is
+    sm100::grid_dep_wait();
+    sm100::grid_dep_launch();
 
     const int bh = blockIdx.x / (DV / RB);    // b * H + h
     const int rblk = blockIdx.x % (DV / RB);
