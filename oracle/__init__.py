@@ -19,6 +19,9 @@ What is computed and why (each function cites its source):
                      Design section 04, drafts verified as best-first trees); ``tree_path`` lists the
                      nodes from the root to a node.
 * ``states_at``   -- the recurrence with the state captured at cut points (Design section 07).
+* ``chunk_operator``, ``chunk_step`` -- one chunk's state-independent WY/UT quantities (the decay
+                     matrix, A, T = (I + A)^-1, T'' = T diag(beta), P, P T'', the cross-chunk Gram G'
+                     and the gates) and the chunk step built from them, for checks of one stage.
 * ``l2norm``      -- the L2 normalisation the method's q and k carry.
 
 The recurrence (published gated delta rule, Yang, Kautz and Hatamizadeh, "Gated Delta Networks"):
@@ -187,6 +190,61 @@ def states_at(q, k, v, g, beta, cuts, cu_seqlens=None, state_in=None):
                 snaps[inner[j][0]] = s[0]
         st[n] = s[0]
     return out, st, snaps
+
+
+def chunk_operator(q, k, g, beta, k_prev=None, chunk=32):
+    """The state-independent quantities of one chunk of one head in the chunkwise WY/UT form (Ferrite
+    project page, Design section 03: chunks of 32 rows, WY/UT form), in fp64.  Inputs: q, k
+    ``[L, dk]``, g, beta ``[L]`` with L <= chunk rows (the rest of the chunk is padding: g = 0,
+    beta = 0, q = k = 0), k_prev ``[chunk, dk]`` the previous chunk's keys or None.  With gamma_i the
+    chunk-local cumulative sum of g and D_ij = exp(gamma_i - gamma_j):
+
+      A = strictly-lower(diag(beta) (D o K K^T)),  T = (I + A)^-1,  T'' = T diag(beta),
+      P = lower-incl-diagonal(D o Q K^T),          G' = [K; Q] K_prev^T,
+      Gamma_i = exp(gamma_i),  delta_i = exp(gamma_C - gamma_i),  Gamma_C = exp(gamma_C).
+
+    Returns a dict of numpy arrays: A, T, Tpp (T''), P, PTpp (P T''), Gp (G', zeros without k_prev),
+    Gamma, delta, GammaC."""
+    q, k = _d(q), _d(k)
+    g, beta = _d(g).reshape(-1), _d(beta).reshape(-1)
+    L, dk = k.shape
+    if L > chunk:
+        raise ValueError("at most %d rows" % chunk)
+    Q = np.zeros((chunk, dk))
+    K = np.zeros((chunk, dk))
+    G = np.zeros(chunk)
+    Bt = np.zeros(chunk)
+    Q[:L], K[:L], G[:L], Bt[:L] = q, k, g, beta
+    gam = np.cumsum(G)
+    D = np.exp(gam[:, None] - gam[None, :])
+    i, j = np.indices((chunk, chunk))
+    A = np.where(j < i, Bt[:, None] * D * (K @ K.T), 0.0)
+    T = np.linalg.inv(np.eye(chunk) + A)
+    Tpp = T * Bt[None, :]
+    P = np.where(j <= i, D * (Q @ K.T), 0.0)
+    KQ = np.concatenate([K, Q], axis=0)
+    Gp = np.zeros((2 * chunk, chunk)) if k_prev is None else KQ @ _d(k_prev).T
+    return dict(A=A, T=T, Tpp=Tpp, P=P, PTpp=P @ Tpp, Gp=Gp, Gamma=np.exp(gam), delta=np.exp(gam[-1] - gam),
+                GammaC=float(np.exp(gam[-1])))
+
+
+def chunk_step(op, q, k, v, state, chunk=32):
+    """One chunk of one head from the quantities of ``chunk_operator``: with X = K S0^T, Z = Q S0^T,
+    U = T'' (V - diag(Gamma) X), the outputs O = s (diag(Gamma) Z + P U) and the state after the
+    chunk S1 = Gamma_C S0 + (diag(delta) U)^T K.  Inputs q, k ``[L, dk]``, v ``[L, dv]``, state
+    ``[dv, dk]``; returns (O ``[L, dv]``, S1)."""
+    q, k, v, S0 = _d(q), _d(k), _d(v), _d(state)
+    L, dk = k.shape
+    dv = v.shape[1]
+    Q = np.zeros((chunk, dk))
+    K = np.zeros((chunk, dk))
+    V = np.zeros((chunk, dv))
+    Q[:L], K[:L], V[:L] = q, k, v
+    X, Z = K @ S0.T, Q @ S0.T
+    U = op["Tpp"] @ (V - op["Gamma"][:, None] * X)
+    O = (op["Gamma"][:, None] * Z + op["P"] @ U) / np.sqrt(dk)
+    S1 = op["GammaC"] * S0 + (op["delta"][:, None] * U).T @ K
+    return O[:L], S1
 
 
 def decode_verify(q, k, v, g, beta, state):

@@ -340,6 +340,68 @@ def test_decode_verify_equals_one_sequence_per_draft_chain():
     assert rel(st[:, -1], s2) < 1e-13
 
 
+def _one_head(L, d, seed, gate=(-0.5, 0.0)):
+    q, k, v, g, b, _ = rnd(L, 1, d, d, seed, gate=gate)
+    return q[:, 0], k[:, 0], v[:, 0], g[:, 0], b[:, 0]
+
+
+@pytest.mark.parametrize("L", [1, 5, 31, 32])
+@pytest.mark.parametrize("gate", [(-0.5, 0.0), (-4.0, -1.0)])
+def test_chunk_operator_reconstructs_the_recurrence(L, gate):
+    """One chunk built from the WY/UT quantities (T'', P T'', gates) gives the recurrence's outputs
+    and state, for ragged chunks and strong gates."""
+    d = 16
+    q, k, v, g, b = _one_head(L, d, 60 + L, gate)
+    S0 = 0.05 * np.random.default_rng(61).standard_normal((d, d))
+    op = oracle.chunk_operator(q, k, g, b)
+    O, S1 = oracle.chunk_step(op, q, k, v, S0)
+    o2, s2 = oracle.recurrence(q[:, None], k[:, None], v[:, None], g[:, None], b[:, None], state_in=S0[None, None])
+    assert rel(O, o2[:, 0]) < 1e-12 and rel(S1, s2[0, 0]) < 1e-12
+
+
+def test_cross_chunk_gram_gives_the_lookahead_identity():
+    """[X_c; Z_c] from the exact state equals Gamma_C(c-1) [K;Q]_c S_{c-2}^T + G'_c U~_{c-1}: the
+    identity that lets the state-dependent product of a chunk run one chunk early."""
+    d, C = 16, 32
+    q, k, v, g, b = _one_head(3 * C, d, 63)
+    S = 0.05 * np.random.default_rng(64).standard_normal((d, d))
+    sl = [slice(c * C, (c + 1) * C) for c in range(3)]
+    op0 = oracle.chunk_operator(q[sl[0]], k[sl[0]], g[sl[0]], b[sl[0]])
+    _, S_a = oracle.chunk_step(op0, q[sl[0]], k[sl[0]], v[sl[0]], S)           # S_{c-2}
+    op1 = oracle.chunk_operator(q[sl[1]], k[sl[1]], g[sl[1]], b[sl[1]], k_prev=k[sl[0]])
+    X1 = k[sl[1]] @ S_a.T
+    U1 = op1["Tpp"] @ (v[sl[1]] - op1["Gamma"][:, None] * X1)
+    Ut1 = op1["delta"][:, None] * U1                                           # U~_{c-1}
+    _, S_b = oracle.chunk_step(op1, q[sl[1]], k[sl[1]], v[sl[1]], S_a)         # S_{c-1}
+    op2 = oracle.chunk_operator(q[sl[2]], k[sl[2]], g[sl[2]], b[sl[2]], k_prev=k[sl[1]])
+    KQ = np.concatenate([k[sl[2]], q[sl[2]]])
+    direct = KQ @ S_b.T
+    lookahead = op1["GammaC"] * (KQ @ S_a.T) + op2["Gp"] @ Ut1
+    assert rel(lookahead, direct) < 1e-12
+
+
+def test_chunk_operator_planted_mistake_is_caught():
+    """A that keeps its diagonal (j <= i instead of j < i) must break the reconstruction."""
+    d, L = 16, 20
+    q, k, v, g, b = _one_head(L, d, 65)
+    S0 = 0.05 * np.random.default_rng(66).standard_normal((d, d))
+    op = oracle.chunk_operator(q, k, g, b)
+    C = 32
+    K = np.zeros((C, d))
+    K[:L] = k
+    Bt = np.zeros(C)
+    Bt[:L] = b
+    gam = np.cumsum(np.concatenate([g, np.zeros(C - L)]))
+    D = np.exp(gam[:, None] - gam[None, :])
+    i, j = np.indices((C, C))
+    A_bad = np.where(j <= i, Bt[:, None] * D * (K @ K.T), 0.0)
+    bad = dict(op)
+    bad["Tpp"] = np.linalg.inv(np.eye(C) + A_bad) * Bt[None, :]
+    O, S1 = oracle.chunk_step(bad, q, k, v, S0)
+    o2, s2 = oracle.recurrence(q[:, None], k[:, None], v[:, None], g[:, None], b[:, None], state_in=S0[None, None])
+    assert rel(S1, s2[0, 0]) > 1e-6
+
+
 # a best-first draft tree of 8 nodes per sequence: a main chain with side branches, and a root
 # sibling (parent -1); every parent precedes its child
 TREE8 = [[-1, 0, 1, 1, 3, 0, -1, 6],
