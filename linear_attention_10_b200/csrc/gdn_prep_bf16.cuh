@@ -1,7 +1,9 @@
 // gdn_prep_bf16.cuh -- per-(chunk, head) WY/UT operator for bf16 q/k (sm_100a).
 //
-// Builds the same record as gdn_prep_kernel (gdn_prefill_tc.cuh): the TF32 hi/lo image of
-// [T''; P T''] and the gates of one chunk of 32 rows, where (chunk-local cumulative log-gate gamma)
+// Builds the operator record the bf16 scan reads, for one chunk of 32 rows of one head: [T''; P T'']
+// and the cross-chunk Gram G' = [K; Q] K_prev^T, each as three bf16 parts in the 64-byte-swizzled
+// K-major layout of a tensor-core A operand, and the gates Gamma_i, delta_i, Gamma_C, where
+// (chunk-local cumulative log-gate gamma)
 //
 //   A = strictly-lower(diag(beta) (D o K K^T)),  P = lower-incl-diagonal(D o Q K^T),
 //   D_ij = exp(gamma_i - gamma_j),  T = (I + A)^-1,  T'' = T diag(beta).
