@@ -28,7 +28,12 @@
  *     4-byte aligned (GDN_ERR_MISALIGNED otherwise).
  *   - The caller owns every buffer; the library never allocates device memory in these calls.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  All work is
- *     enqueued on it; no call synchronises the host except gdn_get_device_status.
+ *     enqueued on it; no call synchronises the host except gdn_get_device_status.  Within a call,
+ *     and from one call to the next, kernels are launched as programmatic dependents of the
+ *     kernel before them: each waits on the device for its predecessor to complete before reading
+ *     anything.  A caller kernel launched after a call with the programmatic-serialisation launch
+ *     attribute must likewise wait (griddepcontrol.wait) before reading the call's results; a
+ *     normal launch needs nothing.
  *   - Return value: GDN_OK (0) when the work was enqueued, a negative GDN_ERR_* otherwise (nothing
  *     is enqueued then).  Errors the host cannot see (bad cu_seqlens contents, an expired bounded
  *     wait) are recorded by the kernels in a per-device status word; read it with
