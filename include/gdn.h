@@ -242,6 +242,15 @@ int gdn_decode_verify_tree(const void* q, const void* k, const void* v, const fl
 int gdn_get_device_status(void* stream);
 
 /*
+ * Failure-path self-test (a test aid, not part of the computation): enqueues one kernel whose single
+ * waiting thread waits on a barrier that nothing completes.  The bounded wait gives up after about
+ * limit_ns nanoseconds, records GDN_ERR_TIMEOUT in the status word and the kernel returns normally,
+ * so the next gdn_get_device_status returns GDN_ERR_TIMEOUT and later calls run as usual.
+ *   limit_ns in [1e6, 2e9] (GDN_ERR_INVALID_ARG otherwise).
+ */
+int gdn_selftest_wait_timeout(long long limit_ns, void* stream);
+
+/*
  * Measurement aid (no counterpart on the pages): per-kernel device time of the library's own
  * launches.  After gdn_profile_start, every kernel the library launches (from any host thread) is
  * bracketed by a pair of CUDA events recorded on the launch's stream.  gdn_profile_stop

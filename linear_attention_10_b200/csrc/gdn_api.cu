@@ -586,6 +586,32 @@ int gdn_decode_verify_tree(const void* q, const void* k, const void* v, const fl
     return verify_entry(q, k, v, g, beta, parents, state_in, states_out, out, B, Tk, H, dk, dv, dtype, stream);
 }
 
+// Failure-path self-test: one thread waits on an mbarrier that nothing arrives on.  The bounded
+// wait gives up after about limit_ns, the kernel records GDN_ERR_TIMEOUT in the status word and
+// returns normally (the context stays usable), exactly as a timed-out wait in the prefill does.
+__global__ void gdn_selftest_timeout_kernel(int* status, unsigned long long limit_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int never;
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(&bar, 1);
+        sm100::fence_mbar_init();
+        never = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !sm100::mbar_wait(&bar, 0, &never, limit_ns)) report(status, GDN_ERR_TIMEOUT);
+}
+
+int gdn_selftest_wait_timeout(long long limit_ns, void* stream)
+{
+    if (limit_ns < 1000000LL || limit_ns > 2000000000LL) return GDN_ERR_INVALID_ARG;
+    int* status = status_ptr();
+    if (!status) return GDN_ERR_CUDA;
+    gdn_selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status,
+                                                                                 (unsigned long long)limit_ns);
+    return cudaPeekAtLastError() == cudaSuccess ? GDN_OK : GDN_ERR_LAUNCH;
+}
+
 int gdn_get_device_status(void* stream)
 {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDN_ERR_CUDA;

@@ -33,6 +33,7 @@ EXPORTS = (
     "gdn_decode_verify",
     "gdn_decode_verify_tree",
     "gdn_get_device_status",
+    "gdn_selftest_wait_timeout",
     "gdn_profile_start",
     "gdn_profile_stop",
 )
@@ -80,6 +81,8 @@ def lib() -> ctypes.CDLL:
     L.gdn_decode_verify_tree.restype = i32
     L.gdn_get_device_status.argtypes = [vp]
     L.gdn_get_device_status.restype = i32
+    L.gdn_selftest_wait_timeout.argtypes = [i64, vp]
+    L.gdn_selftest_wait_timeout.restype = i32
     L.gdn_profile_start.argtypes = []
     L.gdn_profile_start.restype = i32
     L.gdn_profile_stop.argtypes = [i32, ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),

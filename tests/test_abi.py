@@ -154,6 +154,12 @@ def test_status_string_names_bad_parents(L):
     assert b"BAD_PARENTS" in L.gdn_status_string(-9)
 
 
+def test_selftest_rejects_out_of_range_limits(L):
+    """Both limits are refused before any launch."""
+    assert L.gdn_selftest_wait_timeout(999_999, None) == -1
+    assert L.gdn_selftest_wait_timeout(2_000_000_001, None) == -1
+
+
 def prefill_cuts(L, **kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu=FAKE, N=2, T=64, cuts=FAKE, nc=2, s_in=None, out=FAKE,
              s_out=FAKE, snaps=FAKE, H=2, dk=128, dv=128, dtype=1, ws=FAKE, ws_bytes=1 << 30, stream=None)
