@@ -1,7 +1,8 @@
-"""The prefill on a side stream, back to back with the call that feeds it, and inside a CUDA graph.
+"""The prefill on a side stream, back to back with the call that feeds it, and inside a CUDA graph;
+a chain of decode steps and a tree verify inside a CUDA graph.
 
-The prep and scan kernels of a call are launched as programmatic dependents of the kernel before
-them in the stream, and wait for it on the device before reading its results. These checks
+The prep, scan, decode and verify kernels are launched as programmatic dependents of the kernel
+before them in the stream, and wait for it on the device before reading its results. These checks
 confirm that the dependency holds in the ways a caller uses the library:
 - on a non-default stream;
 - two calls in a row where the second resumes from the first's final state, with nothing between
@@ -96,4 +97,46 @@ def test_cuda_graph_replay_matches_eager(dtype):
         torch.cuda.synchronize()
         assert gdn.gdn_get_device_status() == 0
         assert torch.equal(out, ref_out) and torch.equal(st, ref_st)
+    del graph
+
+
+def test_decode_chain_and_tree_verify_graph_replay_matches_eager():
+    """Eight chained decode steps and a tree verify recorded into one CUDA graph: each replay
+    equals the eager sequence bit for bit (the decode and verify kernels are dependent launches)."""
+    from linear_attention_10_b200.workloads import best_first_parents, make_decode_inputs, make_verify_inputs
+    B, H, d, steps = 4, 3, 128, 8
+    dd = make_decode_inputs(B, H, d, d, steps, dtype="bf16", seed=41, device=DEV)
+    vd = make_verify_inputs(B, H, d, d, 6, dtype="bf16", seed=42, device=DEV)
+    par = torch.tensor([best_first_parents(6)] * B, dtype=torch.int32, device=DEV)
+
+    def sequence(S, outs, vout, vst, stream=None):
+        for t in range(steps):
+            gdn.gdn_decode_step(dd["q"][t], dd["k"][t], dd["v"][t], dd["g"][t], dd["beta"][t], S, out=outs[t],
+                                stream=stream)
+        gdn.gdn_decode_verify_tree(vd["q"], vd["k"], vd["v"], vd["g"], vd["beta"], par, S, states_out=vst,
+                                   out=vout, stream=stream)
+
+    def buffers():
+        return (dd["state"].clone(), [torch.empty((B, H, d), dtype=torch.bfloat16, device=DEV) for _ in range(steps)],
+                torch.empty((B, 6, H, d), dtype=torch.bfloat16, device=DEV),
+                torch.empty((B, 6, H, d, d), dtype=torch.float32, device=DEV))
+
+    S_ref, o_ref, vo_ref, vs_ref = buffers()
+    sequence(S_ref, o_ref, vo_ref, vs_ref)
+    torch.cuda.synchronize()
+    assert gdn.gdn_get_device_status() == 0
+
+    S, outs, vout, vst = buffers()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        sequence(S, outs, vout, vst, stream=torch.cuda.current_stream())
+    for _ in range(2):
+        S.copy_(dd["state"])
+        graph.replay()
+        torch.cuda.synchronize()
+        assert gdn.gdn_get_device_status() == 0
+        assert torch.equal(S, S_ref) and torch.equal(vout, vo_ref) and torch.equal(vst, vs_ref)
+        assert all(torch.equal(a, b) for a, b in zip(outs, o_ref))
     del graph
