@@ -377,6 +377,16 @@ def run_ours(args, rank, world, local_rank):
     prof = gdn.gdn_profile_stop()
     if gdn.gdn_get_device_status() != 0:
         raise RuntimeError("device status error in the profiled pass")
+    # ---- the per-call distribution: the same K steps with an event pair around each whole call (an
+    # event between calls separates nothing: each call's first kernel is an ordinary launch) ----
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        evs[i][0].record(stream)
+        step(i)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    per_call_ms = sorted(max_over_ranks(a.elapsed_time(b_), world, dev) for a, b_ in evs)
     ms_per_step = ms / args.steps
     value = job_throughput(T_PREFILL, args.steps, world, ms)
 
@@ -654,6 +664,8 @@ def run_ours(args, rank, world, local_rank):
     launches = sum(v[1] for v in prof.values())
     line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
                 ms_per_step=ms_per_step, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="tf32x3",
+                per_call_ms=dict(median=statistics.median(per_call_ms), min=per_call_ms[0], max=per_call_ms[-1],
+                                 calls=len(per_call_ms), timing="an event pair around each whole call"),
                 data="synthetic",
                 config=dict(workload="%s: %s" % (WORKLOAD, WORKLOAD_DESC), global_batch=world, seq_len=T_PREFILL,
                             parallelism="one independent prefill per GPU" if world > 1 else "1 GPU",
