@@ -7,6 +7,8 @@ One step = one ``gdn_chunk_prefill`` call over the 4096-token workload (B=1, T=4
 dk=dv=128, bf16 q/k/v, fp32 g/beta, C=32, zero initial state, final state written).  Under torchrun
 every rank runs its own independent prefill (weak scaling, no data-path collective).  The line also
 carries the recurrent decode step (B=64, H=32, d=128, 1000 chained steps) as ``decode``.
+``--shard heads`` instead splits one layer's 32 heads over the ranks (strong scaling; ``--gather``
+adds an all-gather of the outputs to every step).
 
 Timing: CUDA events on the launching stream, W warm-up steps, barrier + synchronize around the K
 timed steps, max over ranks.  L2: every step reads one of three rotating input sets (about 300 MB
@@ -684,6 +686,76 @@ def run_ours(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_sharded(args, rank, world, local_rank):
+    """--shard heads: one layer's prefill split by heads over the ranks (strong scaling).  Every rank
+    builds the same layer (same seeds) and runs the library on its own contiguous block of heads;
+    there is no data-path exchange.  value = the layer's tokens per second over the slowest rank.
+    With --gather every step also all-gathers the output blocks (one NCCL all-gather), so that each
+    rank holds the whole layer's output."""
+    import torch
+    import torch.distributed as dist
+    from linear_attention_10_b200 import gdn
+    from linear_attention_10_b200.shard import gather_heads, head_range, shard_heads
+    from linear_attention_10_b200.workloads import workload_inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    gdn.lib()
+    stream = torch.cuda.current_stream()
+    if args.gather and H % world:
+        raise SystemExit("--gather needs the %d heads to divide evenly over %d ranks" % (H, world))
+    h0, h1 = head_range(rank, world, H)
+    Hl = h1 - h0
+    sets = [shard_heads(workload_inputs(WORKLOAD, device=dev, seed=1000 + i), rank, world) for i in range(3)]
+    ws = torch.empty(gdn.workspace_bytes(T_PREFILL, 1, Hl, D, D), dtype=torch.uint8, device=dev)
+    out = torch.empty((T_PREFILL, Hl, D), dtype=torch.bfloat16, device=dev)
+    st_out = torch.empty((1, Hl, D, D), dtype=torch.float32, device=dev)
+
+    def step(i):
+        s = sets[i % 3]
+        gdn.gdn_chunk_prefill(s["q"], s["k"], s["v"], s["g"], s["beta"], cu_seqlens=s["cu_seqlens"],
+                              out=out, state_out=st_out, workspace=ws)
+        if args.gather:
+            gather_heads(out, world)
+
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    if gdn.gdn_get_device_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+    clocks = ClockSampler(None)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    clk = clocks.stop()
+    if gdn.gdn_get_device_status() != 0:
+        raise RuntimeError("device status error in the timed region")
+    if rank != 0:
+        return
+    value = T_PREFILL * args.steps / (ms / 1e3)
+    line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
+                ms_per_step=ms / args.steps, higher_is_better=True, scaling="strong", vs_baseline=None,
+                dtype="tf32x3", data="synthetic",
+                config=dict(workload="%s: %s" % (WORKLOAD, WORKLOAD_DESC), global_batch=1, seq_len=T_PREFILL,
+                            parallelism="heads sharded over %d GPUs (%d heads on rank 0)%s"
+                                        % (world, Hl, ", outputs all-gathered every step" if args.gather else ""),
+                            l2="3 rotating input sets"),
+                roofline=None, e2e=None, gpu_launches=3 * args.steps, clocks=clk,
+                note="head-sharded layout of one layer; the default mode carries the roofline and e2e figures")
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -697,6 +769,9 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-cpu-all", action="store_true", help="skip the all-cores oracle timing")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--shard", choices=["none", "heads"], default="none",
+                    help="heads: split one layer's heads over the ranks instead of one prefill per rank")
+    ap.add_argument("--gather", action="store_true", help="with --shard heads: all-gather the outputs every step")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -712,7 +787,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, rank, world, local_rank)
+        if args.shard == "heads":
+            run_sharded(args, rank, world, local_rank)
+        else:
+            run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist
