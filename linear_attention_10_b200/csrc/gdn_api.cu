@@ -265,7 +265,7 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PL::kBytes) != cudaSuccess)
             return GDN_ERR_LAUNCH;
         const int64_t items = lay.nc_max * (int64_t)H;
-        const int64_t cap = (int64_t)g_num_sms * 4;
+        const int64_t cap = (int64_t)g_num_sms * kPrepBf16CtasPerSm;
         const unsigned grid = (unsigned)(items < cap ? items : cap);
         ProfScope prof("gdn_prep_bf16_kernel", st);
         if (launch_dependent(k1, dim3(grid), dim3(128), PL::kBytes, st, tq, tk, g, beta, meta, chunk_off, chunk_tab,

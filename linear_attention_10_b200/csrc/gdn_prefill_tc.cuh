@@ -110,6 +110,10 @@ __device__ __forceinline__ void stg128(void* p, const uint32_t (&w)[4])
 {
     asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
 }
+__device__ __forceinline__ void stg64(void* p, const uint32_t (&w)[2])
+{
+    asm volatile("st.global.v2.b32 [%0], {%1, %2};" ::"l"(p), "r"(w[0]), "r"(w[1]));
+}
 
 // Stores 8 consecutive K-elements (k0 % 8 == 0) of row r of a K-major SW128 tile of R rows, as hi
 // (and lo when SPLIT) parts.

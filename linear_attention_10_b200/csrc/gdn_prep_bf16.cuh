@@ -9,8 +9,9 @@
 //   D_ij = exp(gamma_i - gamma_j),  T = (I + A)^-1,  T'' = T diag(beta).
 //
 // What is specific to bf16 inputs: the chunk's [K; Q] rows are exact bf16 values, so the tensor-
-// memory-access engine copies them straight into the 128-byte-swizzled operand layout (two items
-// in flight per CTA) and one bf16 tensor-core product (M = 128, N = 32, K = dk) forms both Gram
+// memory-access engine copies them straight into the 128-byte-swizzled operand layout (the next
+// item's rows arrive while this one is gated, solved and written out, five CTAs per SM) and one
+// bf16 tensor-core product (M = 128, N = 32, K = dk) forms both Gram
 // matrices exactly in fp32.  The gates are applied while the Gram rows come out of tensor memory.
 // The inverse uses the 2 x 2 block form with 16 x 16 blocks,
 //
@@ -41,9 +42,10 @@ struct PrepBf16Smem {
     // at least 8 KB of this CTA's shared memory on both sides.
     static constexpr uint32_t kTile = NP * 8192;                      // [K;Q] bf16: NP panels x 64 rows x 128 B
     static constexpr uint32_t oPrev = 0;                              // previous chunk's K: NP x 32 rows x 128 B
-    static constexpr uint32_t oTile = 8192;                           // two buffers
+    static constexpr uint32_t oTile = 8192;                           // one buffer, refilled once the item's
+                                                                      // products have read it
     static constexpr int LD = 36;                                     // row pitch: 16-byte rows, no bank conflicts
-    static constexpr uint32_t oG = oTile + 2 * kTile;                 // [32][LD] A
+    static constexpr uint32_t oG = oTile + kTile;                     // [32][LD] A
     static constexpr uint32_t oP = oG + 32 * LD * 4;                  // [32][LD] P
     static constexpr uint32_t oT = oP + 32 * LD * 4;                  // [32][LD] T
     static constexpr int LM = 16;                                     // pitch of M (2-way write conflicts)
@@ -51,18 +53,21 @@ struct PrepBf16Smem {
     static constexpr uint32_t oGam = oM + 16 * LM * 4;
     static constexpr uint32_t oBet = oGam + 128;
     static constexpr uint32_t oAlph = oBet + 128;                     // per-token decays exp(g), one spare
-    static constexpr uint32_t oBar = oAlph + 136;   // tile_full[2], mma, drain[2], prev_full, cross
+    static constexpr uint32_t oBar = oAlph + 136;   // tile_full, (spare), mma, drain[2], prev_full, cross
     static constexpr uint32_t oTmem = oBar + 56;
     static constexpr uint32_t oAbort = oTmem + 4;
     static constexpr uint32_t kTotal = oAbort + 4;
     static constexpr uint32_t kBytes = kTotal + 1024;
     static_assert(NP * 4096 <= oTile, "previous-K buffer; 8 KB before the first tile");
     static_assert(kTotal >= oG + 8192, "rows read after the last tile's last panel");
-    static_assert(kBytes <= 57344, "four CTAs per SM");
+    static_assert(5 * (kBytes + 1024) <= 233472, "five CTAs per SM (1 KB reserved per CTA)");
 };
 
+// CTAs resident per SM (shared memory and registers are sized for it; the launch sizes its grid so)
+constexpr int kPrepBf16CtasPerSm = 5;
+
 template <int DK>
-__global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
+__global__ void __launch_bounds__(128, kPrepBf16CtasPerSm) gdn_prep_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                                const __grid_constant__ CUtensorMap tm_k,
                                                                const float* __restrict__ g,
                                                                const float* __restrict__ beta,
@@ -120,16 +125,17 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
 
     // whether chunk gc has a previous chunk in its sequence (then the cross-chunk Gram is built)
     auto has_prev = [&](int gc) { return gc > chunk_off[chunk_tab[gc].x]; };
-    // copies the [K; Q] rows of one item into tile buffer `b` (one thread per fill)
-    auto issue_tile = [&](int item, int b) {
+    // copies the [K; Q] rows of one item into the tile buffer (one thread per fill; issued once the
+    // previous item's products have read the buffer)
+    auto issue_tile = [&](int item) {
         const int gc = item / H, h = item % H;
         const int t0 = chunk_tab[gc].y;
-        const uint32_t dst = sbase + L::oTile + b * L::kTile;
-        mbar_arrive_expect_tx(&tile_full[b], NP * 2 * 4096);
+        const uint32_t dst = sbase + L::oTile;
+        mbar_arrive_expect_tx(tile_full, NP * 2 * 4096);
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
-            tma_load_2d(dst + p * 8192, &tm_k, h * DK + p * 64, t0, &tile_full[b]);
-            tma_load_2d(dst + p * 8192 + 4096, &tm_q, h * DK + p * 64, t0, &tile_full[b]);
+            tma_load_2d(dst + p * 8192, &tm_k, h * DK + p * 64, t0, tile_full);
+            tma_load_2d(dst + p * 8192 + 4096, &tm_q, h * DK + p * 64, t0, tile_full);
         }
     };
     // copies the previous chunk's K rows of one item into the single previous-K buffer (one thread;
@@ -153,8 +159,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
     };
 
     if (tid == 0) {
-        if ((int)blockIdx.x < nitems) issue_tile(blockIdx.x, 0);
-        if ((int)(blockIdx.x + gridDim.x) < nitems) issue_tile(blockIdx.x + gridDim.x, 1);
+        if ((int)blockIdx.x < nitems) issue_tile(blockIdx.x);
         if ((int)blockIdx.x < nitems) issue_prev(blockIdx.x);
     }
     float gv_cur = 0.f, bv_cur = 0.f;
@@ -164,18 +169,17 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
     uint32_t iter = 0;
     for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++iter) {
         GDN_PREP_TRACE(iter, 0);
-        const int b = iter & 1;
         const int gc = item / H, h = item % H;
         const int Lr = chunk_tab[gc].z;
         const bool prev = has_prev(gc);
 
         // Gram products D[r][n] = [K; Q]_r . K_n on the tensor cores, rows in lanes 0..63 (thread 0)
         if (tid == 0) {
-            if (!mbar_wait(&tile_full[b], (iter >> 1) & 1u, abort_flag)) {
+            if (!mbar_wait(tile_full, iter & 1u, abort_flag)) {
                 tc_abort(status, abort_flag);
             } else {
                 tc_fence_after();
-                const uint64_t a = sw128_desc(sbase + L::oTile + b * L::kTile, 0, 64);
+                const uint64_t a = sw128_desc(sbase + L::oTile, 0, 64);
 #pragma unroll
                 for (int ks = 0; ks < DK / 16; ++ks) {
                     const uint64_t o = sw128_ks_off(ks, 64);
@@ -188,13 +192,12 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
             // G' = [K; Q] K_prev^T (thread 96), completes while the gates are applied.  A starts 64
             // rows (8 KB) before the tile, so row r of [K; Q] is row 64 + r of the product: lanes
             // 64..127, and its columns 32..63
-            if (!mbar_wait(&tile_full[b], (iter >> 1) & 1u, abort_flag) ||
-                !mbar_wait(prev_full, iter & 1u, abort_flag)) {
+            if (!mbar_wait(tile_full, iter & 1u, abort_flag) || !mbar_wait(prev_full, iter & 1u, abort_flag)) {
                 tc_abort(status, abort_flag);
             } else {
                 tc_fence_after();
                 if (prev) {
-                    const uint64_t a = sw128_desc(sbase + L::oTile + b * L::kTile - 8192, 0, 64);
+                    const uint64_t a = sw128_desc(sbase + L::oTile - 8192, 0, 64);
                     const uint64_t bp = sw128_desc(sbase + L::oPrev, 0, 32);
 #pragma unroll
                     for (int ks = 0; ks < DK / 16; ++ks)
@@ -245,15 +248,17 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
                              "f"(vals[4 * q + 1]), "f"(vals[4 * q + 2]), "f"(vals[4 * q + 3]));
             GDN_PREP_TRACE(iter, 6);
         } else {
-            // warps 2 and 3: the tile buffers are free once G' has been formed (the chunk's own Gram
-            // was waited for before the barrier above): fetch the item after next and the next item's
+            // warps 2 and 3: the tile buffer is free once G' has been formed (the chunk's own Gram
+            // was waited for before the barrier above): fetch the next item's [K; Q] rows and
             // previous-chunk keys, then split G'
             if (tid == 64 && !mbar_wait(cross_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
             named_bar(1, 64);
             tc_fence_after();
             if (tid == 64 && !*abort_flag) {
-                if (item + 2 * (int)gridDim.x < nitems) issue_tile(item + 2 * gridDim.x, b);
-                if (item + (int)gridDim.x < nitems) issue_prev(item + gridDim.x);
+                if (item + (int)gridDim.x < nitems) {
+                    issue_tile(item + gridDim.x);
+                    issue_prev(item + gridDim.x);
+                }
             }
             if (prev) {
                 // row (32 (w - 2) + lane) of G', in lane 32 w + lane -> three bf16 parts, K-major
@@ -299,82 +304,96 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_bf16_kernel(const __grid_cons
         }
         __syncthreads();
         {
-            // M1 = A21 T11 (16 x 16): two outputs per thread
+            // M1 = A21 T11 (16 x 16): two outputs per thread; row r of A21 in four 16-byte loads,
+            // the two T11 columns as pairs
             const int r = tid >> 3, c = (tid & 7) * 2;
             float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float am = G[(16 + r) * LD + m];
-                a0 = fmaf(am, Tm[m * LD + c], a0);
-                a1 = fmaf(am, Tm[m * LD + c + 1], a1);
+            for (int m4 = 0; m4 < 4; ++m4) {
+                const float4 av = *reinterpret_cast<const float4*>(G + (16 + r) * LD + 4 * m4);
+                const float am[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 tv = *reinterpret_cast<const float2*>(Tm + (4 * m4 + e) * LD + c);
+                    a0 = fmaf(am[e], tv.x, a0);
+                    a1 = fmaf(am[e], tv.y, a1);
+                }
             }
-            M1[r * L::LM + c] = a0;
-            M1[r * L::LM + c + 1] = a1;
+            *reinterpret_cast<float2*>(M1 + r * L::LM + c) = make_float2(a0, a1);
         }
         __syncthreads();
         {
-            // T21 = -T22 M1
+            // T21 = -T22 M1, the same way
             const int r = tid >> 3, c = (tid & 7) * 2;
             float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float tm = Tm[(16 + r) * LD + 16 + m];
-                a0 = fmaf(tm, M1[m * L::LM + c], a0);
-                a1 = fmaf(tm, M1[m * L::LM + c + 1], a1);
+            for (int m4 = 0; m4 < 4; ++m4) {
+                const float4 tv4 = *reinterpret_cast<const float4*>(Tm + (16 + r) * LD + 16 + 4 * m4);
+                const float tm[4] = {tv4.x, tv4.y, tv4.z, tv4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 mv = *reinterpret_cast<const float2*>(M1 + (4 * m4 + e) * L::LM + c);
+                    a0 = fmaf(tm[e], mv.x, a0);
+                    a1 = fmaf(tm[e], mv.y, a1);
+                }
             }
-            Tm[(16 + r) * LD + c] = -a0;
-            Tm[(16 + r) * LD + c + 1] = -a1;
+            *reinterpret_cast<float2*>(Tm + (16 + r) * LD + c) = make_float2(-a0, -a1);
         }
         __syncthreads();
         GDN_PREP_TRACE(iter, 3);
 
-        // operator record: thread (i, cb) forms columns 8 cb .. 8 cb + 7 of row i of T'' = T diag(beta)
-        // and of P T'' = (P T) diag(beta), and writes each as three bf16 parts of 16 bytes into the
+        // operator record: thread (a, cb) forms columns 4 cb .. 4 cb + 3 of rows 2a and 2a + 1 of
+        // T'' = T diag(beta) and of P T'' = (P T) diag(beta) (a 2 x 4 block: each T row it loads
+        // serves both rows), and writes each as three bf16 parts of 8 bytes per row into the
         // 64-byte-swizzled A-operand image (rows 0..31: T'', rows 32..63: P T'')
         uint8_t* dst = op + ((size_t)gc * H + h) * kOpBytesB;
         {
-            const int i = tid >> 2, c0 = (tid & 3) * 8;
-            const float4 b0 = *reinterpret_cast<const float4*>(bet + c0);
-            const float4 b1 = *reinterpret_cast<const float4*>(bet + c0 + 4);
-            const float bc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-            float acc[8];
+            const int i0 = (tid >> 3) * 2, c0 = (tid & 7) * 4;
+            const float4 bv4 = *reinterpret_cast<const float4*>(bet + c0);
+            const float bc[4] = {bv4.x, bv4.y, bv4.z, bv4.w};
+            float acc[2][4];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-            const float4* prow = reinterpret_cast<const float4*>(P + i * LD);
+            for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[rr][c] = 0.f;
+            const float4* p0 = reinterpret_cast<const float4*>(P + i0 * LD);
+            const float4* p1 = reinterpret_cast<const float4*>(P + (i0 + 1) * LD);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const float4 pv = prow[q];
-                const float pm[4] = {pv.x, pv.y, pv.z, pv.w};
+                const float4 u0 = p0[q], u1 = p1[q];
+                const float pa[4] = {u0.x, u0.y, u0.z, u0.w}, pb[4] = {u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float4* trow = reinterpret_cast<const float4*>(Tm + (4 * q + e) * LD + c0);
-                    const float4 t0 = trow[0], t1 = trow[1];
-                    acc[0] = fmaf(pm[e], t0.x, acc[0]);
-                    acc[1] = fmaf(pm[e], t0.y, acc[1]);
-                    acc[2] = fmaf(pm[e], t0.z, acc[2]);
-                    acc[3] = fmaf(pm[e], t0.w, acc[3]);
-                    acc[4] = fmaf(pm[e], t1.x, acc[4]);
-                    acc[5] = fmaf(pm[e], t1.y, acc[5]);
-                    acc[6] = fmaf(pm[e], t1.z, acc[6]);
-                    acc[7] = fmaf(pm[e], t1.w, acc[7]);
+                    const float4 t = *reinterpret_cast<const float4*>(Tm + (4 * q + e) * LD + c0);
+                    acc[0][0] = fmaf(pa[e], t.x, acc[0][0]);
+                    acc[0][1] = fmaf(pa[e], t.y, acc[0][1]);
+                    acc[0][2] = fmaf(pa[e], t.z, acc[0][2]);
+                    acc[0][3] = fmaf(pa[e], t.w, acc[0][3]);
+                    acc[1][0] = fmaf(pb[e], t.x, acc[1][0]);
+                    acc[1][1] = fmaf(pb[e], t.y, acc[1][1]);
+                    acc[1][2] = fmaf(pb[e], t.z, acc[1][2]);
+                    acc[1][3] = fmaf(pb[e], t.w, acc[1][3]);
                 }
             }
-            const float4* tri = reinterpret_cast<const float4*>(Tm + i * LD + c0);
-            const float4 ti0 = tri[0], ti1 = tri[1];
-            const float tv[8] = {ti0.x, ti0.y, ti0.z, ti0.w, ti1.x, ti1.y, ti1.z, ti1.w};
-            uint32_t w1[4], w2[4], w3[4], x1[4], x2[4], x3[4];
 #pragma unroll
-            for (int c = 0; c < 8; c += 2) {
-                bf16x2_split3(tv[c] * bc[c], tv[c + 1] * bc[c + 1], w1[c / 2], w2[c / 2], w3[c / 2]);
-                bf16x2_split3(acc[c] * bc[c], acc[c + 1] * bc[c + 1], x1[c / 2], x2[c / 2], x3[c / 2]);
+            for (int rr = 0; rr < 2; ++rr) {
+                const int i = i0 + rr;
+                const float4 tv4 = *reinterpret_cast<const float4*>(Tm + i * LD + c0);
+                const float tv[4] = {tv4.x, tv4.y, tv4.z, tv4.w};
+                uint32_t w1[2], w2[2], w3[2], x1[2], x2[2], x3[2];
+#pragma unroll
+                for (int c = 0; c < 4; c += 2) {
+                    bf16x2_split3(tv[c] * bc[c], tv[c + 1] * bc[c + 1], w1[c / 2], w2[c / 2], w3[c / 2]);
+                    bf16x2_split3(acc[rr][c] * bc[c], acc[rr][c + 1] * bc[c + 1], x1[c / 2], x2[c / 2], x3[c / 2]);
+                }
+                const uint32_t ot = sw64_off_h(i, c0), op2 = sw64_off_h(32 + i, c0);
+                stg64(dst + ot, w1);
+                stg64(dst + kOpBPart + ot, w2);
+                stg64(dst + 2 * kOpBPart + ot, w3);
+                stg64(dst + op2, x1);
+                stg64(dst + kOpBPart + op2, x2);
+                stg64(dst + 2 * kOpBPart + op2, x3);
             }
-            const uint32_t ot = sw64_off_h(i, c0), op2 = sw64_off_h(32 + i, c0);
-            stg128(dst + ot, w1);
-            stg128(dst + kOpBPart + ot, w2);
-            stg128(dst + 2 * kOpBPart + ot, w3);
-            stg128(dst + op2, x1);
-            stg128(dst + kOpBPart + op2, x2);
-            stg128(dst + 2 * kOpBPart + op2, x3);
         }
         if (tid < 80) {
             float* gt = reinterpret_cast<float*>(dst + kOpBGate);
