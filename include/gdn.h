@@ -2,10 +2,11 @@
  * gdn.h -- C ABI of the B200 (sm_100a) gated-delta-rule library, libgdn.so.
  *
  * The operation.  Ferrite project page (bhcc2025.github.io/ferrite), Design section 03 "Chunked
- * Gated DeltaNet": a linear-attention layer keeps one recurrent state per request; prompt rows go
- * through it in chunks of 32 using the chunkwise WY/UT form of the delta rule on TF32 tensor cores
- * with a 3xTF32 split for fp32 accuracy, and the state is written back for decoding.  The state
- * recurrence is the gated delta rule (Yang, Kautz and Hatamizadeh, "Gated Delta Networks"), per
+ * Gated DeltaNet": the section names the method -- each linear-attention layer holds a recurrent
+ * state for every request, a prompt is processed 32 rows at a time with the WY/UT chunk form of the
+ * delta rule, its products on TF32 tensor cores (three-way TF32 splitting for fp32-level
+ * accuracy), and the state left at the end of the prompt is what the decoder continues from.  The
+ * state recurrence is the gated delta rule (Yang, Kautz and Hatamizadeh, "Gated Delta Networks"), per
  * sequence and head:
  *
  *     S_t = exp(g_t) * S_{t-1} * (I - beta_t k_t k_t^T) + beta_t v_t k_t^T      (S is dv x dk)
@@ -130,9 +131,9 @@ int gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* 
                       void* stream);
 
 /*
- * Chunked prefill with state snapshots at cut points (Ferrite project page, Design section 07:
- * conversations are snapshotted at turn boundaries, and prompts are cut at the same points with or
- * without a resume).  Same as gdn_chunk_prefill, plus: for every cut point c_i, snapshots[i]
+ * Chunked prefill with state snapshots at cut points (Ferrite project page, Design section 07: the
+ * prompt cache saves a conversation's state where each turn ends, and a prompt is split at identical
+ * places whether or not it resumes from such a save).  Same as gdn_chunk_prefill, plus: for every cut point c_i, snapshots[i]
  * receives the state of the sequence that contains c_i after its tokens before c_i.  Chunks restart
  * at every cut, so each snapshot, every output and each final state are bit for bit what a call
  * that stops at c_i and a second call resumed from that state would give.
@@ -214,8 +215,8 @@ int gdn_decode_verify(const void* q, const void* k, const void* v, const float* 
                       int Tk, int H, int dk, int dv, int dtype, void* stream);
 
 /*
- * Tree verify (Ferrite project page, Design section 04: drafted tokens are verified as best-first
- * trees in one pass of the model).  As gdn_decode_verify, but the Tk drafted tokens of a sequence
+ * Tree verify (Ferrite project page, Design section 04: the big model checks the drafter's tokens
+ * in a single pass, with the drafts arranged as a tree grown best-first).  As gdn_decode_verify, but the Tk drafted tokens of a sequence
  * form a tree: token t continues from the state after token parents[b * Tk + t], which must be an
  * earlier token (< t), or from the committed state when the parent is -1.  A linear chain
  * (parents[b * Tk + t] = t - 1) gives exactly gdn_decode_verify.

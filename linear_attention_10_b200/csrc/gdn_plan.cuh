@@ -1,9 +1,9 @@
 // gdn_plan.cuh -- chunk tables of a packed prefill call, and the workspace layout.
 //
 // Chunks of C = 32 rows restart at every sequence start (Ferrite project page, Design section 03:
-// prompt rows go through the layer in chunks of 32) and at every cut point the caller asks a state
-// snapshot for (section 07: conversations are snapshotted at turn boundaries, and prompts are cut at
-// the same points with or without a resume, so that a resumed reply matches one computed in full).
+// the layer takes a prompt 32 rows at a time) and at every cut point the caller asks a state
+// snapshot for (section 07: the prompt cache saves state where each turn ends and splits a prompt at
+// identical places with or without a resume, which is what makes a resumed reply equal to a full one).
 // A segment is the piece of a sequence between two such boundaries.  One CTA validates cu_seqlens
 // and the cut points on the device, places the segments in token order, counts and scans their
 // chunks, and fills a table that maps a global chunk index to (sequence, first token, rows,

@@ -1,8 +1,8 @@
 // gdn_prefill_tc.cuh -- chunkwise WY/UT prefill of the gated delta rule on tcgen05 tensor cores.
 //
-// Ferrite project page, Design section 03 "Chunked Gated DeltaNet": prompt rows go through the
-// recurrent state in chunks of 32 using the chunkwise WY/UT form of the delta rule on TF32 tensor
-// cores with a 3xTF32 split for fp32 accuracy; the final state is written back for decoding.
+// Ferrite project page, Design section 03 "Chunked Gated DeltaNet": a prompt is taken 32 rows at a
+// time with the WY/UT chunk form of the delta rule, its products on TF32 tensor cores, split three
+// ways for fp32-level accuracy, and the decoder continues from the state left at the prompt's end.
 //
 // Notation for one chunk of L <= 32 rows (rows L..31 are padding: q = k = v = 0, g = 0, beta = 0);
 // S is the dv x dk state entering the chunk, s = 1/sqrt(dk):

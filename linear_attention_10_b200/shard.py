@@ -1,9 +1,9 @@
 """Head sharding of one layer over the ranks of a process group (tensor-parallel style).
 
 The heads of a layer are independent: a head's q, k, v, g, beta, state and output rows are read and
-written by that head alone.  The two-node setup of the Ferrite project page (Design section 05) gives
-each node half of every layer; here rank r of W runs the library on a contiguous block of heads of
-its own, with no exchange.  Only a caller that wants a whole layer's output or state on every rank
+written by that head alone.  The two-node setup of the Ferrite project page (Design section 05)
+splits each layer between the two machines; here rank r of W runs the library on a contiguous block
+of heads of its own, with no exchange.  Only a caller that wants a whole layer's output or state on every rank
 gathers the blocks, with one all-gather per tensor (NCCL on GPUs, gloo on the host).
 
 This module is host plumbing: it slices and gathers tensors and calls ``torch.distributed``.  Every

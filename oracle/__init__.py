@@ -16,7 +16,7 @@ What is computed and why (each function cites its source):
 * ``decode_step``, ``decode_verify``, ``decode_verify_tree`` -- the recurrence one token at a time
                      from a given state: one step, a chain of drafted tokens, and a tree of drafted
                      tokens where each node continues from its parent's state (Ferrite project page,
-                     Design section 04, drafts verified as best-first trees); ``tree_path`` lists the
+                     Design section 04: drafts checked in one pass as a best-first tree); ``tree_path`` lists the
                      nodes from the root to a node.
 * ``states_at``   -- the recurrence with the state captured at cut points (Design section 07).
 * ``chunk_operator``, ``chunk_step`` -- one chunk's state-independent WY/UT quantities (the decay
@@ -266,7 +266,7 @@ def decode_verify(q, k, v, g, beta, state):
 
 def decode_verify_tree(q, k, v, g, beta, parents, state):
     """Tk drafted tokens per sequence arranged as a tree (Ferrite project page, Design section 04:
-    drafts are verified as best-first trees in one pass of the model).  Node t of sequence b follows
+    the big model checks the drafts in a single pass, arranged as a tree grown best-first).  Node t of sequence b follows
     node ``parents[b, t]`` (an earlier node, < t) or, when that is -1, the committed ``state`` (not
     modified): its state is the decode step of its token applied to its parent's state.  Inputs as
     ``decode_verify`` plus ``parents`` int ``[B, Tk]``.  Returns ``(out [B, Tk, H, dv], states

@@ -6,10 +6,10 @@
  * header, table or constant with the CUDA library.
  *
  * What it computes.  The Ferrite project page (bhcc2025.github.io/ferrite), Design section 03
- * "Chunked Gated DeltaNet", says that the linear-attention layers keep one recurrent state per
- * request, push prompt rows through it in chunks of 32 with the chunkwise WY/UT form of the delta
- * rule on TF32 tensor cores (3xTF32 split), and write the state back for decoding.  The page does
- * not print the recurrence; the one used here is the published gated delta rule (Yang, Kautz and
+ * "Chunked Gated DeltaNet", names the method without writing it down: each linear-attention layer
+ * carries a recurrent state for every request, a prompt is handled 32 rows at a time with the WY/UT
+ * chunk form of the delta rule, its products on TF32 tensor cores (3xTF32 split), and the decoder
+ * continues from the state the prompt leaves.  The page does not print the recurrence; the one used here is the published gated delta rule (Yang, Kautz and
  * Hatamizadeh, "Gated Delta Networks: Improving Mamba2 with Delta Rule", 2024/2025).  Per sequence
  * and head, with S_0 the initial state (dv x dk, zero when none is given):
  *

@@ -1,6 +1,6 @@
 """GPU parity of gdn_chunk_prefill_cuts (state snapshots at cut points inside a prefill) against the
-fp64 oracle, and the resume property: the same cut points give the same result, bit for bit, in one
-call or in calls resumed from the snapshots."""
+fp64 oracle, and the resume property: one call with cut points and a chain of calls resumed from its
+snapshots give identical results, bit for bit."""
 import numpy as np
 import pytest
 import torch
