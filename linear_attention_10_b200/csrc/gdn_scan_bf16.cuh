@@ -179,6 +179,19 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
     // [X; Z] from the exact state before it, as a call resumed at the cut would
     auto seg_first = [&](int c) { return c == 0 || (CUTS && chunk_tab[c_begin + c - 1].w >= 0); };
 
+    // Operand descriptors of stage 0 and of the shared operand tiles, formed once: the copy in stage s
+    // is kStage * s bytes further, which adds kStage * s / 16 to the 14-bit start-address field (no
+    // carry: every address is below 256 KB).  The issuing threads then only add constants.
+    static_assert(L::kStage % 16 == 0 && kOpBPart % 16 == 0, "descriptor offsets");
+    constexpr uint64_t kStageD = L::kStage >> 4, kPartD = kOpBPart >> 4;
+    const uint64_t dOp0 = sw64_desc(sbase + L::oOp);                 // [T''; PT''] part 1, stage 0
+    const uint64_t dCr0 = sw64_desc(sbase + L::oOp + kOpBCross);     // G' part 1, stage 0
+    const uint64_t dKt0 = sw128_desc_mn(sbase + L::oAKQ, 8192, 1024); // K^T, stage 0
+    const uint64_t dKQ0 = sw128_desc(sbase + L::oAKQ, 0, 64);        // [K; Q], stage 0
+    const uint64_t dY = sw128_desc_mn(sbase + L::oBY, L::kLboU, 1024);
+    const uint64_t dU = sw128_desc_mn(sbase + L::oBU, L::kLboU, 1024);
+    const uint64_t dS = sw128_desc_mn(sbase + L::oBS, L::kLboS, 1024);
+
     const bool chain = warp < 8 && (warp & 3) < 2;
     const bool sgrp = (warp < 8) ? ((warp & 3) >= 2) : (warp == 8 || warp == 9 || warp == 12 || warp == 13);
 
@@ -321,13 +334,13 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
             // ---- MMA_b: [U; PU] = [T''; PT''] Y
             if (tid == 0) {
                 tc_fence_after();
-                const uint64_t b = sw128_desc_mn(sbase + L::oBY, L::kLboU, 1024);
+                const uint64_t a1 = dOp0 + (uint64_t)s * kStageD;
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks) {
                     const uint64_t ob = (uint64_t)(ks * 128), oa = (uint64_t)(ks * 2);
-                    mma_bf16(tD2, sw64_desc(st + L::oOp) + oa, b + ob, idB3, ks > 0);
-                    mma_bf16(tD2, sw64_desc(st + L::oOp + kOpBPart) + oa, b + ob, idB2, 1);
-                    mma_bf16(tD2, sw64_desc(st + L::oOp + 2 * kOpBPart) + oa, b + ob, idB1, 1);
+                    mma_bf16(tD2, a1 + oa, dY + ob, idB3, ks > 0);
+                    mma_bf16(tD2, a1 + kPartD + oa, dY + ob, idB2, 1);
+                    mma_bf16(tD2, a1 + 2 * kPartD + oa, dY + ob, idB1, 1);
                 }
                 mma_commit(bar_b);
             }
@@ -366,8 +379,8 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
                 bool ok2 = (c == 0) || mbar_wait(s_done, (uint32_t)(c - 1) & 1u, abort_flag);
                 GDN_SCAN_TRACE(c, 8);
                 if (ok2) {
-                    const uint64_t a = sw128_desc_mn(st + L::oAKQ, 8192, 1024);
-                    const uint64_t b = sw128_desc_mn(sbase + L::oBU, L::kLboU, 1024);
+                    const uint64_t a = dKt0 + (uint64_t)s * kStageD;
+                    const uint64_t b = dU;
 #pragma unroll
                     for (int ks = 0; ks < 2; ++ks)
                         mma_bf16(tD3, a + (uint64_t)(ks * 128), b + (uint64_t)(ks * 128), idC, ks > 0);
@@ -376,17 +389,17 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
                     // ---- MMA_x of the next chunk: D1 = G'_{c+1} U~_c
                     if (c + 1 < nch && (!CUTS || ctab_w < 0)) {
                         const int s1 = stage_of(c + 1);
+                        const uint64_t g1 = dCr0 + (uint64_t)s1 * kStageD;
                         ok2 = mbar_wait(&full[s1], phase_of(c + 1), abort_flag);
                         GDN_SCAN_TRACE(c, 10);
                         if (ok2) {
                             tc_fence_after();
-                            const uint32_t g = sbase + s1 * L::kStage + L::oOp + kOpBCross;
 #pragma unroll
                             for (int ks = 0; ks < 2; ++ks) {
                                 const uint64_t ob = (uint64_t)(ks * 128), oa = (uint64_t)(ks * 2);
-                                mma_bf16(tD1, sw64_desc(g) + oa, b + ob, idB3, ks > 0);
-                                mma_bf16(tD1, sw64_desc(g + kOpBPart) + oa, b + ob, idB2, 1);
-                                mma_bf16(tD1, sw64_desc(g + 2 * kOpBPart) + oa, b + ob, idB1, 1);
+                                mma_bf16(tD1, g1 + oa, b + ob, idB3, ks > 0);
+                                mma_bf16(tD1, g1 + kPartD + oa, b + ob, idB2, 1);
+                                mma_bf16(tD1, g1 + 2 * kPartD + oa, b + ob, idB1, 1);
                             }
                             mma_commit(bar_x);
                         }
@@ -414,10 +427,10 @@ __global__ void __launch_bounds__(kScanBf16Threads, 1)
         // W_k = [K; Q]_k S^T into DW[k & 1], where the S parts hold the state entering chunk k - 1
         auto issue_w = [&](int k) -> bool {
             const int sk = stage_of(k);
+            const uint64_t a = dKQ0 + (uint64_t)sk * kStageD;
+            const uint64_t b = dS;
             if (!mbar_wait(&full[sk], phase_of(k), abort_flag)) return false;
             tc_fence_after();
-            const uint64_t a = sw128_desc(sbase + sk * L::kStage + L::oAKQ, 0, 64);
-            const uint64_t b = sw128_desc_mn(sbase + L::oBS, L::kLboS, 1024);
             const uint32_t d = (k & 1) ? tDW1 : tDW0;
 #pragma unroll
             for (int ks = 0; ks < DK / 16; ++ks)
