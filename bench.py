@@ -72,7 +72,7 @@ KERNELS = {
 # and verify figures undercount writes: ncu starts each replay from a clean L2, and 56-58 MB of the
 # written states are still resident (dirty) in L2 when the launch ends.
 TRAFFIC = {
-    "gdn_scan_bf16_kernel": 202.95e6 + 26.51e6,
+    "gdn_scan_bf16_kernel": 202.96e6 + 28.44e6,
     "gdn_prep_bf16_kernel": 68.24e6 + 48.38e6,
     "gdn_l2norm_kernel": 67.12e6 + 21.02e6,
     "gdn_decode_step_kernel": 135.83e6 + 77.84e6,
