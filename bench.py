@@ -93,6 +93,35 @@ def load_peaks():
                     source="fallback")
 
 
+# Nominal dense peaks of one B200, stated for the "% of roofline" the metric asks for beside the
+# measured-peak figures: TF32 tensor 1.125 PFLOP/s (half the 2:4-sparse datasheet figure), HBM3e 8 TB/s.
+NOMINAL_TF32_TFLOPS = 1125.0
+NOMINAL_HBM_GBS = 8000.0
+
+
+def prefill_api_bytes(T, Hh, d, N, state_in, es=2):
+    """Algorithmic bytes of one prefill call: the API's inputs and outputs only (q, k, v, out in the
+    storage type of es bytes, g and beta fp32, state_in if given and state_out fp32)."""
+    return 4 * T * Hh * d * es + 2 * T * Hh * 4 + (2 if state_in else 1) * N * Hh * d * d * 4
+
+
+def method_roofline_of(T, Hh, d, N, state_in, call_ms, peaks, es=2):
+    """Whole-call roofline of the method, max(3 F T H / TF32 peak, API bytes / HBM peak), against the
+    measured call time; at the measured-derived peaks (the headline) and at the nominal ones."""
+    flops3 = 3 * flops_whole(d) * T * Hh
+    nbytes = prefill_api_bytes(T, Hh, d, N, state_in, es)
+
+    def at(tf32, hbm):
+        t_flop, t_byte = flops3 / (tf32 * 1e12), nbytes / (hbm * 1e9)
+        r = max(t_flop, t_byte)
+        return dict(bound="tensor(TF32 x3)" if t_flop >= t_byte else "hbm", roofline_us=r * 1e6,
+                    frac=r / (call_ms / 1e3), tf32_peak_tflops=tf32, hbm_peak_gbs=hbm)
+    tf32, _, _ = peak_for("tensor", peaks)
+    return dict(achieved_us=call_ms * 1e3, flops_x3=flops3, api_bytes=nbytes,
+                measured_peaks=at(tf32, peaks["hbm_gbs"]), nominal_peaks=at(NOMINAL_TF32_TFLOPS, NOMINAL_HBM_GBS),
+                headline="measured_peaks")
+
+
 def peak_for(bound, peaks):
     if bound == "tensor":
         return peaks["bf16_tflops"] * (1.1 / 2.25), "TFLOP/s", "%s bf16 GEMM x 1.1/2.25 (TF32)" % peaks["source"]
@@ -301,6 +330,135 @@ def run_reference(args, rank, world):
                 cpu_baseline=dict(value=value, unit=UNIT, cores=1, kind="oracle", sample=sample),
                 e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
     print(json.dumps(line), flush=True)
+
+
+
+# ---------------------------------------------------------------------------------------------------
+# the other prefill workloads of the method (varlen resume, 128K context, tiny fp32)
+# ---------------------------------------------------------------------------------------------------
+WORKLOAD_DESCS = {
+    "varlen_resume": "4 packed sequences of 8192/3000/517/13000 tokens (24,709), H=32, dk=dv=128, bf16 q/k/v, "
+                     "initial states ~N(0,0.05^2) per sequence, C=32, final states written",
+    "long_128k": "B=1, T=131072, H=32, dk=dv=128, bf16 q/k/v, zero initial state, C=32 (4096 sequential chunks)",
+    "tiny_fp32": "B=1, T=128 (4 chunks), H=2, dk=dv=64, fp32 q/k/v, g~U[-0.5,0), zero initial state",
+}
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel for these workloads
+# (None until captured, reset whenever the kernel changes)
+TRAFFIC_BY_WORKLOAD = {}
+
+
+def l2_flush_buffer(dev):
+    import torch
+    return torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+
+def bench_prefill_workload(name, reps, world, dev, stream, peaks, rank, flush=None):
+    """Times `reps` prefill calls of one named workload and returns its bench entry.  Workloads whose
+    q/k/v exceed L2 run back to back between one event pair (no call finds its inputs in L2); smaller
+    ones get an event pair per call with a 256 MB write between calls (outside the pairs) flushing L2,
+    and report the median call.  A second pass with an event pair around every launch gives the
+    per-kernel durations and the roofline of the dominant kernel."""
+    import torch
+    from linear_attention_10_b200 import gdn
+    from linear_attention_10_b200.workloads import WORKLOADS, workload_inputs
+    w = WORKLOADS[name]
+    inp = workload_inputs(name, device=dev, seed=w.seed + 1000 * rank)
+    T, N, Hh, d = w.total_tokens, len(w.lengths), w.H, w.dk
+    es = 2 if w.dtype == "bf16" else 4
+    out = torch.empty((T, Hh, w.dv), dtype=inp["q"].dtype, device=dev)
+    st = torch.empty((N, Hh, w.dv, d), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.workspace_bytes(T, N, Hh, d, w.dv), dtype=torch.uint8, device=dev)
+
+    def call(_i=0):
+        gdn.gdn_chunk_prefill(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], cu_seqlens=inp["cu_seqlens"],
+                              state_in=inp["state_in"], out=out, state_out=st, workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    big = 3 * T * Hh * d * es > 2 * 126e6
+    if big:
+        ms_all, prof = timed_passes(call, reps, world, dev, stream)
+        call_ms = ms_all / reps
+        timing = "%d calls back to back between one event pair (q/k/v %.0f MB > L2)" % (reps, 3 * T * Hh * d * es / 1e6)
+    else:
+        if flush is None:
+            flush = l2_flush_buffer(dev)
+        pairs = []
+        for _ in range(reps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call()
+            b.record(stream)
+            pairs.append((a, b))
+        torch.cuda.synchronize()
+        call_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in pairs), world, dev)
+        gdn.gdn_profile_start()
+        for _ in range(reps):
+            flush.fill_(1)
+            call()
+        torch.cuda.synchronize()
+        prof = gdn.gdn_profile_stop()
+        timing = "median of %d calls, each between its own event pair, L2 flushed (256 MB write) between calls" % reps
+    if gdn.gdn_get_device_status() != 0:
+        raise RuntimeError("device status error in workload %s" % name)
+    dom = max((n for n in prof if "flops_per_token_head" in KERNELS.get(n, {})), key=lambda n: prof[n][0])
+    kms, kl = prof[dom]
+    spec = KERNELS[dom]
+    per_unit = flops_scan(d) if "scan" in dom else flops_prep(d)
+    flops = per_unit * spec["split"] * T * Hh
+    ach = flops / (kms / kl / 1e3) / 1e12
+    pk, pu, pdesc = peak_for(spec["bound"], peaks)
+    total = sum(v[0] for v in prof.values())
+    roof = dict(kernel=dom, bound=spec["bound"], achieved=ach, peak=pk, unit=pu, frac=ach / pk, peak_source=pdesc,
+                flops_per_launch=flops, avg_launch_us=kms / kl * 1e3, traffic=TRAFFIC_BY_WORKLOAD.get((name, dom)),
+                kernels={n: dict(avg_us=v[0] / v[1] * 1e3, launches=v[1], share=v[0] / total) for n, v in prof.items()})
+    entry = dict(workload="%s: %s" % (name, WORKLOAD_DESCS[name]), value=job_throughput(T, 1, world, call_ms),
+                 unit=UNIT, us_per_call=call_ms * 1e3, reps=reps, timing=timing, roofline=roof,
+                 method_roofline=method_roofline_of(T, Hh, d, N, w.state_std is not None, call_ms, peaks, es))
+    del inp, out, st, ws
+    return entry
+
+
+def run_case(args, rank, world, local_rank):
+    """--case NAME: only the prefill of one named workload (optionally its first --case-tokens tokens),
+    --warmup + --steps calls, for profiler captures of one kernel on a bounded case."""
+    import torch
+    from linear_attention_10_b200 import gdn
+    from linear_attention_10_b200.workloads import WORKLOADS, make_prefill_inputs
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.case]
+    lengths = list(w.lengths)
+    if args.case_tokens:
+        keep, left = [], args.case_tokens
+        for L in lengths:
+            if left <= 0:
+                break
+            keep.append(min(L, left))
+            left -= keep[-1]
+        lengths = keep
+    inp = make_prefill_inputs(lengths, w.H, w.dk, w.dv, w.dtype, w.gate, w.seed, w.state_std, dev)
+    T, N = sum(lengths), len(lengths)
+    ws = torch.empty(gdn.workspace_bytes(T, N, w.H, w.dk, w.dv), dtype=torch.uint8, device=dev)
+    call = lambda: gdn.gdn_chunk_prefill(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                                         cu_seqlens=inp["cu_seqlens"], state_in=inp["state_in"], workspace=ws)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    if gdn.gdn_get_device_status() != 0:
+        raise RuntimeError("device status error")
+    ms = e0.elapsed_time(e1) / max(args.steps, 1)
+    if rank == 0:
+        print(json.dumps(dict(case=args.case, lengths=lengths, H=w.H, d=w.dk, ms_per_call=ms,
+                              tokens_per_s=T / (ms / 1e3))), flush=True)
 
 
 # ---------------------------------------------------------------------------------------------------
@@ -621,6 +779,14 @@ def run_ours(args, rank, world, local_rank):
                                          traffic=TRAFFIC.get("gdn_decode_verify_kernel (tree, verify_tree_b64_k8)")))
         del vd, vst, vout, par
 
+    # ---- the other prefill workloads of the method ----
+    workloads = None
+    if not args.no_workloads:
+        workloads = {}
+        for wname, reps in (("varlen_resume", 20), ("long_128k", 5), ("tiny_fp32", 100)):
+            workloads[wname] = bench_prefill_workload(wname, reps, world, dev, stream, peaks, rank)
+            torch.cuda.empty_cache()
+
     clk = clocks.stop()
 
     # ---- roofline of the dominant prefill kernel ----
@@ -639,14 +805,7 @@ def run_ours(args, rank, world, local_rank):
                     kernels={n: dict(avg_us=v[0] / v[1] * 1e3, launches=v[1], share=v[0] / total_prof_ms)
                              for n, v in prof.items()})
     # whole-call roofline of the method (TF32 3x split vs HBM), as the metric defines "% of roofline"
-    tf32, _, _ = peak_for("tensor", peaks)
-    t_flop = 3 * flops_whole() * T_PREFILL * H / (tf32 * 1e12)
-    alg_bytes = 3 * T_PREFILL * H * D * 2 + 2 * T_PREFILL * H * 4 + T_PREFILL * H * D * 2 + N * H * D * D * 4
-    t_byte = alg_bytes / (peaks["hbm_gbs"] * 1e9)
-    roof_s = max(t_flop, t_byte)
-    method_roofline = dict(bound="tensor(TF32 x3)" if t_flop >= t_byte else "hbm", roofline_us=roof_s * 1e6,
-                           achieved_us=ms_per_step * 1e3, frac=roof_s / (ms_per_step / 1e3),
-                           tf32_peak_tflops=tf32, hbm_peak_gbs=peaks["hbm_gbs"])
+    method_roofline = method_roofline_of(T_PREFILL, H, D, N, False, ms_per_step, peaks)
 
     cpu = None
     cpu_all = None
@@ -665,7 +824,7 @@ def run_ours(args, rank, world, local_rank):
 
     launches = sum(v[1] for v in prof.values())
     line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
-                ms_per_step=ms_per_step, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="tf32x3",
+                ms_per_step=ms_per_step, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16x3",
                 per_call_ms=dict(median=statistics.median(per_call_ms), min=per_call_ms[0], max=per_call_ms[-1],
                                  calls=len(per_call_ms), timing="an event pair around each whole call"),
                 data="synthetic",
@@ -681,7 +840,7 @@ def run_ours(args, rank, world, local_rank):
                          h2d_alone_ms_per_step=h2d_ms, h2d_gbs=h2d / (h2d_ms / 1e3) / 1e9,
                          bound="the host->device copy of each step's inputs (h2d_alone_ms_per_step)"),
                 gpu_launches=launches, clocks=clk, decode=decode, verify=verify, verify_tree=verify_tree,
-                cuts=cuts_line, norm=norm_line)
+                cuts=cuts_line, norm=norm_line, workloads=workloads)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -746,7 +905,7 @@ def run_sharded(args, rank, world, local_rank):
     value = T_PREFILL * args.steps / (ms / 1e3)
     line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
                 ms_per_step=ms / args.steps, higher_is_better=True, scaling="strong", vs_baseline=None,
-                dtype="tf32x3", data="synthetic",
+                dtype="bf16x3", data="synthetic",
                 config=dict(workload="%s: %s" % (WORKLOAD, WORKLOAD_DESC), global_batch=1, seq_len=T_PREFILL,
                             parallelism="heads sharded over %d GPUs (%d heads on rank 0)%s"
                                         % (world, Hl, ", outputs all-gathered every step" if args.gather else ""),
@@ -767,6 +926,9 @@ def main():
     ap.add_argument("--no-cuts", action="store_true")
     ap.add_argument("--no-norm", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the varlen / 128K / tiny prefill lines")
+    ap.add_argument("--case", default=None, help="profiling aid: run only this workload's prefill")
+    ap.add_argument("--case-tokens", type=int, default=0, help="with --case: keep only the first N tokens")
     ap.add_argument("--no-cpu-all", action="store_true", help="skip the all-cores oracle timing")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--shard", choices=["none", "heads"], default="none",
@@ -778,6 +940,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.case:
+        run_case(args, rank, world, local_rank)
         return
     if world > 1:
         import datetime

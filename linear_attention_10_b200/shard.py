@@ -51,12 +51,21 @@ def shard_heads(tensors: dict, rank: int, world: int, head_dim: int = 1) -> dict
 
 def gather_heads(local, world: int, head_dim: int = 1, group=None):
     """The whole layer's tensor on every rank, from each rank's block of heads along `head_dim`
-    (one all-gather).  The blocks must have equal sizes: H divisible by the world size."""
+    (one all-gather).  The blocks must have equal shapes (H divisible by the world size): the ranks
+    first exchange their block shapes, and every rank raises ValueError when they differ, before
+    the data all-gather, so that no rank is left waiting in a collective with mismatched sizes."""
     import torch
     import torch.distributed as dist
     if world == 1:
         return local
     local = local.contiguous()
+    dev = local.device if dist.get_backend(group) == "nccl" else torch.device("cpu")
+    mine = torch.tensor(list(local.shape), dtype=torch.int64, device=dev)
+    shapes = [torch.empty_like(mine) for _ in range(world)]
+    dist.all_gather(shapes, mine, group=group)
+    if any(not torch.equal(x, shapes[0]) for x in shapes):
+        raise ValueError("gather_heads needs equal head blocks on every rank; got shapes %s (the heads "
+                         "must divide evenly over the %d ranks)" % ([tuple(x.tolist()) for x in shapes], world))
     parts = [torch.empty_like(local) for _ in range(world)]
     dist.all_gather(parts, local, group=group)
     return torch.cat(parts, dim=head_dim)

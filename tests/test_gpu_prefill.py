@@ -10,7 +10,8 @@ import torch
 from linear_attention_10_b200 import gdn
 from linear_attention_10_b200.workloads import WORKLOADS, make_prefill_inputs, workload_inputs
 
-from helpers import TOL, f64, oracle_full, pick_rows, rel_err, sampled_rows_check
+from helpers import (OUT_TOL_BF16_ROUNDING, STATE_TOL_BF16_FP32LEVEL, TOL, f64, full_heads_check, oracle_full,
+                     rel_err, sampled_rows_check)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -193,18 +194,49 @@ def test_prefix_invariance(t):
 
 
 # ---------------------------------------------------------------------------------------------
-# full-size workloads, sampled rows against the oracle
+# full-size workloads against the oracle
 # ---------------------------------------------------------------------------------------------
-@pytest.mark.parametrize("name,count", [("prefill_4k", 48), ("varlen_resume", 48), ("long_128k", 12)])
-def test_full_size_workloads_sampled(name, count):
+def _bf16_fp32_level(name, eo, es):
+    """The bf16 path's extra bars: final states at fp32 level, outputs within bf16 rounding."""
+    print("%s fp32-level bars: s_err=%.3e (<= %g), o_err=%.3e (<= %g)"
+          % (name, es, STATE_TOL_BF16_FP32LEVEL, eo, OUT_TOL_BF16_ROUNDING))
+    assert es <= STATE_TOL_BF16_FP32LEVEL, (name, es)
+    assert eo <= OUT_TOL_BF16_ROUNDING, (name, eo)
+
+
+@pytest.mark.parametrize("name", ["prefill_4k", "varlen_resume"])
+def test_full_size_workloads_every_element(name):
+    """Every output element and every final-state element of the workload against the oracle (all
+    heads, all rows; the oracle runs one head per host thread)."""
+    inp = workload_inputs(name, device=DEV)
+    out, st = run(inp)
+    torch.cuda.synchronize()
+    assert gdn.gdn_get_device_status() == 0
+    eo, es = full_heads_check(inp, out, st)
+    tol = TOL[inp["q"].dtype]
+    print("%s every element: o_err=%.3e s_err=%.3e tol=%g" % (name, eo, es, tol))
+    assert eo <= tol and es <= tol
+    _bf16_fp32_level(name, eo, es)
+
+
+def test_long_128k_full_heads_and_sampled_rows():
+    """T = 131072 (4096 sequential chunks): heads 0 and 21 in full (all 128 state rows, so every
+    dv slice of the scan) and two sampled rows of each of the 32 heads."""
+    name = "long_128k"
     w = WORKLOADS[name]
     inp = workload_inputs(name, device=DEV)
     out, st = run(inp)
     torch.cuda.synchronize()
     assert gdn.gdn_get_device_status() == 0
     assert torch.isfinite(out.float()).all() and torch.isfinite(st).all()
-    picks = pick_rows(len(w.lengths), w.H, w.dv, count, seed=1, lengths=w.lengths)
-    eo, es = sampled_rows_check(inp, out, st, picks)
+    eo, es = full_heads_check(inp, out, st, heads=[0, 21])
     tol = TOL[inp["q"].dtype]
-    print("%s sampled o_err=%.3e s_err=%.3e tol=%g" % (name, eo, es, tol))
+    print("%s heads 0, 21 in full: o_err=%.3e s_err=%.3e tol=%g" % (name, eo, es, tol))
     assert eo <= tol and es <= tol
+    _bf16_fp32_level(name + " full heads", eo, es)
+    rng = np.random.default_rng(7)
+    picks = [(0, h, int(r)) for h in range(w.H) for r in rng.choice(w.dv, 2, replace=False)]
+    so, ss = sampled_rows_check(inp, out, st, picks)
+    print("%s 64 sampled rows over 32 heads: o_err=%.3e s_err=%.3e" % (name, so, ss))
+    assert so <= tol and ss <= tol
+    _bf16_fp32_level(name + " sampled rows", so, ss)

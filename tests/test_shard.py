@@ -82,3 +82,35 @@ def test_two_gloo_ranks_gather_the_whole_layer():
                                      cu_seqlens=inp["cu_seqlens"].numpy(), state_in=f(inp["state_in"]))
     for _, o_all, s_all in res:
         assert np.array_equal(o_all, o_ref) and np.array_equal(s_all, s_ref)
+
+
+def _uneven_rank_main(rank, world, port, q):
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method="tcp://127.0.0.1:%d" % port, rank=rank, world_size=world)
+    try:
+        h0, h1 = head_range(rank, world, 3)          # 2 heads on rank 0, 1 on rank 1
+        local = torch.full((5, h1 - h0, 4), float(rank))
+        try:
+            gather_heads(local, world)
+            q.put((rank, "gathered"))
+        except ValueError as e:
+            q.put((rank, "ValueError: %s" % e))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gather_heads_refuses_unequal_blocks_on_every_rank():
+    """3 heads over 2 ranks: both ranks raise ValueError before the data all-gather (none hangs)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_uneven_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert sorted(res) == [0, 1]
+    for r in (0, 1):
+        assert res[r].startswith("ValueError") and "equal head blocks" in res[r], res[r]
