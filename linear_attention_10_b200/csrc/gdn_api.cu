@@ -41,6 +41,23 @@ static int* status_ptr()
     return cache[dev];
 }
 
+// ---- detail of the last CUDA error met by a library call on this thread (gdn_last_error) ----------
+static thread_local char g_last_err[256] = "";
+
+// Returns e == cudaSuccess; otherwise records "what: <CUDA's message>" for gdn_last_error.
+static bool cuda_ok(cudaError_t e, const char* what)
+{
+    if (e == cudaSuccess) return true;
+    snprintf(g_last_err, sizeof(g_last_err), "%s: %s (%d)", what, cudaGetErrorString(e), (int)e);
+    return false;
+}
+
+template <typename K>
+static bool set_dyn_smem(K kernel, size_t bytes, const char* name)
+{
+    return cuda_ok(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes), name);
+}
+
 // ---- optional per-kernel event timing (gdn_profile_start / gdn_profile_stop) ----------------------
 struct ProfRec {
     const char* name;
@@ -101,7 +118,9 @@ static cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 b
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    cuda_ok(e, "cudaLaunchKernelEx");
+    return e;
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -247,22 +266,21 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         gdn_plan_kernel<<<1, 1024, 0, st>>>(cu, N, T_total, fixed_len, cuts.pos, cuts.n, meta, chunk_off, chunk_tab,
                                             seg, status);
     }
-    if (cudaPeekAtLastError() != cudaSuccess) return GDN_ERR_LAUNCH;
+    if (!cuda_ok(cudaPeekAtLastError(), "gdn_plan_kernel launch")) return GDN_ERR_LAUNCH;
 
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-    CUtensorMap tq{}, tk{}, tv{};
+    CUtensorMap tq{}, tk{};
     if constexpr (kBf16) {
         const uint64_t Tn = (uint64_t)(T_total > 0 ? T_total : 1);
         if (!make_tmap_bf16(&tq, q, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, 128) ||
-            !make_tmap_bf16(&tk, k, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, 128) ||
-            !make_tmap_bf16(&tv, v, (uint64_t)H * DV, Tn, (uint64_t)H * DV, 32, 32, 64))
+            !make_tmap_bf16(&tk, k, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, 128))
             return GDN_ERR_CUDA;
     }
     if constexpr (kBf16) {
       if (lay.nc_max > 0 && T_total > 0) {
         using PL = PrepBf16Smem<DK>;
         auto k1 = gdn_prep_bf16_kernel<DK>;
-        if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PL::kBytes) != cudaSuccess)
+        if (!set_dyn_smem(k1, PL::kBytes, "cudaFuncSetAttribute(max dynamic shared memory)"))
             return GDN_ERR_LAUNCH;
         const int64_t items = lay.nc_max * (int64_t)H;
         const int64_t cap = (int64_t)g_num_sms * kPrepBf16CtasPerSm;
@@ -275,7 +293,7 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
     } else if (lay.nc_max > 0 && T_total > 0) {
         using PL = PrepSmem<T, DK>;
         auto k1 = gdn_prep_kernel<T, DK>;
-        if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PL::kBytes) != cudaSuccess)
+        if (!set_dyn_smem(k1, PL::kBytes, "cudaFuncSetAttribute(max dynamic shared memory)"))
             return GDN_ERR_LAUNCH;
         const int64_t items = lay.nc_max * (int64_t)H;
         const int64_t cap = (int64_t)g_num_sms * 4;
@@ -288,22 +306,20 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
     }
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         // bf16 inputs: operands staged by tensor maps, bf16 tensor-core products for K and Q
-        constexpr int MSB = 32;
-        using SB3 = ScanBf16Smem<DK, MSB, 3>;
-        using SB4 = ScanBf16Smem<DK, MSB, 4>;
+        using SB4 = ScanBf16Smem<DK, 4>;
+        using SB3 = ScanBf16Smem<DK, 3>;
         constexpr int ST = (SB4::kBytes <= 227 * 1024) ? 4 : 3;
-        using SB = ScanBf16Smem<DK, MSB, ST>;
+        using SB = ScanBf16Smem<DK, ST>;
         static_assert(SB3::kBytes <= 227 * 1024, "bf16 scan shared memory");
-        static_assert(MSB == 32, "the V tensor map boxes 32 columns");
-        auto kb = cuts.n > 0 ? gdn_scan_bf16_kernel<DK, DV, MSB, ST, true> : gdn_scan_bf16_kernel<DK, DV, MSB, ST, false>;
-        if (cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SB::kBytes) != cudaSuccess)
+        auto kb = cuts.n > 0 ? gdn_scan_bf16_kernel<DK, DV, ST, true> : gdn_scan_bf16_kernel<DK, DV, ST, false>;
+        if (!set_dyn_smem(kb, SB::kBytes, "cudaFuncSetAttribute(max dynamic shared memory)"))
             return GDN_ERR_LAUNCH;
         {
             ProfScope prof("gdn_scan_bf16_kernel", st);
-            if (launch_dependent(kb, dim3((unsigned)N, H, DV / MSB), dim3(kScanBf16Threads), SB::kBytes, st, tq, tk,
-                                 tv, (const int*)meta, (const int*)chunk_off, (const int4*)chunk_tab,
-                                 reinterpret_cast<const uint8_t*>(op), state_in, static_cast<__nv_bfloat16*>(out),
-                                 state_out, cuts.snaps, H, status) != cudaSuccess)
+            if (launch_dependent(kb, dim3((unsigned)N, H, DV / 32), dim3(kScanBf16Threads), SB::kBytes, st, tq, tk,
+                                 static_cast<const __nv_bfloat16*>(v), (const int*)meta, (const int*)chunk_off,
+                                 (const int4*)chunk_tab, reinterpret_cast<const uint8_t*>(op), state_in,
+                                 static_cast<__nv_bfloat16*>(out), state_out, cuts.snaps, H, status) != cudaSuccess)
                 return GDN_ERR_LAUNCH;
         }
         return GDN_OK;
@@ -317,7 +333,7 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
     using SL = ScanSmem<T, DK, MS, STAGES>;
     static_assert((SL::kBytes + 1024) * MINB <= 228 * 1024, "scan kernel shared memory");
     auto k2 = gdn_scan_tc_kernel<T, DK, DV, MS, STAGES, MINB>;
-    if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SL::kBytes) != cudaSuccess)
+    if (!set_dyn_smem(k2, SL::kBytes, "cudaFuncSetAttribute(max dynamic shared memory)"))
         return GDN_ERR_LAUNCH;
     {
         ProfScope prof("gdn_scan_tc_kernel", st);
@@ -472,6 +488,8 @@ const char* gdn_status_string(int s)
 }
 
 int gdn_version(void) { return 100; }
+
+const char* gdn_last_error(void) { return g_last_err; }
 
 size_t gdn_chunk_prefill_workspace_bytes(int64_t total_tokens, int num_seqs, int H, int dk, int dv)
 {

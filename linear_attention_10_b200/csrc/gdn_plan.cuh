@@ -12,6 +12,7 @@
 #pragma once
 
 #include "gdn_common.cuh"
+#include "gdn_prefill_tc.cuh"
 #include "gdn_sm100.cuh"
 
 namespace gdn {
@@ -24,7 +25,7 @@ struct PrefillLayout {
     size_t off_chunk_off; // int32[NS + 1]: first global chunk of each sequence
     size_t off_chunk_tab; // int4[nc_max]: (sequence, first token, rows, snapshot index or -1)
     size_t off_seg;       // int32[6 NS + 1]: segment start, sequence, cut, end, snapshot, chunk offset
-    size_t off_op;        // [nc_max][H] operator records (up to 25088 bytes each)
+    size_t off_op;        // [nc_max][H] operator records (kOpBytesMax bytes each)
     size_t total;
 
     static size_t align(size_t x) { return (x + 255) & ~size_t(255); }
@@ -37,7 +38,7 @@ struct PrefillLayout {
         off_chunk_off = o; o = align(o + (size_t)(NS + 1) * sizeof(int));
         off_chunk_tab = o; o = align(o + (size_t)nc_max * sizeof(int4));
         off_seg = o;       o = align(o + (size_t)(6 * NS + 1) * sizeof(int));
-        off_op = o;        o = align(o + (size_t)nc_max * H * 25088);   // largest record of the two paths
+        off_op = o;        o = align(o + (size_t)nc_max * H * kOpBytesMax);   // larger record of the two paths
         total = o;
         (void)dk;
     }

@@ -23,6 +23,7 @@ CHUNK = 32
 # symbols declared in include/gdn.h
 EXPORTS = (
     "gdn_status_string",
+    "gdn_last_error",
     "gdn_version",
     "gdn_chunk_prefill_workspace_bytes",
     "gdn_chunk_prefill_workspace_bytes_ex",
@@ -44,7 +45,14 @@ _lib = None
 class GdnError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
-        super().__init__("%s failed: %s (%d)" % (what, status_string(code), code))
+        detail = ""
+        try:
+            d = lib().gdn_last_error()
+            if d:
+                detail = " [%s]" % d.decode()
+        except Exception:  # pragma: no cover
+            pass
+        super().__init__("%s failed: %s (%d)%s" % (what, status_string(code), code, detail))
 
 
 def lib() -> ctypes.CDLL:
@@ -61,6 +69,8 @@ def lib() -> ctypes.CDLL:
     L.gdn_status_string.restype = ctypes.c_char_p
     L.gdn_version.argtypes = []
     L.gdn_version.restype = i32
+    L.gdn_last_error.argtypes = []
+    L.gdn_last_error.restype = ctypes.c_char_p
     L.gdn_chunk_prefill_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
     L.gdn_chunk_prefill_workspace_bytes.restype = sz
     L.gdn_chunk_prefill_workspace_bytes_ex.argtypes = [i64, i32, i32, i32, i32, i32]
