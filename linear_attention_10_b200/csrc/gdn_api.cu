@@ -255,6 +255,7 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
     int4* chunk_tab = reinterpret_cast<int4*>(ws + lay.off_chunk_tab);
     float* op = reinterpret_cast<float*>(ws + lay.off_op);
     int* seg = reinterpret_cast<int*>(ws + lay.off_seg);
+    int* order = reinterpret_cast<int*>(ws + lay.off_order);
     if (g_num_sms == 0) {
         int dev = 0;
         cudaGetDevice(&dev);
@@ -264,16 +265,17 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
     {
         ProfScope prof("gdn_plan_kernel", st);
         gdn_plan_kernel<<<1, 1024, 0, st>>>(cu, N, T_total, fixed_len, cuts.pos, cuts.n, meta, chunk_off, chunk_tab,
-                                            seg, status);
+                                            seg, order, status);
     }
     if (!cuda_ok(cudaPeekAtLastError(), "gdn_plan_kernel launch")) return GDN_ERR_LAUNCH;
 
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-    CUtensorMap tq{}, tk{};
+    CUtensorMap tq{}, tk{}, tv{};
     if constexpr (kBf16) {
         const uint64_t Tn = (uint64_t)(T_total > 0 ? T_total : 1);
         if (!make_tmap_bf16(&tq, q, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, 128) ||
-            !make_tmap_bf16(&tk, k, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, 128))
+            !make_tmap_bf16(&tk, k, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, 128) ||
+            !make_tmap_bf16(&tv, v, (uint64_t)H * DV, Tn, (uint64_t)H * DV, 32, 32, 64))
             return GDN_ERR_CUDA;
     }
     if constexpr (kBf16) {
@@ -306,20 +308,25 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
     }
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
         // bf16 inputs: operands staged by tensor maps, bf16 tensor-core products for K and Q
-        using SB4 = ScanBf16Smem<DK, 4>;
-        using SB3 = ScanBf16Smem<DK, 3>;
+        constexpr int MSB = 32;
+        using SB3 = ScanBf16Smem<DK, MSB, 3>;
+        using SB4 = ScanBf16Smem<DK, MSB, 4>;
         constexpr int ST = (SB4::kBytes <= 227 * 1024) ? 4 : 3;
-        using SB = ScanBf16Smem<DK, ST>;
+        using SB = ScanBf16Smem<DK, MSB, ST>;
         static_assert(SB3::kBytes <= 227 * 1024, "bf16 scan shared memory");
-        auto kb = cuts.n > 0 ? gdn_scan_bf16_kernel<DK, DV, ST, true> : gdn_scan_bf16_kernel<DK, DV, ST, false>;
+        static_assert(MSB == 32, "the V tensor map boxes 32 columns");
+        auto kb = cuts.n > 0 ? gdn_scan_bf16_kernel<DK, DV, MSB, ST, true> : gdn_scan_bf16_kernel<DK, DV, MSB, ST, false>;
         if (!set_dyn_smem(kb, SB::kBytes, "cudaFuncSetAttribute(max dynamic shared memory)"))
             return GDN_ERR_LAUNCH;
         {
             ProfScope prof("gdn_scan_bf16_kernel", st);
-            if (launch_dependent(kb, dim3((unsigned)N, H, DV / 32), dim3(kScanBf16Threads), SB::kBytes, st, tq, tk,
-                                 static_cast<const __nv_bfloat16*>(v), (const int*)meta, (const int*)chunk_off,
-                                 (const int4*)chunk_tab, reinterpret_cast<const uint8_t*>(op), state_in,
-                                 static_cast<__nv_bfloat16*>(out), state_out, cuts.snaps, H, status) != cudaSuccess)
+            // one CTA per (32 state rows, head, sequence), the sequence's rank in `order` slowest
+            const int64_t ctas = (int64_t)(DV / MSB) * H * N;
+            if (ctas > INT32_MAX) return GDN_ERR_INVALID_ARG;
+            if (launch_dependent(kb, dim3((unsigned)ctas), dim3(kScanBf16Threads), SB::kBytes, st, tq, tk,
+                                 tv, (const int*)meta, (const int*)order, (const int*)chunk_off, (const int4*)chunk_tab,
+                                 reinterpret_cast<const uint8_t*>(op), state_in, static_cast<__nv_bfloat16*>(out),
+                                 state_out, cuts.snaps, H, status) != cudaSuccess)
                 return GDN_ERR_LAUNCH;
         }
         return GDN_OK;

@@ -12,7 +12,6 @@
 #pragma once
 
 #include "gdn_common.cuh"
-#include "gdn_prefill_tc.cuh"
 #include "gdn_sm100.cuh"
 
 namespace gdn {
@@ -25,7 +24,8 @@ struct PrefillLayout {
     size_t off_chunk_off; // int32[NS + 1]: first global chunk of each sequence
     size_t off_chunk_tab; // int4[nc_max]: (sequence, first token, rows, snapshot index or -1)
     size_t off_seg;       // int32[6 NS + 1]: segment start, sequence, cut, end, snapshot, chunk offset
-    size_t off_op;        // [nc_max][H] operator records (kOpBytesMax bytes each)
+    size_t off_order;     // int32[NS]: the sequences in the order the bf16 scan takes them
+    size_t off_op;        // [nc_max][H] operator records (up to 25088 bytes each)
     size_t total;
 
     static size_t align(size_t x) { return (x + 255) & ~size_t(255); }
@@ -38,7 +38,8 @@ struct PrefillLayout {
         off_chunk_off = o; o = align(o + (size_t)(NS + 1) * sizeof(int));
         off_chunk_tab = o; o = align(o + (size_t)nc_max * sizeof(int4));
         off_seg = o;       o = align(o + (size_t)(6 * NS + 1) * sizeof(int));
-        off_op = o;        o = align(o + (size_t)nc_max * H * kOpBytesMax);   // larger record of the two paths
+        off_order = o;     o = align(o + (size_t)NS * sizeof(int));
+        off_op = o;        o = align(o + (size_t)nc_max * H * 25088);   // largest record of the two paths
         total = o;
         (void)dk;
     }
@@ -85,11 +86,37 @@ __device__ __forceinline__ int count_less(const int32_t* a, int n, int64_t x, bo
 // <<<1, 1024>>>.  cu_seqlens may be null: N sequences of equal length `fixed_len`.  cuts: n_cuts
 // token offsets, strictly increasing, each strictly inside one sequence (may be null when n_cuts
 // is 0).  seg: the workspace's segment arrays, 6 (N + n_cuts) + 1 ints.
+// The order in which the bf16 scan takes the sequences of a packed call: most chunks first (ties by
+// index).  The scan's CTAs are numbered with the sequence's rank slowest, so the longest sequences'
+// CTAs start first and shorter ones fill the SMs behind them; a packed call then ends close to
+// max(longest sequence, total chunks / SMs) instead of whenever its longest sequence happened to
+// start.  Ranks are counted in one pass per sequence (sequences <= 1024), identity order beyond.
+__device__ __forceinline__ void plan_order(int N, const int* chunk_off, int* order, int* s_cnt)
+{
+    if (N > 1024) {
+        for (int n = threadIdx.x; n < N; n += 1024) order[n] = n;
+        return;
+    }
+    const int n = threadIdx.x;
+    if (n < N) s_cnt[n] = chunk_off[n + 1] - chunk_off[n];
+    __syncthreads();
+    if (n < N) {
+        const int cn = s_cnt[n];
+        int r = 0;
+        for (int m = 0; m < N; ++m) {
+            const int cm = s_cnt[m];
+            r += (cm > cn) || (cm == cn && m < n);
+        }
+        order[r] = n;
+    }
+}
+
 __global__ void __launch_bounds__(1024) gdn_plan_kernel(const int32_t* __restrict__ cu, int N, int64_t T,
                                                     int fixed_len, const int32_t* __restrict__ cuts, int n_cuts,
                                                     int* meta, int* chunk_off, int4* chunk_tab, int* seg,
-                                                    int* status)
+                                                    int* order, int* status)
 {
+    __shared__ int s_cnt[1024];
     __shared__ int warp_tot[32];
     __shared__ int s_err;
     __shared__ int s_running;
@@ -143,6 +170,7 @@ __global__ void __launch_bounds__(1024) gdn_plan_kernel(const int32_t* __restric
             const int64_t e = start_of(lo + 1);
             chunk_tab[gc] = make_int4(lo, (int)t0, (int)((e - t0) < kChunk ? (e - t0) : kChunk), -1);
         }
+        plan_order(N, chunk_off, order, s_cnt);
         return;
     }
 
@@ -247,6 +275,7 @@ __global__ void __launch_bounds__(1024) gdn_plan_kernel(const int32_t* __restric
         const int snap = (t0 + rows == seg_end[j]) ? seg_snap[j] : -1;
         chunk_tab[gc] = make_int4(seg_seq[j], t0, rows, snap);
     }
+    plan_order(N, chunk_off, order, s_cnt);
 }
 
 }  // namespace gdn

@@ -49,21 +49,14 @@ constexpr uint32_t kOpLo = 8192;
 constexpr uint32_t kOpGate = 16384;
 constexpr uint32_t kOpCopyBytes = 16384 + 80 * 4;   // staged per chunk (operator + gates)
 constexpr uint32_t kOpBytes = 16384 + 512;          // record stride in the workspace
-// bf16-input path record (22,848 bytes): the tensor-core operands of the scan, which it copies into
-// shared memory in one piece -- three bf16 parts of [T''; P T''] (64 x 32 each, K-major, 64-byte
-// swizzle) and three of R (32 x 32 each, same layout) -- then M (32 x 32 fp32, row-major) and the
-// gates.  With G'_K, G'_Q the chunk's K and Q rows against the previous chunk's keys,
-//   M = diag(delta) T'' diag(Gamma) G'_K,   R = diag(Gamma) G'_Q - P T'' diag(Gamma) G'_K
-// (both zero for a chunk that starts its sequence).
+// bf16-input path record: three bf16 parts (each 64 x 32, K-major, 64-byte swizzle) of
+// [T''; P T''], then three of the cross-chunk Gram matrix G' = [K; Q] K_prev^T (the chunk's rows
+// against the previous chunk's keys in the same sequence), then the gates.
 constexpr uint32_t kOpBPart = 4096;
-constexpr uint32_t kOpBR = 3 * kOpBPart;
-constexpr uint32_t kOpBRPart = 2048;
-constexpr uint32_t kOpBTcBytes = kOpBR + 3 * kOpBRPart;     // staged by the scan (18,432 bytes)
-constexpr uint32_t kOpBM = kOpBTcBytes;
-constexpr uint32_t kOpBGate = kOpBM + 32 * 32 * 4;
-constexpr uint32_t kOpBytesB = kOpBGate + 80 * 4;
-// the workspace reserves the larger of the two record sizes per (chunk, head)
-constexpr uint32_t kOpBytesMax = kOpBytesB > kOpBytes ? kOpBytesB : kOpBytes;
+constexpr uint32_t kOpBCross = 3 * kOpBPart;
+constexpr uint32_t kOpBGate = 6 * kOpBPart;
+constexpr uint32_t kOpBCopyBytes = 6 * kOpBPart + 80 * 4;
+constexpr uint32_t kOpBytesB = 25088;
 
 template <typename T>
 struct ExactTF32 { static constexpr bool value = false; };

@@ -1,35 +1,29 @@
 // gdn_prep_bf16.cuh -- per-(chunk, head) WY/UT operator for bf16 q/k (sm_100a).
 //
-// Builds the operator record the bf16 scan reads, for one chunk of 32 rows of one head, where
+// Builds the operator record the bf16 scan reads, for one chunk of 32 rows of one head: [T''; P T'']
+// and the cross-chunk Gram G' = [K; Q] K_prev^T, each as three bf16 parts in the 64-byte-swizzled
+// K-major layout of a tensor-core A operand, and the gates Gamma_i, delta_i, Gamma_C, where
 // (chunk-local cumulative log-gate gamma)
 //
 //   A = strictly-lower(diag(beta) (D o K K^T)),  P = lower-incl-diagonal(D o Q K^T),
-//   D_ij = exp(gamma_i - gamma_j),  T = (I + A)^-1,  T'' = T diag(beta),
-//
-// and, with G'_K = K K_prev^T and G'_Q = Q K_prev^T the chunk's rows against the previous chunk's
-// keys in the same sequence (H = diag(Gamma) G'_K),
-//
-//   M = diag(delta) T'' H,   R = diag(Gamma) G'_Q - P T'' H.
-//
-// The record holds [T''; P T''] and R as three bf16 parts each in the 64-byte-swizzled K-major
-// layout of a tensor-core A operand, M in fp32 and the gates Gamma_i, delta_i, Gamma_C.
+//   D_ij = exp(gamma_i - gamma_j),  T = (I + A)^-1,  T'' = T diag(beta).
 //
 // What is specific to bf16 inputs: the chunk's [K; Q] rows are exact bf16 values, so the tensor-
 // memory-access engine copies them straight into the 128-byte-swizzled operand layout (the next
-// item's rows arrive while this one is gated, solved and written out) and one bf16 tensor-core
-// product (M = 128, N = 32, K = dk) forms both Gram matrices exactly in fp32.  The gates are applied
-// while the Gram rows come out of tensor memory.  The inverse uses the 2 x 2 block form with 16 x 16
-// blocks,
+// item's rows arrive while this one is gated, solved and written out, five CTAs per SM) and one
+// bf16 tensor-core product (M = 128, N = 32, K = dk) forms both Gram
+// matrices exactly in fp32.  The gates are applied while the Gram rows come out of tensor memory.
+// The inverse uses the 2 x 2 block form with 16 x 16 blocks,
 //
 //   T11 = (I + A11)^-1,  T22 = (I + A22)^-1  (forward substitution, in parallel),
 //   T21 = -T22 (A21 T11),
 //
 // which shortens the dependent chain of the substitution from 31 steps to 15.
 //
-// The cross-chunk Gram G' = [K; Q] K_prev^T is issued by a second thread with the A descriptor
-// started 64 rows before the tile, so its rows land in tensor-memory lanes 64..127 and stay there
-// until the item's last phase: warps 2 and 3, which only those lanes are visible to, read them out
-// once T'' and P T'' exist, and all four warps form [T''; P T''] H on the CUDA cores.
+// The cross-chunk Gram G' = [K; Q] K_prev^T (the scan's MMA_x operand) is issued by a second thread
+// with the A descriptor started 64 rows before the tile, so its rows land in tensor-memory lanes
+// 64..127: warps 2 and 3, which only those lanes are visible to, split and store it while warps 0
+// and 1 gate the chunk's own Gram rows in lanes 0..63.
 #pragma once
 
 #include <cuda.h>
@@ -56,9 +50,7 @@ struct PrepBf16Smem {
     static constexpr uint32_t oT = oP + 32 * LD * 4;                  // [32][LD] T
     static constexpr int LM = 16;                                     // pitch of M (2-way write conflicts)
     static constexpr uint32_t oM = oT + 32 * LD * 4;                  // [16][LM] A21 T11
-    // last phase: T'' (fp32) over A, P T'' in its own rows, H over P, Gamma G'_Q over T
-    static constexpr uint32_t oYB = oM + 16 * LM * 4;                 // [32][LD] P T''
-    static constexpr uint32_t oGam = oYB + 32 * LD * 4;
+    static constexpr uint32_t oGam = oM + 16 * LM * 4;
     static constexpr uint32_t oBet = oGam + 128;
     static constexpr uint32_t oAlph = oBet + 128;                     // per-token decays exp(g), one spare
     static constexpr uint32_t oBar = oAlph + 136;   // tile_full, (spare), mma, drain[2], prev_full, cross
@@ -258,7 +250,7 @@ __global__ void __launch_bounds__(128, kPrepBf16CtasPerSm) gdn_prep_bf16_kernel(
         } else {
             // warps 2 and 3: the tile buffer is free once G' has been formed (the chunk's own Gram
             // was waited for before the barrier above): fetch the next item's [K; Q] rows and
-            // previous-chunk keys (G' itself stays in tensor memory until the last phase)
+            // previous-chunk keys, then split G'
             if (tid == 64 && !mbar_wait(cross_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
             named_bar(1, 64);
             tc_fence_after();
@@ -266,6 +258,26 @@ __global__ void __launch_bounds__(128, kPrepBf16CtasPerSm) gdn_prep_bf16_kernel(
                 if (item + (int)gridDim.x < nitems) {
                     issue_tile(item + gridDim.x);
                     issue_prev(item + gridDim.x);
+                }
+            }
+            if (prev) {
+                // row (32 (w - 2) + lane) of G', in lane 32 w + lane -> three bf16 parts, K-major
+                // 64-byte-swizzled A operand rows
+                float e[32];
+                tmem_ld32(tmem + 32 + ((uint32_t)(warp * 32) << 16), e);
+                tmem_ld_wait();
+                uint8_t* rec = op + ((size_t)gc * H + h) * kOpBytesB + kOpBCross;
+                const int row = (warp - 2) * 32 + lane;
+#pragma unroll
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    uint32_t w1[4], w2[4], w3[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        bf16x2_split3(e[c8 * 8 + 2 * q], e[c8 * 8 + 2 * q + 1], w1[q], w2[q], w3[q]);
+                    const uint32_t o = sw64_off_h(row, c8 * 8);
+                    stg128(rec + o, w1);
+                    stg128(rec + kOpBPart + o, w2);
+                    stg128(rec + 2 * kOpBPart + o, w3);
                 }
             }
         }
@@ -333,11 +345,8 @@ __global__ void __launch_bounds__(128, kPrepBf16CtasPerSm) gdn_prep_bf16_kernel(
         // operator record: thread (a, cb) forms columns 4 cb .. 4 cb + 3 of rows 2a and 2a + 1 of
         // T'' = T diag(beta) and of P T'' = (P T) diag(beta) (a 2 x 4 block: each T row it loads
         // serves both rows), and writes each as three bf16 parts of 8 bytes per row into the
-        // 64-byte-swizzled A-operand image (rows 0..31: T'', rows 32..63: P T''), and in fp32 into
-        // shared memory for the last phase (T'' over A, which the solve no longer needs)
+        // 64-byte-swizzled A-operand image (rows 0..31: T'', rows 32..63: P T'')
         uint8_t* dst = op + ((size_t)gc * H + h) * kOpBytesB;
-        float* YT = G;
-        float* YB = reinterpret_cast<float*>(sm + L::oYB);
         {
             const int i0 = (tid >> 3) * 2, c0 = (tid & 7) * 4;
             const float4 bv4 = *reinterpret_cast<const float4*>(bet + c0);
@@ -366,29 +375,16 @@ __global__ void __launch_bounds__(128, kPrepBf16CtasPerSm) gdn_prep_bf16_kernel(
                     acc[1][3] = fmaf(pb[e], t.w, acc[1][3]);
                 }
             }
-            float tpp[2][4], ptpp[2][4];
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                const float4 tv4 = *reinterpret_cast<const float4*>(Tm + (i0 + rr) * LD + c0);
-                const float tv[4] = {tv4.x, tv4.y, tv4.z, tv4.w};
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tpp[rr][c] = tv[c] * bc[c];
-                    ptpp[rr][c] = acc[rr][c] * bc[c];
-                }
-            }
-            // every thread has read its T rows: T'' may now overwrite A (no reader left)
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
                 const int i = i0 + rr;
-                *reinterpret_cast<float4*>(YT + i * LD + c0) = make_float4(tpp[rr][0], tpp[rr][1], tpp[rr][2], tpp[rr][3]);
-                *reinterpret_cast<float4*>(YB + i * LD + c0) =
-                    make_float4(ptpp[rr][0], ptpp[rr][1], ptpp[rr][2], ptpp[rr][3]);
+                const float4 tv4 = *reinterpret_cast<const float4*>(Tm + i * LD + c0);
+                const float tv[4] = {tv4.x, tv4.y, tv4.z, tv4.w};
                 uint32_t w1[2], w2[2], w3[2], x1[2], x2[2], x3[2];
 #pragma unroll
                 for (int c = 0; c < 4; c += 2) {
-                    bf16x2_split3(tpp[rr][c], tpp[rr][c + 1], w1[c / 2], w2[c / 2], w3[c / 2]);
-                    bf16x2_split3(ptpp[rr][c], ptpp[rr][c + 1], x1[c / 2], x2[c / 2], x3[c / 2]);
+                    bf16x2_split3(tv[c] * bc[c], tv[c + 1] * bc[c + 1], w1[c / 2], w2[c / 2], w3[c / 2]);
+                    bf16x2_split3(acc[rr][c] * bc[c], acc[rr][c + 1] * bc[c + 1], x1[c / 2], x2[c / 2], x3[c / 2]);
                 }
                 const uint32_t ot = sw64_off_h(i, c0), op2 = sw64_off_h(32 + i, c0);
                 stg64(dst + ot, w1);
@@ -411,91 +407,6 @@ __global__ void __launch_bounds__(128, kPrepBf16CtasPerSm) gdn_prep_bf16_kernel(
         (void)Lr;
         __syncthreads();
         GDN_PREP_TRACE(iter, 4);
-
-        // last phase: M = diag(delta) T'' H and R = diag(Gamma) G'_Q - P T'' H with H = diag(Gamma)
-        // G'_K.  Warp 2 writes H (over P), warp 3 Gamma G'_Q (over T), from the G' rows still in
-        // tensor memory (zero for a chunk that starts its sequence).
-        float* Hs = P;
-        float* GQs = Tm;
-        if (warp >= 2) {
-            const int i = lane;
-            const float Gi = exp2f(gam[i]);
-            float e[32];
-            if (prev) {
-                tc_fence_after();
-                tmem_ld32(tmem + 32 + ((uint32_t)(warp * 32) << 16), e);
-                tmem_ld_wait();
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) e[j] = 0.f;
-            }
-            float* rowp = (warp == 2 ? Hs : GQs) + i * LD;
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                *reinterpret_cast<float4*>(rowp + 4 * q) =
-                    make_float4(Gi * e[4 * q], Gi * e[4 * q + 1], Gi * e[4 * q + 2], Gi * e[4 * q + 3]);
-        }
-        tc_fence_before();
-        __syncthreads();
-        {
-            // thread (rp, cb): rows 2 rp, 2 rp + 1 of [T''; P T''] H, columns 8 cb .. 8 cb + 7
-            const int rp = tid >> 2, cb = tid & 3;
-            const int r0 = 2 * rp;
-            const float* A0 = (r0 < 32) ? (YT + r0 * LD) : (YB + (r0 - 32) * LD);
-            const float* A1 = A0 + LD;
-            float y[2][8];
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr)
-#pragma unroll
-                for (int c = 0; c < 8; ++c) y[rr][c] = 0.f;
-#pragma unroll
-            for (int k4 = 0; k4 < 8; ++k4) {
-                const float4 a0 = *reinterpret_cast<const float4*>(A0 + 4 * k4);
-                const float4 a1 = *reinterpret_cast<const float4*>(A1 + 4 * k4);
-                const float av0[4] = {a0.x, a0.y, a0.z, a0.w}, av1[4] = {a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float* hr = Hs + (4 * k4 + e) * LD + 8 * cb;
-                    const float4 h0 = *reinterpret_cast<const float4*>(hr);
-                    const float4 h1 = *reinterpret_cast<const float4*>(hr + 4);
-                    const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        y[0][c] = fmaf(av0[e], hv[c], y[0][c]);
-                        y[1][c] = fmaf(av1[e], hv[c], y[1][c]);
-                    }
-                }
-            }
-            if (r0 < 32) {
-                // M rows, fp32, row-major
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const int i = r0 + rr;
-                    const float dl = exp2f(gam[31] - gam[i]);
-                    float* mrow = reinterpret_cast<float*>(dst + kOpBM) + i * 32 + 8 * cb;
-                    *reinterpret_cast<float4*>(mrow) = make_float4(dl * y[rr][0], dl * y[rr][1], dl * y[rr][2], dl * y[rr][3]);
-                    *reinterpret_cast<float4*>(mrow + 4) =
-                        make_float4(dl * y[rr][4], dl * y[rr][5], dl * y[rr][6], dl * y[rr][7]);
-                }
-            } else {
-                // R rows as three bf16 parts, K-major 64-byte-swizzled A-operand rows
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const int i = r0 - 32 + rr;
-                    const float* gq = GQs + i * LD + 8 * cb;
-                    uint32_t w1[4], w2[4], w3[4];
-#pragma unroll
-                    for (int c = 0; c < 8; c += 2)
-                        bf16x2_split3(gq[c] - y[rr][c], gq[c + 1] - y[rr][c + 1], w1[c / 2], w2[c / 2], w3[c / 2]);
-                    const uint32_t o = sw64_off_h(i, 8 * cb);
-                    stg128(dst + kOpBR + o, w1);
-                    stg128(dst + kOpBR + kOpBRPart + o, w2);
-                    stg128(dst + kOpBR + 2 * kOpBRPart + o, w3);
-                }
-            }
-        }
-        __syncthreads();
-        GDN_PREP_TRACE(iter, 7);
     }
     tc_fence_before();
     __syncthreads();

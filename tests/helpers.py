@@ -118,61 +118,3 @@ def full_heads_check(inp, out, state_out, heads=None):
     s_got = np.stack([f64(state_out[:, h]) for h in hs], axis=1)
     return rel_err(o_got, o_ref), rel_err(s_got, s_ref)
 
-
-def chain_form_operators(op):
-    """The two per-chunk operators of the chain form of the chunked scan, from one chunk's WY/UT
-    quantities (``oracle.chunk_operator`` with the previous chunk's keys):
-
-      M = diag(delta) T'' diag(Gamma) G'_K,      R = diag(Gamma) G'_Q - P T'' diag(Gamma) G'_K,
-
-    with G'_K, G'_Q the K and Q rows of G' = [K; Q] K_prev^T.  With them a chunk's compressed writes
-    U~_c = diag(delta) U_c and outputs follow from the previous chunk's U~ and a state two chunks
-    back (see ``chain_form_prefill``).  Returns (M, R), each C x C."""
-    C = op["Tpp"].shape[0]
-    GK, GQ = op["Gp"][:C], op["Gp"][C:]
-    H = op["Gamma"][:, None] * GK
-    M = op["delta"][:, None] * (op["Tpp"] @ H)
-    R = op["Gamma"][:, None] * GQ - op["PTpp"] @ H
-    return M, R
-
-
-def chain_form_prefill(q, k, v, g, beta, state, chunk=32, mistake=None):
-    """One head of one sequence evaluated in the chain form that the CUDA scan uses, in fp64, from the
-    oracle's per-chunk quantities.  With S_c the state after chunk c (S_-1 the initial state,
-    S_-2 := S_-1), Gamma_-1 := 1 and U~_-1 := 0:
-
-      W_c  = [K; Q]_c S_{c-2}^T                      (W_K, W_Q: its K and Q rows)
-      E_c  = V_c - Gamma_{c-1} diag(Gamma) W_K
-      D_c  = diag(delta) T'' E_c,   U~_c = D_c - M_c U~_{c-1}
-      O_c  = s (Gamma_{c-1} diag(Gamma) W_Q + P T'' E_c + R_c U~_{c-1})
-      S_c  = Gamma_C S_{c-1} + U~_c^T K_c
-
-    ``mistake`` plants one error for the tests that must catch it.  Returns (o [T, dv], S_final)."""
-    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
-    g, beta = np.asarray(g, dtype=np.float64), np.asarray(beta, dtype=np.float64)
-    T, dk = q.shape
-    dv = v.shape[1]
-    s = 1.0 / np.sqrt(dk)
-    S_prev2 = S_prev = np.asarray(state, dtype=np.float64)
-    Ut_prev = np.zeros((chunk, dv))
-    gam_prev = 1.0
-    out = np.zeros((T, dv))
-    for c, t0 in enumerate(range(0, T, chunk)):
-        L = min(chunk, T - t0)
-        rows = slice(t0, t0 + L)
-        kp = None if c == 0 else k[t0 - chunk:t0]
-        op = oracle.chunk_operator(q[rows], k[rows], g[rows], beta[rows], k_prev=kp)
-        M, R = chain_form_operators(op)
-        Qc, Kc, Vc = (np.zeros((chunk, x.shape[1])) for x in (q, k, v))
-        Qc[:L], Kc[:L], Vc[:L] = q[rows], k[rows], v[rows]
-        WK, WQ = Kc @ S_prev2.T, Qc @ S_prev2.T
-        gp = op["GammaC"] if mistake == "gate_of_this_chunk" else gam_prev
-        E = Vc - gp * op["Gamma"][:, None] * WK
-        D = op["delta"][:, None] * (op["Tpp"] @ E)
-        Ut = D - M @ Ut_prev
-        Rterm = 0.0 if mistake == "no_R" else R @ Ut_prev
-        O = s * (gam_prev * op["Gamma"][:, None] * WQ + op["PTpp"] @ E + Rterm)
-        out[rows] = O[:L]
-        S_new = op["GammaC"] * S_prev + Ut.T @ Kc
-        S_prev2, S_prev, Ut_prev, gam_prev = S_prev, S_new, Ut, op["GammaC"]
-    return out, S_prev

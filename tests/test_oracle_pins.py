@@ -532,19 +532,3 @@ def test_planted_mistakes_are_caught(mistake):
     ok_proj = np.max(np.abs(sv[0, 0] @ k2[-1, 0] - v2[-1, 0])) < 1e-12
     assert not (ok_hand and ok_proj), "planted mistake %r passed the pins" % mistake
 
-
-def test_chain_form_of_the_scan_reproduces_the_recurrence():
-    """The chain form the CUDA scan evaluates (per chunk: U~_c = D_c - M_c U~_{c-1} with everything
-    else a chunk or more off the chain) gives the recurrence's outputs and final state, over six
-    chunks with a ragged last chunk; two planted mistakes in it are caught."""
-    from helpers import chain_form_prefill
-    d, L = 16, 5 * 32 + 11
-    q, k, v, g, b = _one_head(L, d, 91)
-    S0 = 0.05 * np.random.default_rng(92).standard_normal((d, d))
-    o_ref, s_ref = oracle.recurrence(q[:, None], k[:, None], v[:, None], g[:, None], b[:, None],
-                                     state_in=S0[None, None])
-    o, s = chain_form_prefill(q, k, v, g, b, S0)
-    assert rel(o, o_ref[:, 0]) < 1e-11 and rel(s, s_ref[0, 0]) < 1e-11
-    for m in ("gate_of_this_chunk", "no_R"):
-        o2, s2 = chain_form_prefill(q, k, v, g, b, S0, mistake=m)
-        assert rel(o2, o_ref[:, 0]) > 1e-6, m
