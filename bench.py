@@ -72,8 +72,8 @@ KERNELS = {
 # and verify figures undercount writes: ncu starts each replay from a clean L2, and 56-58 MB of the
 # written states are still resident (dirty) in L2 when the launch ends.
 TRAFFIC = {
-    "gdn_scan_bf16_kernel": 202.96e6 + 28.44e6,
-    "gdn_prep_bf16_kernel": 68.24e6 + 48.38e6,
+    "gdn_scan_bf16_kernel": 203.06e6 + 23.54e6,
+    "gdn_prep_bf16_kernel": 68.21e6 + 48.69e6,
     "gdn_l2norm_kernel": 67.12e6 + 21.02e6,
     "gdn_decode_step_kernel": 135.83e6 + 77.84e6,
     "gdn_decode_verify_kernel": 140.59e6 + 479.75e6,
@@ -343,8 +343,12 @@ WORKLOAD_DESCS = {
     "tiny_fp32": "B=1, T=128 (4 chunks), H=2, dk=dv=64, fp32 q/k/v, g~U[-0.5,0), zero initial state",
 }
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel for these workloads
-# (None until captured, reset whenever the kernel changes)
-TRAFFIC_BY_WORKLOAD = {}
+# (None until captured, reset whenever the kernel changes).  long_128k: captured on its first 32,768
+# tokens (1,025 chunks; the full launch holds too much memory for a multi-pass capture) and scaled by
+# the chunk count 4,097 / 1,025, the traffic per chunk-row being the same at every length.
+TRAFFIC_BY_WORKLOAD = {
+    ("long_128k", "gdn_scan_bf16_kernel"): (1623.81e6 + 259.82e6) * 4097 / 1025,
+}
 
 
 def l2_flush_buffer(dev):
