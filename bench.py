@@ -59,9 +59,9 @@ def flops_prep(d=D):
 # copy bandwidth.
 KERNELS = {
     "gdn_scan_tc_kernel": dict(bound="tensor", flops_per_token_head=flops_scan(), split=3),
-    "gdn_scan_bf16_kernel": dict(bound="tensor", flops_per_token_head=flops_scan(), split=3),
+    "gdn_scan_pair_kernel": dict(bound="tensor", flops_per_token_head=flops_scan(), split=3),
     "gdn_prep_kernel": dict(bound="tensor", flops_per_token_head=flops_prep(), split=3),
-    "gdn_prep_bf16_kernel": dict(bound="tensor", flops_per_token_head=flops_prep(), split=3),
+    "gdn_prep_pair_kernel": dict(bound="tensor", flops_per_token_head=flops_prep(), split=3),
     "gdn_plan_kernel": dict(bound="latency"),
     "gdn_decode_step_kernel": dict(bound="hbm"),
     "gdn_decode_verify_kernel": dict(bound="hbm"),
@@ -72,8 +72,6 @@ KERNELS = {
 # and verify figures undercount writes: ncu starts each replay from a clean L2, and 56-58 MB of the
 # written states are still resident (dirty) in L2 when the launch ends.
 TRAFFIC = {
-    "gdn_scan_bf16_kernel": 203.06e6 + 23.54e6,
-    "gdn_prep_bf16_kernel": 68.21e6 + 48.69e6,
     "gdn_l2norm_kernel": 67.12e6 + 21.02e6,
     "gdn_decode_step_kernel": 135.83e6 + 77.84e6,
     "gdn_decode_verify_kernel": 140.59e6 + 479.75e6,
@@ -347,7 +345,6 @@ WORKLOAD_DESCS = {
 # tokens (1,025 chunks; the full launch holds too much memory for a multi-pass capture) and scaled by
 # the chunk count 4,097 / 1,025, the traffic per chunk-row being the same at every length.
 TRAFFIC_BY_WORKLOAD = {
-    ("long_128k", "gdn_scan_bf16_kernel"): (1623.81e6 + 259.82e6) * 4097 / 1025,
 }
 
 

@@ -172,9 +172,9 @@ int gdn_chunk_prefill_cuts(const void* q, const void* k, const void* v, const fl
  *   Arguments, layouts and results are those of gdn_chunk_prefill minus workspace/workspace_bytes.
  *   Limit: the problem must satisfy gdn_chunk_prefill_workspace_bytes_ex(total_tokens, num_seqs,
  *   H, dk, dv, dtype) <= 64 MiB; larger problems return GDN_ERR_WORKSPACE and enqueue nothing.
- *   The workspace is almost all operator records, one of 25,088 bytes per (chunk, head) over
- *   floor(total_tokens / 32) + num_seqs chunks, so the scratch holds about
- *   floor(64 MiB / (H x 25,088)) - num_seqs chunks: for H = 32, d = 128 about 2,650 tokens in one
+ *   The workspace is almost all operator records, one of 49,664 bytes per (pair of chunks, head)
+ *   over floor(total_tokens / 64) + num_seqs pairs on the bf16 path, so the scratch holds about
+ *   floor(64 MiB / (H x 49,664)) - num_seqs pairs: for H = 32, d = 128 about 2,680 tokens in one
  *   sequence.  With GDN_QK_L2NORM in dtype the normalised q/k copies live in the scratch too, which
  *   lowers the limit (about 1,600 tokens in one sequence at H = 32, d = 128, bf16).
  *   Set-up: the first call on a device looks up that device's copy of the scratch array (a CUDA

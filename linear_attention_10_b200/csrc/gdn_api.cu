@@ -18,8 +18,8 @@
 #include "gdn_norm.cuh"
 #include "gdn_plan.cuh"
 #include "gdn_prefill_tc.cuh"
-#include "gdn_prep_bf16.cuh"
-#include "gdn_scan_bf16.cuh"
+#include "gdn_prep_pair.cuh"
+#include "gdn_scan_pair.cuh"
 
 namespace gdn {
 
@@ -262,14 +262,15 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         if (cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) g_num_sms = 148;
     }
 
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     {
+        // table entries: pairs of chunks on the bf16 path, chunks on the fp32 path
         ProfScope prof("gdn_plan_kernel", st);
-        gdn_plan_kernel<<<1, 1024, 0, st>>>(cu, N, T_total, fixed_len, cuts.pos, cuts.n, meta, chunk_off, chunk_tab,
-                                            seg, order, status);
+        gdn_plan_kernel<kBf16 ? kPair : kChunk><<<1, 1024, 0, st>>>(cu, N, T_total, fixed_len, cuts.pos, cuts.n, meta,
+                                                                    chunk_off, chunk_tab, seg, order, status);
     }
     if (!cuda_ok(cudaPeekAtLastError(), "gdn_plan_kernel launch")) return GDN_ERR_LAUNCH;
 
-    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     CUtensorMap tq{}, tk{}, tv{};
     if constexpr (kBf16) {
         const uint64_t Tn = (uint64_t)(T_total > 0 ? T_total : 1);
@@ -279,17 +280,18 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
             return GDN_ERR_CUDA;
     }
     if constexpr (kBf16) {
-      if (lay.nc_max > 0 && T_total > 0) {
-        using PL = PrepBf16Smem<DK>;
-        auto k1 = gdn_prep_bf16_kernel<DK>;
+      if (lay.np_max > 0 && T_total > 0) {
+        using PL = PrepPairSmem<DK>;
+        auto k1 = gdn_prep_pair_kernel<DK>;
         if (!set_dyn_smem(k1, PL::kBytes, "cudaFuncSetAttribute(max dynamic shared memory)"))
             return GDN_ERR_LAUNCH;
-        const int64_t items = lay.nc_max * (int64_t)H;
-        const int64_t cap = (int64_t)g_num_sms * kPrepBf16CtasPerSm;
+        const int64_t items = lay.np_max * (int64_t)H;
+        const int64_t cap = (int64_t)g_num_sms * kPrepPairCtasPerSm;
         const unsigned grid = (unsigned)(items < cap ? items : cap);
-        ProfScope prof("gdn_prep_bf16_kernel", st);
-        if (launch_dependent(k1, dim3(grid), dim3(128), PL::kBytes, st, tq, tk, g, beta, meta, chunk_off, chunk_tab,
-                             reinterpret_cast<uint8_t*>(op), H, status) != cudaSuccess)
+        ProfScope prof("gdn_prep_pair_kernel", st);
+        if (launch_dependent(k1, dim3(grid), dim3(kPrepPairThreads), PL::kBytes, st, tq, tk, g, beta,
+                             (const int*)meta, (const int4*)chunk_tab, reinterpret_cast<uint8_t*>(op), H,
+                             status) != cudaSuccess)
             return GDN_ERR_LAUNCH;
       }
     } else if (lay.nc_max > 0 && T_total > 0) {
@@ -306,24 +308,19 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
                              status) != cudaSuccess)
             return GDN_ERR_LAUNCH;
     }
-    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-        // bf16 inputs: operands staged by tensor maps, bf16 tensor-core products for K and Q
-        constexpr int MSB = 32;
-        using SB3 = ScanBf16Smem<DK, MSB, 3>;
-        using SB4 = ScanBf16Smem<DK, MSB, 4>;
-        constexpr int ST = (SB4::kBytes <= 227 * 1024) ? 4 : 3;
-        using SB = ScanBf16Smem<DK, MSB, ST>;
-        static_assert(SB3::kBytes <= 227 * 1024, "bf16 scan shared memory");
-        static_assert(MSB == 32, "the V tensor map boxes 32 columns");
-        auto kb = cuts.n > 0 ? gdn_scan_bf16_kernel<DK, DV, MSB, ST, true> : gdn_scan_bf16_kernel<DK, DV, MSB, ST, false>;
-        if (!set_dyn_smem(kb, SB::kBytes, "cudaFuncSetAttribute(max dynamic shared memory)"))
+    if constexpr (kBf16) {
+        // bf16 inputs: operands staged by tensor maps, bf16 tensor-core products, two chunks per step
+        using SP = ScanPairSmem<DK>;
+        static_assert(SP::kBytes <= 227 * 1024, "bf16 scan shared memory");
+        auto kb = cuts.n > 0 ? gdn_scan_pair_kernel<DK, DV, true> : gdn_scan_pair_kernel<DK, DV, false>;
+        if (!set_dyn_smem(kb, SP::kBytes, "cudaFuncSetAttribute(max dynamic shared memory)"))
             return GDN_ERR_LAUNCH;
         {
-            ProfScope prof("gdn_scan_bf16_kernel", st);
+            ProfScope prof("gdn_scan_pair_kernel", st);
             // one CTA per (32 state rows, head, sequence), the sequence's rank in `order` slowest
-            const int64_t ctas = (int64_t)(DV / MSB) * H * N;
+            const int64_t ctas = (int64_t)(DV / 32) * H * N;
             if (ctas > INT32_MAX) return GDN_ERR_INVALID_ARG;
-            if (launch_dependent(kb, dim3((unsigned)ctas), dim3(kScanBf16Threads), SB::kBytes, st, tq, tk,
+            if (launch_dependent(kb, dim3((unsigned)ctas), dim3(kScanPairThreads), SP::kBytes, st, tq, tk,
                                  tv, (const int*)meta, (const int*)order, (const int*)chunk_off, (const int4*)chunk_tab,
                                  reinterpret_cast<const uint8_t*>(op), state_in, static_cast<__nv_bfloat16*>(out),
                                  state_out, cuts.snaps, H, status) != cudaSuccess)

@@ -12,6 +12,17 @@ namespace gdn {
 // Chunk size of the chunkwise WY/UT form (Ferrite project page, Design section 03: 32 rows).
 constexpr int kChunk = 32;
 
+// Rows per step of the bf16 path: two chunks.  Its operator for the 64 rows is the 2 x 2 block
+// combination of the two chunks' 32 x 32 WY/UT inverses, so that [K; Q] and [T''; P T''] fill the
+// 128 rows of one M = 128 tensor-core tile and the state advances once per pair of chunks.
+constexpr int kPair = 64;
+
+// Operator record of one (pair, head) on the bf16 path: [T''; P T''] (128 x 64) as three bf16 parts
+// of 16 KB in the 128-byte-swizzled K-major layout, then Gamma_i and delta_i (64 floats each).
+constexpr uint32_t kPairPart = 16384;
+constexpr uint32_t kPairGate = 3 * kPairPart;
+constexpr uint32_t kPairRecordBytes = kPairGate + 2 * 64 * 4;
+
 // The per-device status word lives in gdn_api.cu; kernels receive its address.
 __device__ __forceinline__ void report(int* status, int code)
 {

@@ -1,6 +1,7 @@
 // gdn_plan.cuh -- chunk tables of a packed prefill call, and the workspace layout.
 //
-// Chunks of C = 32 rows restart at every sequence start (Ferrite project page, Design section 03:
+// Chunks of C = 32 rows (the fp32 path) or pairs of them (64 rows, the bf16 path) restart at every
+// sequence start (Ferrite project page, Design section 03:
 // the layer takes a prompt 32 rows at a time) and at every cut point the caller asks a state
 // snapshot for (section 07: the prompt cache saves state where each turn ends and splits a prompt at
 // identical places with or without a resume, which is what makes a resumed reply equal to a full one).
@@ -12,6 +13,7 @@
 #pragma once
 
 #include "gdn_common.cuh"
+#include "gdn_prefill_tc.cuh"
 #include "gdn_sm100.cuh"
 
 namespace gdn {
@@ -19,13 +21,15 @@ namespace gdn {
 // Workspace layout of gdn_chunk_prefill (all offsets 256-byte aligned).  NS = number of segments
 // (sequences + cut points).
 struct PrefillLayout {
-    int64_t nc_max;       // upper bound on the number of chunks: floor(T / C) + NS
-    size_t off_meta;      // int32[8]: [0] chunk count, [1] error flag
-    size_t off_chunk_off; // int32[NS + 1]: first global chunk of each sequence
+    int64_t nc_max;       // upper bound on the number of 32-row chunks: floor(T / 32) + NS
+    int64_t np_max;       // upper bound on the number of 64-row pairs: floor(T / 64) + NS
+    size_t off_meta;      // int32[8]: [0] chunk (or pair) count, [1] error flag
+    size_t off_chunk_off; // int32[NS + 1]: first global chunk (or pair) of each sequence
     size_t off_chunk_tab; // int4[nc_max]: (sequence, first token, rows, snapshot index or -1)
     size_t off_seg;       // int32[6 NS + 1]: segment start, sequence, cut, end, snapshot, chunk offset
     size_t off_order;     // int32[NS]: the sequences in the order the bf16 scan takes them
-    size_t off_op;        // [nc_max][H] operator records (up to 25088 bytes each)
+    size_t off_op;        // operator records: [nc_max][H] x 16,896 B (fp32 path) or
+                          // [np_max][H] x 49,664 B (bf16 path), whichever is larger
     size_t total;
 
     static size_t align(size_t x) { return (x + 255) & ~size_t(255); }
@@ -33,13 +37,16 @@ struct PrefillLayout {
     PrefillLayout(int64_t T, int NS, int H, int dk)
     {
         nc_max = T / kChunk + NS;
+        np_max = T / kPair + NS;
+        const size_t rec_f32 = (size_t)nc_max * H * kOpBytes;
+        const size_t rec_pair = (size_t)np_max * H * kPairRecordBytes;
         size_t o = 0;
         off_meta = o;      o = align(o + 8 * sizeof(int));
         off_chunk_off = o; o = align(o + (size_t)(NS + 1) * sizeof(int));
         off_chunk_tab = o; o = align(o + (size_t)nc_max * sizeof(int4));
         off_seg = o;       o = align(o + (size_t)(6 * NS + 1) * sizeof(int));
         off_order = o;     o = align(o + (size_t)NS * sizeof(int));
-        off_op = o;        o = align(o + (size_t)nc_max * H * 25088);   // largest record of the two paths
+        off_op = o;        o = align(o + (rec_f32 > rec_pair ? rec_f32 : rec_pair));
         total = o;
         (void)dk;
     }
@@ -111,6 +118,8 @@ __device__ __forceinline__ void plan_order(int N, const int* chunk_off, int* ord
     }
 }
 
+// CL: rows per table entry (32: chunks, 64: pairs of chunks).
+template <int CL>
 __global__ void __launch_bounds__(1024) gdn_plan_kernel(const int32_t* __restrict__ cu, int N, int64_t T,
                                                     int fixed_len, const int32_t* __restrict__ cuts, int n_cuts,
                                                     int* meta, int* chunk_off, int4* chunk_tab, int* seg,
@@ -143,7 +152,7 @@ __global__ void __launch_bounds__(1024) gdn_plan_kernel(const int32_t* __restric
                 const int64_t a = start_of(n), b = start_of(n + 1);
                 const bool bad = (b < a) || (n == 0 && a != 0) || (n == N - 1 && b != T) || b > T;
                 if (bad) s_err = 1;
-                nch = bad ? 0 : (int)((b - a + kChunk - 1) / kChunk);
+                nch = bad ? 0 : (int)((b - a + CL - 1) / CL);
             }
             const int incl = block_inclusive_scan_1024(nch, warp_tot);
             if (n < N) chunk_off[n] = s_running + incl - nch;
@@ -166,9 +175,9 @@ __global__ void __launch_bounds__(1024) gdn_plan_kernel(const int32_t* __restric
                 const int mid = (lo + hi + 1) >> 1;
                 if (chunk_off[mid] <= gc) lo = mid; else hi = mid - 1;
             }
-            const int64_t t0 = start_of(lo) + (int64_t)(gc - chunk_off[lo]) * kChunk;
+            const int64_t t0 = start_of(lo) + (int64_t)(gc - chunk_off[lo]) * CL;
             const int64_t e = start_of(lo + 1);
-            chunk_tab[gc] = make_int4(lo, (int)t0, (int)((e - t0) < kChunk ? (e - t0) : kChunk), -1);
+            chunk_tab[gc] = make_int4(lo, (int)t0, (int)((e - t0) < CL ? (e - t0) : CL), -1);
         }
         plan_order(N, chunk_off, order, s_cnt);
         return;
@@ -244,7 +253,7 @@ __global__ void __launch_bounds__(1024) gdn_plan_kernel(const int32_t* __restric
             }
             seg_end[j] = end;
             seg_snap[j] = snap;
-            nch = (end - seg_start[j] + kChunk - 1) / kChunk;
+            nch = (end - seg_start[j] + CL - 1) / CL;
         }
         const int incl = block_inclusive_scan_1024(nch, warp_tot);
         if (j < NS) seg_off[j] = s_running + incl - nch;
@@ -270,8 +279,8 @@ __global__ void __launch_bounds__(1024) gdn_plan_kernel(const int32_t* __restric
         }
         while (lo + 1 < NS && seg_off[lo + 1] <= gc) ++lo;
         const int j = lo;
-        const int t0 = seg_start[j] + (gc - seg_off[j]) * kChunk;
-        const int rows = (seg_end[j] - t0 < kChunk) ? (seg_end[j] - t0) : kChunk;
+        const int t0 = seg_start[j] + (gc - seg_off[j]) * CL;
+        const int rows = (seg_end[j] - t0 < CL) ? (seg_end[j] - t0) : CL;
         const int snap = (t0 + rows == seg_end[j]) ? seg_snap[j] : -1;
         chunk_tab[gc] = make_int4(seg_seq[j], t0, rows, snap);
     }

@@ -49,14 +49,6 @@ constexpr uint32_t kOpLo = 8192;
 constexpr uint32_t kOpGate = 16384;
 constexpr uint32_t kOpCopyBytes = 16384 + 80 * 4;   // staged per chunk (operator + gates)
 constexpr uint32_t kOpBytes = 16384 + 512;          // record stride in the workspace
-// bf16-input path record: three bf16 parts (each 64 x 32, K-major, 64-byte swizzle) of
-// [T''; P T''], then three of the cross-chunk Gram matrix G' = [K; Q] K_prev^T (the chunk's rows
-// against the previous chunk's keys in the same sequence), then the gates.
-constexpr uint32_t kOpBPart = 4096;
-constexpr uint32_t kOpBCross = 3 * kOpBPart;
-constexpr uint32_t kOpBGate = 6 * kOpBPart;
-constexpr uint32_t kOpBCopyBytes = 6 * kOpBPart + 80 * 4;
-constexpr uint32_t kOpBytesB = 25088;
 
 template <typename T>
 struct ExactTF32 { static constexpr bool value = false; };

@@ -1,0 +1,438 @@
+// gdn_prep_pair.cuh -- per-(pair of chunks, head) WY/UT operator for bf16 q/k (sm_100a).
+//
+// The chunkwise WY/UT form (Ferrite project page, Design section 03) takes each chunk of 32 rows with
+// T = (I + A)^-1.  The bf16 scan advances the state once per pair of chunks (rows 0..31: chunk a,
+// rows 32..63: chunk b), and this kernel builds the pair's operator record for it:
+//
+//   A = strictly-lower(diag(beta) (D o K K^T)),  P = lower-incl-diagonal(D o Q K^T),
+//   D_ij = exp(gamma_i - gamma_j)   (gamma: cumulative log-gate from the pair's first row),
+//   T = (I + A)^-1 = [[T_a, 0], [T_ba, T_b]],   T_a, T_b: the two chunks' 32 x 32 inverses,
+//   T_ba = -T_b A_ba T_a,   T'' = T diag(beta),
+//
+// and writes [T''; P T''] (128 x 64) as three bf16 parts in the 128-byte-swizzled K-major layout of a
+// tensor-core A operand, with Gamma_i = exp(gamma_i) and delta_i = exp(gamma_63 - gamma_i).  A
+// chunk's own inverse uses the same 2 x 2 block form one level down (16 x 16 blocks by forward
+// substitution, then T21 = -T22 A21 T11), which shortens the dependent chain of the substitution.
+//
+// What is specific to bf16 inputs: the pair's [K; Q] rows are exact bf16 values, so the tensor-
+// memory-access engine copies them straight into the operand layout (the next item's rows arrive
+// while this one is gated, solved and written out) and one bf16 tensor-core product (M = 128, N = 64,
+// K = dk) forms both Gram matrices exactly in fp32.  The gates are applied while the Gram rows come
+// out of tensor memory.
+//
+// Rows past a sequence's end (the pair's last rows may hold the next sequence's tokens) get g = 0
+// and beta = 0: their rows of A and columns of T'' are zero, so they never reach the scan's state.
+#pragma once
+
+#include <cuda.h>
+
+#include "gdn_common.cuh"
+#include "gdn_prefill_tc.cuh"
+#include "gdn_sm100.cuh"
+
+namespace gdn {
+
+template <int DK>
+struct PrepPairSmem {
+    static constexpr int NP = DK / 64;
+    static constexpr uint32_t kPanel = 128 * 128;                    // [K; Q]: 128 rows x 128 B per panel
+    static constexpr uint32_t oTile = 0;                             // one buffer, refilled once the Gram
+                                                                     // product has read it
+    static constexpr int LD = 68;                                    // fp32 row pitch (16-byte rows)
+    static constexpr uint32_t oA = NP * kPanel;                      // [64][LD] A
+    static constexpr uint32_t oP = oA + 64 * LD * 4;                 // [64][LD] P
+    static constexpr uint32_t oT = oP + 64 * LD * 4;                 // [64][LD] T
+    static constexpr int LM = 36;
+    static constexpr uint32_t oM = oT + 64 * LD * 4;                 // [32][LM] block products
+    static constexpr uint32_t oGam = oM + 32 * LM * 4;               // [64] log2(e) gamma
+    static constexpr uint32_t oBet = oGam + 256;                     // [64] beta
+    static constexpr uint32_t oAlph = oBet + 256;                    // [64] exp(g), 4 spare
+    static constexpr uint32_t oPre = oAlph + 272;                    // [64] exp(gamma_i - gamma_31), i >= 32
+    static constexpr uint32_t oBar = oPre + 256;                     // tile_full, mma, drain
+    static constexpr uint32_t oTmem = oBar + 24;
+    static constexpr uint32_t oAbort = oTmem + 4;
+    static constexpr uint32_t kTotal = oAbort + 4;
+    static constexpr uint32_t kBytes = kTotal + 1024;
+    static_assert(oA % 1024 == 0, "tile panels on 1024-byte boundaries");
+};
+
+// CTAs resident per SM (shared memory and registers are sized for it; the launch sizes its grid so)
+constexpr int kPrepPairCtasPerSm = 2;
+constexpr int kPrepPairThreads = 256;
+static_assert(kPrepPairCtasPerSm * (PrepPairSmem<128>::kBytes + 1024) <= 233472, "two CTAs per SM");
+
+template <int DK>
+__global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
+    gdn_prep_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const float* __restrict__ g, const float* __restrict__ beta, const int* __restrict__ meta,
+                         const int4* __restrict__ chunk_tab, uint8_t* __restrict__ op, int H, int* status)
+{
+    using namespace sm100;
+    using L = PrepPairSmem<DK>;
+    constexpr int NP = L::NP;
+    constexpr int LD = L::LD, LM = L::LM;
+    // launched as a dependent of the plan kernel: its pair table is read below
+    grid_dep_wait();
+    grid_dep_launch();
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    float* A = reinterpret_cast<float*>(sm + L::oA);
+    float* P = reinterpret_cast<float*>(sm + L::oP);
+    float* Tm = reinterpret_cast<float*>(sm + L::oT);
+    float* M = reinterpret_cast<float*>(sm + L::oM);
+    float* gam = reinterpret_cast<float*>(sm + L::oGam);
+    float* bet = reinterpret_cast<float*>(sm + L::oBet);
+    float* alph = reinterpret_cast<float*>(sm + L::oAlph);
+    float* pre = reinterpret_cast<float*>(sm + L::oPre);
+    uint64_t* tile_full = reinterpret_cast<uint64_t*>(sm + L::oBar);
+    uint64_t* mma_bar = tile_full + 1;
+    uint64_t* drain = tile_full + 2;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::oTmem);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::oAbort);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nitems = meta[0] * H;
+    if (tid == 0) {
+        mbar_init(tile_full, 1);
+        mbar_init(mma_bar, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tslot, 64);      // the Gram product: 128 lanes x 64 columns
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+
+    // copies the [K; Q] rows of one item into the tile buffer (one thread; issued once the previous
+    // item's product has read the buffer).  Panel p: K rows 0..63, then Q rows 0..63.
+    auto issue_tile = [&](int item) {
+        const int gc = item / H, h = item % H;
+        const int t0 = chunk_tab[gc].y;
+        const int t1 = (t0 < INT32_MAX - 32) ? t0 + 32 : INT32_MAX;   // rows past the tensor read as zeros
+        mbar_arrive_expect_tx(tile_full, NP * L::kPanel);
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            const uint32_t pan = sbase + L::oTile + p * L::kPanel;
+            tma_load_2d(pan, &tm_k, h * DK + p * 64, t0, tile_full);
+            tma_load_2d(pan + 4096, &tm_k, h * DK + p * 64, t1, tile_full);
+            tma_load_2d(pan + 8192, &tm_q, h * DK + p * 64, t0, tile_full);
+            tma_load_2d(pan + 12288, &tm_q, h * DK + p * 64, t1, tile_full);
+        }
+    };
+    // gate inputs of one item for lane `lane` of warp 7: rows 2 lane and 2 lane + 1 (zero past the
+    // pair's rows)
+    auto load_gates = [&](int item, float (&gv)[2], float (&bv)[2]) {
+        const int gc = item / H, h = item % H;
+        const int4 ct = chunk_tab[gc];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int r = 2 * lane + e;
+            const bool ok = r < ct.z;
+            gv[e] = ok ? __ldg(g + (size_t)(ct.y + r) * H + h) : 0.f;
+            bv[e] = ok ? __ldg(beta + (size_t)(ct.y + r) * H + h) : 0.f;
+        }
+    };
+
+    if (tid == 0 && (int)blockIdx.x < nitems) issue_tile(blockIdx.x);
+    float gv_cur[2] = {0.f, 0.f}, bv_cur[2] = {0.f, 0.f};
+    if (warp == 7 && (int)blockIdx.x < nitems) load_gates(blockIdx.x, gv_cur, bv_cur);
+
+    constexpr uint32_t idG = idesc_bf16(128, 64);
+    constexpr float kLog2e = 1.4426950408889634f;
+    uint32_t iter = 0;
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++iter) {
+        GDN_PREP_TRACE(iter, 0);
+        const int gc = item / H, h = item % H;
+
+        // Gram products D[r][n] = [K; Q]_r . K_n, n < 64, on the tensor cores (thread 0)
+        if (tid == 0) {
+            if (!mbar_wait(tile_full, iter & 1u, abort_flag)) {
+                tc_abort(status, abort_flag);
+            } else {
+                tc_fence_after();
+                const uint64_t a = sw128_desc(sbase + L::oTile, 0, 128);
+#pragma unroll
+                for (int ks = 0; ks < DK / 16; ++ks) {
+                    const uint64_t o = sw128_ks_off(ks, 128);
+                    mma_bf16(tmem, a + o, a + o, idG, ks > 0);
+                }
+                mma_commit(mma_bar);
+                if (!mbar_wait(mma_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
+            }
+        } else if (warp == 7) {
+            // cumulative log-gate over the pair (two rows per lane), beta, exp(g), and the running
+            // products exp(gamma_i - gamma_31) of the second chunk's rows; then prefetch the next item's
+            const float s2 = gv_cur[0] + gv_cur[1];
+            float inc = s2;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += y;
+            }
+            const float ex = inc - s2;
+            const float a0 = exp2f(gv_cur[0] * kLog2e), a1 = exp2f(gv_cur[1] * kLog2e);
+            // product of exp(g) over rows 32 .. 2 lane + 1 (lanes 16..31; the others multiply by 1)
+            const float pp = (lane >= 16) ? a0 * a1 : 1.f;
+            float incp = pp;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incp, o);
+                if (lane >= o) incp *= y;
+            }
+            const int r = 2 * lane;
+            gam[r] = (ex + gv_cur[0]) * kLog2e;
+            gam[r + 1] = inc * kLog2e;
+            bet[r] = bv_cur[0];
+            bet[r + 1] = bv_cur[1];
+            alph[r] = a0;
+            alph[r + 1] = a1;
+            const float exclp = __shfl_up_sync(0xffffffffu, incp, 1);
+            if (lane >= 16) {
+                pre[r] = (lane > 16 ? exclp : 1.f) * a0;
+                pre[r + 1] = incp;
+            }
+            if (item + (int)gridDim.x < nitems) load_gates(item + gridDim.x, gv_cur, bv_cur);
+        }
+        __syncthreads();
+        GDN_PREP_TRACE(iter, 1);
+        if (*abort_flag) break;
+        tc_fence_after();
+        // the tile buffer is free (the Gram product has completed): fetch the next item's rows
+        if (tid == 0 && item + (int)gridDim.x < nitems) issue_tile(item + gridDim.x);
+        {
+            // thread (q = warp % 4, hf = warp / 4, lane): Gram row r = 32 q + lane, columns 32 hf ..
+            // 32 hf + 31.  Rows 0..63: K K^T -> A (times beta_i, strictly lower); rows 64..127:
+            // Q K^T -> P (lower, with the diagonal).  Decay ratios exp(gamma_i - gamma_j) as a running
+            // product from the diagonal down (one multiply per entry instead of an exp2).
+            const int q = warp & 3, hf = warp >> 2;
+            const int r = q * 32 + lane;
+            const bool isP = r >= 64;
+            const int i = r & 63;
+            float d[32];
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 32 * hf, d);
+            tmem_ld_wait();
+            const float wr = isP ? 1.f : bet[i];
+            const int lim = isP ? i + 1 : i;
+            const int jtop = 32 * hf + 31;
+            float a = (i > jtop) ? pre[i] : 1.f;
+            float vals[32];
+#pragma unroll
+            for (int jj = 31; jj >= 0; --jj) {
+                const int j = 32 * hf + jj;
+                if (jj < 31) a = (j >= i) ? 1.f : a * alph[j + 1];
+                vals[jj] = (j < lim) ? wr * a * d[jj] : 0.f;
+            }
+            const uint32_t dst = sbase + (isP ? L::oP : L::oA) + (uint32_t)(i * LD * 4 + hf * 128);
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4)
+                asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + c4 * 16), "f"(vals[4 * c4]),
+                             "f"(vals[4 * c4 + 1]), "f"(vals[4 * c4 + 2]), "f"(vals[4 * c4 + 3]));
+        }
+        tc_fence_before();
+        __syncthreads();
+        GDN_PREP_TRACE(iter, 2);
+
+        if (warp < 2) {
+            // the four 16 x 16 diagonal blocks of T by forward substitution: lane -> block
+            // 2 warp + lane / 16, column j
+            const int blk = 2 * warp + (lane >> 4), j = lane & 15, o = blk * 16;
+            float t[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) t[r] = (r == j) ? 1.f : 0.f;
+#pragma unroll
+            for (int i = 0; i < 15; ++i) {
+#pragma unroll
+                for (int r = i + 1; r < 16; ++r) t[r] = fmaf(-A[(o + r) * LD + o + i], t[i], t[r]);
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Tm[(o + r) * LD + o + j] = t[r];
+            if ((blk & 1) == 0) {
+#pragma unroll
+                for (int r = 0; r < 16; ++r) Tm[(o + r) * LD + o + 16 + j] = 0.f;   // upper right of a chunk
+            }
+        } else {
+            // T is zero above the chunk blocks: rows 0..31, columns 32..63
+            for (int e = tid - 64; e < 32 * 8; e += 192) {
+                const int r = e >> 3, c4 = e & 7;
+                *reinterpret_cast<float4*>(Tm + r * LD + 32 + 4 * c4) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        __syncthreads();
+        {
+            // per chunk (tid / 128): M16 = A21 T11 (16 x 16), two outputs per thread
+            const int ch = tid >> 7, t = tid & 127, o = 32 * ch;
+            const int r = t >> 3, c = (t & 7) * 2;
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int m4 = 0; m4 < 4; ++m4) {
+                const float4 av = *reinterpret_cast<const float4*>(A + (o + 16 + r) * LD + o + 4 * m4);
+                const float am[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 tv = *reinterpret_cast<const float2*>(Tm + (o + 4 * m4 + e) * LD + o + c);
+                    a0 = fmaf(am[e], tv.x, a0);
+                    a1 = fmaf(am[e], tv.y, a1);
+                }
+            }
+            *reinterpret_cast<float2*>(M + ch * 16 * 16 + r * 16 + c) = make_float2(a0, a1);
+        }
+        __syncthreads();
+        {
+            // T21 = -T22 M16 inside each chunk
+            const int ch = tid >> 7, t = tid & 127, o = 32 * ch;
+            const int r = t >> 3, c = (t & 7) * 2;
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int m4 = 0; m4 < 4; ++m4) {
+                const float4 tv4 = *reinterpret_cast<const float4*>(Tm + (o + 16 + r) * LD + o + 16 + 4 * m4);
+                const float tm[4] = {tv4.x, tv4.y, tv4.z, tv4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 mv = *reinterpret_cast<const float2*>(M + ch * 16 * 16 + (4 * m4 + e) * 16 + c);
+                    a0 = fmaf(tm[e], mv.x, a0);
+                    a1 = fmaf(tm[e], mv.y, a1);
+                }
+            }
+            *reinterpret_cast<float2*>(Tm + (o + 16 + r) * LD + o + c) = make_float2(-a0, -a1);
+        }
+        __syncthreads();
+        GDN_PREP_TRACE(iter, 3);
+        {
+            // M32 = A_ba T_a (32 x 32; T_a lower triangular): thread -> row r, columns c0 .. c0 + 3
+            const int r = tid >> 3, c0 = (tid & 7) * 4;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int m = c0; m < 32; m += 4) {
+                const float4 av = *reinterpret_cast<const float4*>(A + (32 + r) * LD + m);
+                const float am[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float4 tv = *reinterpret_cast<const float4*>(Tm + (m + e) * LD + c0);
+                    acc[0] = fmaf(am[e], tv.x, acc[0]);
+                    acc[1] = fmaf(am[e], tv.y, acc[1]);
+                    acc[2] = fmaf(am[e], tv.z, acc[2]);
+                    acc[3] = fmaf(am[e], tv.w, acc[3]);
+                }
+            }
+            *reinterpret_cast<float4*>(M + r * LM + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        }
+        __syncthreads();
+        {
+            // T_ba = -T_b M32 (T_b lower triangular)
+            const int r = tid >> 3, c0 = (tid & 7) * 4;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int m = 0; m <= r; m += 4) {
+                const float4 tv4 = *reinterpret_cast<const float4*>(Tm + (32 + r) * LD + 32 + m);
+                const float tb[4] = {tv4.x, tv4.y, tv4.z, tv4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float4 mv = *reinterpret_cast<const float4*>(M + (m + e) * LM + c0);
+                    acc[0] = fmaf(tb[e], mv.x, acc[0]);
+                    acc[1] = fmaf(tb[e], mv.y, acc[1]);
+                    acc[2] = fmaf(tb[e], mv.z, acc[2]);
+                    acc[3] = fmaf(tb[e], mv.w, acc[3]);
+                }
+            }
+            *reinterpret_cast<float4*>(Tm + (32 + r) * LD + c0) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+        }
+        __syncthreads();
+        GDN_PREP_TRACE(iter, 4);
+
+        // operator record: [T''; P T''] with T'' = T diag(beta), P T'' = (P T) diag(beta), each 8-column
+        // row segment as three bf16 parts (one 16-byte store each) in the 128-byte-swizzled image.
+        // Output blocks of 32 x 32: (a, a) and (b, b) by 64 threads each (two rows x 8 columns, sums
+        // over one chunk's rows), (b, a) by 128 threads (one row x 8 columns, sums over both chunks);
+        // the (a, b) blocks of T'' and P T'' are zero.
+        uint8_t* dst = op + ((size_t)gc * H + h) * kPairRecordBytes;
+        {
+            int i0, nrow, c0;
+            if (tid < 64) {
+                i0 = (tid >> 2) * 2; nrow = 2; c0 = (tid & 3) * 8;
+            } else if (tid < 128) {
+                i0 = 32 + ((tid - 64) >> 2) * 2; nrow = 2; c0 = 32 + (tid & 3) * 8;
+            } else {
+                i0 = 32 + ((tid - 128) >> 2); nrow = 1; c0 = (tid & 3) * 8;
+            }
+            const float4 b0 = *reinterpret_cast<const float4*>(bet + c0);
+            const float4 b1 = *reinterpret_cast<const float4*>(bet + c0 + 4);
+            const float bc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            // (P T)[i][c] = sum over m in [c0, i] of P[i][m] T[m][c]  (P lower, T lower)
+            float acc[2][8];
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[rr][c] = 0.f;
+            const int mend = i0 + nrow;                  // exclusive; P[i][m] = 0 for m > i
+            for (int m = c0; m < mend; m += 4) {
+                const float4 p0 = *reinterpret_cast<const float4*>(P + i0 * LD + m);
+                const float4 p1 = *reinterpret_cast<const float4*>(P + (i0 + 1) * LD + m);
+                const float pa[4] = {p0.x, p0.y, p0.z, p0.w}, pb[4] = {p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float4 t0 = *reinterpret_cast<const float4*>(Tm + (m + e) * LD + c0);
+                    const float4 t1 = *reinterpret_cast<const float4*>(Tm + (m + e) * LD + c0 + 4);
+                    const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        acc[0][c] = fmaf(pa[e], tv[c], acc[0][c]);
+                        acc[1][c] = fmaf(pb[e], tv[c], acc[1][c]);
+                    }
+                }
+            }
+            const uint32_t zero4[4] = {0u, 0u, 0u, 0u};
+            for (int rr = 0; rr < nrow; ++rr) {
+                const int i = i0 + rr;
+                const float4 t0 = *reinterpret_cast<const float4*>(Tm + i * LD + c0);
+                const float4 t1 = *reinterpret_cast<const float4*>(Tm + i * LD + c0 + 4);
+                const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+                uint32_t w[3][4], x[3][4];
+#pragma unroll
+                for (int c = 0; c < 8; c += 2) {
+                    bf16x2_split3(tv[c] * bc[c], tv[c + 1] * bc[c + 1], w[0][c / 2], w[1][c / 2], w[2][c / 2]);
+                    bf16x2_split3(acc[rr][c] * bc[c], acc[rr][c + 1] * bc[c + 1], x[0][c / 2], x[1][c / 2],
+                                  x[2][c / 2]);
+                }
+                const uint32_t ot = sw128_off_h(i, c0, 128), opt = sw128_off_h(64 + i, c0, 128);
+#pragma unroll
+                for (int p = 0; p < 3; ++p) {
+                    stg128(dst + p * kPairPart + ot, w[p]);
+                    stg128(dst + p * kPairPart + opt, x[p]);
+                }
+                if (tid < 64) {
+                    // the zero (a, b) blocks
+                    const uint32_t zt = sw128_off_h(i, 32 + c0, 128), zp = sw128_off_h(64 + i, 32 + c0, 128);
+#pragma unroll
+                    for (int p = 0; p < 3; ++p) {
+                        stg128(dst + p * kPairPart + zt, zero4);
+                        stg128(dst + p * kPairPart + zp, zero4);
+                    }
+                }
+            }
+        }
+        if (tid >= 128) {
+            // gates: Gamma_i (i < 64), then delta_i = Gamma_63 / Gamma_i as exp2 of the difference
+            float* gt = reinterpret_cast<float*>(dst + kPairGate);
+            const int e = tid - 128;
+            gt[e] = (e < 64) ? exp2f(gam[e]) : exp2f(gam[63] - gam[e - 64]);
+        }
+        __syncthreads();
+        GDN_PREP_TRACE(iter, 5);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *abort_flag) {
+        // after a timeout, give the product this thread issued a bounded time to finish
+        mma_commit(drain);
+        volatile int never = 0;
+        mbar_wait(drain, 0, &never, 100000000ull);
+    }
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+}  // namespace gdn
