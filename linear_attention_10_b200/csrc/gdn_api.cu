@@ -233,6 +233,11 @@ static bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uin
 #define GDN_SCAN_MINB 1
 #endif
 
+// column groups per lane quarter of the bf16 scan's chain warps (compile-time tuning knob)
+#ifndef GDN_PAIR_NQ
+#define GDN_PAIR_NQ 2
+#endif
+
 static int g_num_sms = 0;
 
 // cut points of one prefill call and where their state snapshots go (n = 0: none)
@@ -312,7 +317,8 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         // bf16 inputs: operands staged by tensor maps, bf16 tensor-core products, two chunks per step
         using SP = ScanPairSmem<DK>;
         static_assert(SP::kBytes <= 227 * 1024, "bf16 scan shared memory");
-        auto kb = cuts.n > 0 ? gdn_scan_pair_kernel<DK, DV, true> : gdn_scan_pair_kernel<DK, DV, false>;
+        constexpr int NQ = GDN_PAIR_NQ;
+        auto kb = cuts.n > 0 ? gdn_scan_pair_kernel<DK, DV, true, NQ> : gdn_scan_pair_kernel<DK, DV, false, NQ>;
         if (!set_dyn_smem(kb, SP::kBytes, "cudaFuncSetAttribute(max dynamic shared memory)"))
             return GDN_ERR_LAUNCH;
         {
@@ -320,7 +326,7 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
             // one CTA per (32 state rows, head, sequence), the sequence's rank in `order` slowest
             const int64_t ctas = (int64_t)(DV / 32) * H * N;
             if (ctas > INT32_MAX) return GDN_ERR_INVALID_ARG;
-            if (launch_dependent(kb, dim3((unsigned)ctas), dim3(kScanPairThreads), SP::kBytes, st, tq, tk,
+            if (launch_dependent(kb, dim3((unsigned)ctas), dim3(scan_pair_threads(NQ)), SP::kBytes, st, tq, tk,
                                  tv, (const int*)meta, (const int*)order, (const int*)chunk_off, (const int4*)chunk_tab,
                                  reinterpret_cast<const uint8_t*>(op), state_in, static_cast<__nv_bfloat16*>(out),
                                  state_out, cuts.snaps, H, status) != cudaSuccess)

@@ -15,16 +15,21 @@
 // substitution, then T21 = -T22 A21 T11), which shortens the dependent chain of the substitution.
 //
 // What is specific to bf16 inputs: the pair's [K; Q] rows are exact bf16 values, so the tensor-
-// memory-access engine copies them straight into the operand layout (the next item's rows arrive
-// while this one is gated, solved and written out) and one bf16 tensor-core product (M = 128, N = 64,
-// K = dk) forms both Gram matrices exactly in fp32.  The gates are applied while the Gram rows come
-// out of tensor memory.
+// memory-access engine copies them straight into the operand layout and one bf16 tensor-core product
+// (M = 128, N = 64, K = dk) forms both Gram matrices exactly in fp32.  The gates are applied while the
+// Gram rows come out of tensor memory.  P T'' is a second tensor-core product (M = 64, N = 64,
+// K = 64): P and T'' as three bf16 parts each, the six part products with p + q <= 4 accumulated in
+// fp32, which keeps every term above 2^-24 relative (fp32-accurate).  T'' is staged in exactly the
+// byte layout of the record's rows 0..63, so the same 16-byte packets go to shared memory (the
+// product's B operand) and to the record.
 //
 // Rows past a sequence's end (the pair's last rows may hold the next sequence's tokens) get g = 0
 // and beta = 0: their rows of A and columns of T'' are zero, so they never reach the scan's state.
 #pragma once
 
 #include <cuda.h>
+
+#include <type_traits>
 
 #include "gdn_common.cuh"
 #include "gdn_prefill_tc.cuh"
@@ -36,30 +41,37 @@ template <int DK>
 struct PrepPairSmem {
     static constexpr int NP = DK / 64;
     static constexpr uint32_t kPanel = 128 * 128;                    // [K; Q]: 128 rows x 128 B per panel
-    static constexpr uint32_t oTile = 0;                             // one buffer, refilled once the Gram
-                                                                     // product has read it
-    static constexpr int LD = 68;                                    // fp32 row pitch (16-byte rows)
-    static constexpr uint32_t oA = NP * kPanel;                      // [64][LD] A
-    static constexpr uint32_t oP = oA + 64 * LD * 4;                 // [64][LD] P
-    static constexpr uint32_t oT = oP + 64 * LD * 4;                 // [64][LD] T
+    // The tile region holds the item's [K; Q] rows until the Gram product has read them, then the
+    // block products of the inverse and the three parts of T'' (8 KB each, the B operand of P T''),
+    // then the next item's rows (copied once P T'' has read T'').
+    static constexpr uint32_t oTile = 0;
+    static constexpr uint32_t oTpp = 0;                              // T'' parts: 3 x 64 rows x 128 B
     static constexpr int LM = 36;
-    static constexpr uint32_t oM = oT + 64 * LD * 4;                 // [32][LM] block products
-    static constexpr uint32_t oGam = oM + 32 * LM * 4;               // [64] log2(e) gamma
+    static constexpr uint32_t oM = 3 * 8192;                         // [32][LM] block products
+    static constexpr uint32_t kTileRegion0 = (NP * kPanel > oM + 32 * LM * 4) ? NP * kPanel : oM + 32 * LM * 4;
+    static constexpr uint32_t kTileRegion = (kTileRegion0 + 1023) & ~1023u;
+    static constexpr int LD = 68;                                    // fp32 row pitch (16-byte rows)
+    // A and T share one buffer: each block of T is written over a block of A that has been read
+    // for the last time (the diagonal blocks by their own substitution, the off-diagonal ones after
+    // the product that consumes them).  Column 67 of row i >= 32 holds exp(gamma_i - gamma_31).
+    static constexpr uint32_t oA = kTileRegion;                      // [64][LD] A, then T
+    static constexpr uint32_t oT = oA;
+    static constexpr uint32_t oPp = oA + 64 * LD * 4;                // P parts: 3 x 64 rows x 128 B
+    static constexpr uint32_t oGam = oPp + 3 * 8192;                 // [64] log2(e) gamma
     static constexpr uint32_t oBet = oGam + 256;                     // [64] beta
     static constexpr uint32_t oAlph = oBet + 256;                    // [64] exp(g), 4 spare
-    static constexpr uint32_t oPre = oAlph + 272;                    // [64] exp(gamma_i - gamma_31), i >= 32
-    static constexpr uint32_t oBar = oPre + 256;                     // tile_full, mma, drain
-    static constexpr uint32_t oTmem = oBar + 24;
+    static constexpr uint32_t oBar = oAlph + 272;                    // tile_full, gram, pt, drain
+    static constexpr uint32_t oTmem = oBar + 32;
     static constexpr uint32_t oAbort = oTmem + 4;
     static constexpr uint32_t kTotal = oAbort + 4;
     static constexpr uint32_t kBytes = kTotal + 1024;
-    static_assert(oA % 1024 == 0, "tile panels on 1024-byte boundaries");
+    static_assert(oA % 1024 == 0 && oPp % 1024 == 0, "operand tiles on 1024-byte boundaries");
 };
 
 // CTAs resident per SM (shared memory and registers are sized for it; the launch sizes its grid so)
-constexpr int kPrepPairCtasPerSm = 2;
+constexpr int kPrepPairCtasPerSm = 3;
 constexpr int kPrepPairThreads = 256;
-static_assert(kPrepPairCtasPerSm * (PrepPairSmem<128>::kBytes + 1024) <= 233472, "two CTAs per SM");
+static_assert(kPrepPairCtasPerSm * (PrepPairSmem<128>::kBytes + 1024) <= 233472, "three CTAs per SM");
 
 template <int DK>
 __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
@@ -78,16 +90,15 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
     float* A = reinterpret_cast<float*>(sm + L::oA);
-    float* P = reinterpret_cast<float*>(sm + L::oP);
     float* Tm = reinterpret_cast<float*>(sm + L::oT);
     float* M = reinterpret_cast<float*>(sm + L::oM);
     float* gam = reinterpret_cast<float*>(sm + L::oGam);
     float* bet = reinterpret_cast<float*>(sm + L::oBet);
     float* alph = reinterpret_cast<float*>(sm + L::oAlph);
-    float* pre = reinterpret_cast<float*>(sm + L::oPre);
     uint64_t* tile_full = reinterpret_cast<uint64_t*>(sm + L::oBar);
-    uint64_t* mma_bar = tile_full + 1;
-    uint64_t* drain = tile_full + 2;
+    uint64_t* mma_bar = tile_full + 1;        // the Gram product done
+    uint64_t* pt_bar = tile_full + 2;         // P T'' done
+    uint64_t* drain = tile_full + 3;
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::oTmem);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::oAbort);
 
@@ -96,12 +107,13 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
     if (tid == 0) {
         mbar_init(tile_full, 1);
         mbar_init(mma_bar, 1);
+        mbar_init(pt_bar, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(tslot, 64);      // the Gram product: 128 lanes x 64 columns
+        tmem_alloc(tslot, 64);      // the Gram product (128 lanes x 64 columns), then P T
         tmem_relinquish();
     }
     tc_fence_before();
@@ -111,9 +123,8 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
 
     // copies the [K; Q] rows of one item into the tile buffer (one thread; issued once the previous
     // item's product has read the buffer).  Panel p: K rows 0..63, then Q rows 0..63.
-    auto issue_tile = [&](int item) {
-        const int gc = item / H, h = item % H;
-        const int t0 = chunk_tab[gc].y;
+    auto issue_tile = [&](int item, int t0) {
+        const int h = item % H;
         const int t1 = (t0 < INT32_MAX - 32) ? t0 + 32 : INT32_MAX;   // rows past the tensor read as zeros
         mbar_arrive_expect_tx(tile_full, NP * L::kPanel);
 #pragma unroll
@@ -139,7 +150,7 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
         }
     };
 
-    if (tid == 0 && (int)blockIdx.x < nitems) issue_tile(blockIdx.x);
+    if (tid == 0 && (int)blockIdx.x < nitems) issue_tile(blockIdx.x, chunk_tab[blockIdx.x / H].y);
     float gv_cur[2] = {0.f, 0.f}, bv_cur[2] = {0.f, 0.f};
     if (warp == 7 && (int)blockIdx.x < nitems) load_gates(blockIdx.x, gv_cur, bv_cur);
 
@@ -149,6 +160,10 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
     for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++iter) {
         GDN_PREP_TRACE(iter, 0);
         const int gc = item / H, h = item % H;
+        const int next = item + (int)gridDim.x;
+        // first token of the next item, read now so that its copy can be issued without waiting
+        int next_t0 = 0;
+        if (tid == 64 && next < nitems) next_t0 = chunk_tab[next / H].y;
 
         // Gram products D[r][n] = [K; Q]_r . K_n, n < 64, on the tensor cores (thread 0)
         if (tid == 0) {
@@ -194,17 +209,15 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
             alph[r + 1] = a1;
             const float exclp = __shfl_up_sync(0xffffffffu, incp, 1);
             if (lane >= 16) {
-                pre[r] = (lane > 16 ? exclp : 1.f) * a0;
-                pre[r + 1] = incp;
+                A[r * LD + 67] = (lane > 16 ? exclp : 1.f) * a0;
+                A[(r + 1) * LD + 67] = incp;
             }
-            if (item + (int)gridDim.x < nitems) load_gates(item + gridDim.x, gv_cur, bv_cur);
+            if (next < nitems) load_gates(next, gv_cur, bv_cur);
         }
         __syncthreads();
         GDN_PREP_TRACE(iter, 1);
         if (*abort_flag) break;
         tc_fence_after();
-        // the tile buffer is free (the Gram product has completed): fetch the next item's rows
-        if (tid == 0 && item + (int)gridDim.x < nitems) issue_tile(item + gridDim.x);
         {
             // thread (q = warp % 4, hf = warp / 4, lane): Gram row r = 32 q + lane, columns 32 hf ..
             // 32 hf + 31.  Rows 0..63: K K^T -> A (times beta_i, strictly lower); rows 64..127:
@@ -214,25 +227,46 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
             const int r = q * 32 + lane;
             const bool isP = r >= 64;
             const int i = r & 63;
-            float d[32];
-            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 32 * hf, d);
-            tmem_ld_wait();
             const float wr = isP ? 1.f : bet[i];
             const int lim = isP ? i + 1 : i;
             const int jtop = 32 * hf + 31;
-            float a = (i > jtop) ? pre[i] : 1.f;
-            float vals[32];
+            float a = (i > jtop) ? A[i * LD + 67] : 1.f;
+            const uint32_t dst = sbase + L::oA + (uint32_t)(i * LD * 4 + hf * 128);
+            // two halves of 16 columns, high half first (the running product goes down the row).
+            // A rows: fp32 for the inverse; P rows: three bf16 parts, the A operand of P T''.
 #pragma unroll
-            for (int jj = 31; jj >= 0; --jj) {
-                const int j = 32 * hf + jj;
-                if (jj < 31) a = (j >= i) ? 1.f : a * alph[j + 1];
-                vals[jj] = (j < lim) ? wr * a * d[jj] : 0.f;
+            for (int half = 1; half >= 0; --half) {
+                float d[16];
+                tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + 32 * hf + 16 * half, d);
+                tmem_ld_wait();
+                float vals[16];
+#pragma unroll
+                for (int jj = 15; jj >= 0; --jj) {
+                    const int j = 32 * hf + 16 * half + jj;
+                    if (half == 0 || jj < 15) a = (j >= i) ? 1.f : a * alph[j + 1];
+                    vals[jj] = (j < lim) ? wr * a * d[jj] : 0.f;
+                }
+                if (!isP) {
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4)
+                        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + half * 64 + c4 * 16),
+                                     "f"(vals[4 * c4]), "f"(vals[4 * c4 + 1]), "f"(vals[4 * c4 + 2]),
+                                     "f"(vals[4 * c4 + 3]));
+                } else {
+#pragma unroll
+                    for (int g8 = 0; g8 < 2; ++g8) {
+                        uint32_t w[3][4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            bf16x2_split3(vals[8 * g8 + 2 * e], vals[8 * g8 + 2 * e + 1], w[0][e], w[1][e], w[2][e]);
+                        const uint32_t o = sw128_off_h(i, 32 * hf + 16 * half + 8 * g8, 64);
+#pragma unroll
+                        for (int pp = 0; pp < 3; ++pp)
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::oPp + pp * 8192 + o),
+                                         "r"(w[pp][0]), "r"(w[pp][1]), "r"(w[pp][2]), "r"(w[pp][3]));
+                    }
+                }
             }
-            const uint32_t dst = sbase + (isP ? L::oP : L::oA) + (uint32_t)(i * LD * 4 + hf * 128);
-#pragma unroll
-            for (int c4 = 0; c4 < 8; ++c4)
-                asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + c4 * 16), "f"(vals[4 * c4]),
-                             "f"(vals[4 * c4 + 1]), "f"(vals[4 * c4 + 2]), "f"(vals[4 * c4 + 3]));
         }
         tc_fence_before();
         __syncthreads();
@@ -250,6 +284,7 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
 #pragma unroll
                 for (int r = i + 1; r < 16; ++r) t[r] = fmaf(-A[(o + r) * LD + o + i], t[i], t[r]);
             }
+            __syncwarp();      // every lane has read this block of A before T is written over it
 #pragma unroll
             for (int r = 0; r < 16; ++r) Tm[(o + r) * LD + o + j] = t[r];
             if ((blk & 1) == 0) {
@@ -343,74 +378,78 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
         __syncthreads();
         GDN_PREP_TRACE(iter, 4);
 
-        // operator record: [T''; P T''] with T'' = T diag(beta), P T'' = (P T) diag(beta), each 8-column
-        // row segment as three bf16 parts (one 16-byte store each) in the 128-byte-swizzled image.
-        // Output blocks of 32 x 32: (a, a) and (b, b) by 64 threads each (two rows x 8 columns, sums
-        // over one chunk's rows), (b, a) by 128 threads (one row x 8 columns, sums over both chunks);
-        // the (a, b) blocks of T'' and P T'' are zero.
+        // T'' = T diag(beta): thread -> row m = tid / 4, columns 16 (tid % 4) .. + 15, as three bf16
+        // parts in the 128-byte-swizzled layout of 64 rows x 64 columns.  The same packets are the
+        // record's rows 0..63 and the B operand of P T'' (K = row m, N = column, N-major).
         uint8_t* dst = op + ((size_t)gc * H + h) * kPairRecordBytes;
         {
-            int i0, nrow, c0;
-            if (tid < 64) {
-                i0 = (tid >> 2) * 2; nrow = 2; c0 = (tid & 3) * 8;
-            } else if (tid < 128) {
-                i0 = 32 + ((tid - 64) >> 2) * 2; nrow = 2; c0 = 32 + (tid & 3) * 8;
-            } else {
-                i0 = 32 + ((tid - 128) >> 2); nrow = 1; c0 = (tid & 3) * 8;
-            }
-            const float4 b0 = *reinterpret_cast<const float4*>(bet + c0);
-            const float4 b1 = *reinterpret_cast<const float4*>(bet + c0 + 4);
-            const float bc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-            // (P T)[i][c] = sum over m in [c0, i] of P[i][m] T[m][c]  (P lower, T lower)
-            float acc[2][8];
+            const int m = tid >> 2, c0 = (tid & 3) * 16;
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr)
+            for (int g8 = 0; g8 < 2; ++g8) {
+                const int c = c0 + 8 * g8;
+                const float4 t0 = *reinterpret_cast<const float4*>(Tm + m * LD + c);
+                const float4 t1 = *reinterpret_cast<const float4*>(Tm + m * LD + c + 4);
+                const float4 b0 = *reinterpret_cast<const float4*>(bet + c);
+                const float4 b1 = *reinterpret_cast<const float4*>(bet + c + 4);
+                uint32_t w[3][4];
+                bf16x2_split3(t0.x * b0.x, t0.y * b0.y, w[0][0], w[1][0], w[2][0]);
+                bf16x2_split3(t0.z * b0.z, t0.w * b0.w, w[0][1], w[1][1], w[2][1]);
+                bf16x2_split3(t1.x * b1.x, t1.y * b1.y, w[0][2], w[1][2], w[2][2]);
+                bf16x2_split3(t1.z * b1.z, t1.w * b1.w, w[0][3], w[1][3], w[2][3]);
+                const uint32_t o = sw128_off_h(m, c, 64);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) acc[rr][c] = 0.f;
-            const int mend = i0 + nrow;                  // exclusive; P[i][m] = 0 for m > i
-            for (int m = c0; m < mend; m += 4) {
-                const float4 p0 = *reinterpret_cast<const float4*>(P + i0 * LD + m);
-                const float4 p1 = *reinterpret_cast<const float4*>(P + (i0 + 1) * LD + m);
-                const float pa[4] = {p0.x, p0.y, p0.z, p0.w}, pb[4] = {p1.x, p1.y, p1.z, p1.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float4 t0 = *reinterpret_cast<const float4*>(Tm + (m + e) * LD + c0);
-                    const float4 t1 = *reinterpret_cast<const float4*>(Tm + (m + e) * LD + c0 + 4);
-                    const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        acc[0][c] = fmaf(pa[e], tv[c], acc[0][c]);
-                        acc[1][c] = fmaf(pb[e], tv[c], acc[1][c]);
-                    }
+                for (int pp = 0; pp < 3; ++pp) {
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::oTpp + pp * 8192 + o),
+                                 "r"(w[pp][0]), "r"(w[pp][1]), "r"(w[pp][2]), "r"(w[pp][3]));
+                    stg128(dst + pp * kPairPart + o, w[pp]);
                 }
             }
-            const uint32_t zero4[4] = {0u, 0u, 0u, 0u};
-            for (int rr = 0; rr < nrow; ++rr) {
-                const int i = i0 + rr;
-                const float4 t0 = *reinterpret_cast<const float4*>(Tm + i * LD + c0);
-                const float4 t1 = *reinterpret_cast<const float4*>(Tm + i * LD + c0 + 4);
-                const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-                uint32_t w[3][4], x[3][4];
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        GDN_PREP_TRACE(iter, 6);
+        // P T'' on the tensor cores (thread 0): M = 64 (row r in lane 32 (r / 16) + r % 16), N = 64,
+        // K = 64; part products a_p t_q with p + q <= 4 into one fp32 accumulator (the Gram's columns)
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idPT = idesc_bf16(64, 64, false, true);
+            const uint64_t da = sw128_desc(sbase + L::oPp, 0, 64);
+            const uint64_t db = sw128_desc_mn(sbase + L::oTpp, 8192, 1024);
+            constexpr int pa[6] = {0, 0, 0, 1, 1, 2}, pb[6] = {0, 1, 2, 0, 1, 0};
 #pragma unroll
-                for (int c = 0; c < 8; c += 2) {
-                    bf16x2_split3(tv[c] * bc[c], tv[c + 1] * bc[c + 1], w[0][c / 2], w[1][c / 2], w[2][c / 2]);
-                    bf16x2_split3(acc[rr][c] * bc[c], acc[rr][c + 1] * bc[c + 1], x[0][c / 2], x[1][c / 2],
-                                  x[2][c / 2]);
-                }
-                const uint32_t ot = sw128_off_h(i, c0, 128), opt = sw128_off_h(64 + i, c0, 128);
+            for (int ks = 0; ks < kPair / 16; ++ks) {
 #pragma unroll
-                for (int p = 0; p < 3; ++p) {
-                    stg128(dst + p * kPairPart + ot, w[p]);
-                    stg128(dst + p * kPairPart + opt, x[p]);
-                }
-                if (tid < 64) {
-                    // the zero (a, b) blocks
-                    const uint32_t zt = sw128_off_h(i, 32 + c0, 128), zp = sw128_off_h(64 + i, 32 + c0, 128);
+                for (int u = 0; u < 6; ++u)
+                    mma_bf16(tmem, da + (uint64_t)(pa[u] * 512 + ks * 2), db + (uint64_t)(pb[u] * 512 + ks * 128), idPT,
+                             ks > 0 || u > 0);
+            }
+            mma_commit(pt_bar);
+            if (!mbar_wait(pt_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
+        }
+        __syncthreads();
+        GDN_PREP_TRACE(iter, 7);
+        tc_fence_after();
+        // the tile region is free (P T'' has read T''): fetch the next item's rows
+        if (tid == 64 && next < nitems && !*abort_flag) issue_tile(next, next_t0);
+        {
+            // P T'' rows -> record rows 64..127: warp (q, hf) lanes 0..15 hold row 16 q + lane, columns
+            // 32 hf .. 32 hf + 31 (lanes 16..31 of an M = 64 product carry no row)
+            const int q = warp & 3, hf = warp >> 2;
+            float d[32];
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 32 * hf, d);
+            tmem_ld_wait();
+            if (lane < 16) {
+                const int i = 16 * q + lane;
 #pragma unroll
-                    for (int p = 0; p < 3; ++p) {
-                        stg128(dst + p * kPairPart + zt, zero4);
-                        stg128(dst + p * kPairPart + zp, zero4);
-                    }
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    uint32_t w[3][4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        bf16x2_split3(d[8 * g8 + 2 * e], d[8 * g8 + 2 * e + 1], w[0][e], w[1][e], w[2][e]);
+                    const uint32_t o = sw128_off_h(64 + i, 32 * hf + 8 * g8, 128);
+#pragma unroll
+                    for (int pp = 0; pp < 3; ++pp) stg128(dst + pp * kPairPart + o, w[pp]);
                 }
             }
         }
@@ -420,6 +459,7 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
             const int e = tid - 128;
             gt[e] = (e < 64) ? exp2f(gam[e]) : exp2f(gam[63] - gam[e - 64]);
         }
+        tc_fence_before();
         __syncthreads();
         GDN_PREP_TRACE(iter, 5);
     }

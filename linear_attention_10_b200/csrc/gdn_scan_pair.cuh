@@ -17,14 +17,15 @@
 // step costs about what one 32-row chunk cost when half of those rows were idle; the dependent chain
 // of a sequence is half as long.
 //
-// One CTA owns MS = 32 rows of one head's state (rows of S evolve independently).  Warps 0..7 run the
-// chain; thread (q4 = warp % 4, hf = warp / 4, lane) reads tensor-memory lane 32 q4 + lane (a lane
-// quarter is only visible to the warps with that warp index mod 4) and the column half hf:
-//   * as state owner: S[hf * 16 + i][32 q4 + lane], i < 16, in registers for the whole sequence;
+// One CTA owns MS = 32 rows of one head's state (rows of S evolve independently).  Warps 0..4 NQ - 1
+// run the chain; thread (q4 = warp % 4, hq = warp / 4, lane) reads tensor-memory lane 32 q4 + lane (a
+// lane quarter is only visible to the warps with that warp index mod 4) and the hq-th group of
+// MH = 32 / NQ columns:
+//   * as state owner: S[hq * MH + i][32 q4 + lane], i < MH, in registers for the whole sequence;
 //   * q4 = 0, 1: token 32 q4 + lane of the pair: X -> Y and U -> U~ (B operands of MMA_b, MMA_c);
 //   * q4 = 2, 3: token 32 (q4 - 2) + lane: Z, then the output row O.
-// Thread 0 issues the products; warp 8 (one thread) stages each pair's K/Q/V tiles with tensor maps
-// and its operator record with a bulk copy, two stages deep.
+// Thread 0 issues the products; warp 4 NQ (one thread) stages each pair's K/Q/V tiles with tensor
+// maps and its operator record with a bulk copy, two stages deep.
 //
 // Precision: q and k are exact bf16 values and enter the products as stored.  The fp32 operands
 // (S, Y, U~ and the operator) are split into three bf16 parts stacked along N;
@@ -66,12 +67,13 @@ struct ScanPairSmem {
     static_assert(kStage % 1024 == 0 && oOp % 1024 == 0, "operand tiles on 1024-byte boundaries");
 };
 
-constexpr int kScanPairThreads = 288;
+// threads of the scan with NQ column groups per lane quarter: 4 NQ chain warps and one producer warp
+constexpr int scan_pair_threads(int nq) { return 32 * (4 * nq + 1); }
 
-// Writes the MH consecutive N-values (N = part * MS + hf * MH + i) of K-row `k` of an N-major
+// Writes the MH consecutive N-values (N = part * MS + hq * MH + i) of K-row `k` of an N-major
 // B tile as three bf16 parts: MH/8 16-byte stores per part.
 template <int MS, int MH>
-__device__ __forceinline__ void put_parts(uint32_t tile, uint32_t lbo, int k, int hf, const float (&x)[MH])
+__device__ __forceinline__ void put_parts(uint32_t tile, uint32_t lbo, int k, int hq, const float (&x)[MH])
 {
     using namespace sm100;
     uint32_t w[3][MH / 2];
@@ -81,7 +83,7 @@ __device__ __forceinline__ void put_parts(uint32_t tile, uint32_t lbo, int k, in
     for (int p = 0; p < 3; ++p) {
 #pragma unroll
         for (int g = 0; g < MH / 8; ++g) {
-            const int n0 = p * MS + hf * MH + g * 8;
+            const int n0 = p * MS + hq * MH + g * 8;
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(tile + sw128_off_nmaj(n0, k, lbo)),
                          "r"(w[p][g * 4]), "r"(w[p][g * 4 + 1]), "r"(w[p][g * 4 + 2]), "r"(w[p][g * 4 + 3]));
         }
@@ -104,8 +106,8 @@ __device__ __forceinline__ void tmem_sum3(uint32_t taddr, float (&r)[MH])
 
 // CUTS: the call has cut points (segments, snapshots); without them pair j of a sequence starts at
 // its token 64 j.  chunk_off / chunk_tab describe pairs (the plan kernel's table with 64-row entries).
-template <int DK, int DV, bool CUTS>
-__global__ void __launch_bounds__(kScanPairThreads, 1)
+template <int DK, int DV, bool CUTS, int NQ>
+__global__ void __launch_bounds__(scan_pair_threads(NQ), 1)
     gdn_scan_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const int* __restrict__ meta,
                          const int* __restrict__ order, const int* __restrict__ chunk_off,
@@ -118,7 +120,9 @@ __global__ void __launch_bounds__(kScanPairThreads, 1)
     // launched as a dependent of the prep kernel: its records (and the plan's table) are read below
     grid_dep_wait();
     constexpr int MS = 32;                    // state rows per CTA
-    constexpr int MH = 16;                    // of which one thread handles
+    constexpr int MH = MS / NQ;               // of which one thread handles
+    constexpr int NCW = 4 * NQ;               // chain warps
+    static_assert(NQ == 2 || NQ == 4, "column groups per lane quarter");
     constexpr int NP = L::NP;
     static_assert(DK == 64 || DK == 128, "DK");
     static_assert(DV % MS == 0, "DV");
@@ -182,7 +186,7 @@ __global__ void __launch_bounds__(kScanPairThreads, 1)
     const uint64_t dS = sw128_desc_mn(sbase + L::oBS, L::kLboS, 1024);
     const uint64_t dY = sw128_desc_mn(sbase + L::oBY, L::kLboY, 1024);
 
-    if (warp == 8) {
+    if (warp == NCW) {
         // ------------------------------------------------------------------ producer (one thread)
         if (lane == 0) {
             int issued = 0;
@@ -225,7 +229,7 @@ __global__ void __launch_bounds__(kScanPairThreads, 1)
         }
     } else {
         // ------------------------------------------------------------------ chain warps
-        const int q4 = warp & 3, hf = warp >> 2;
+        const int q4 = warp & 3, hq = warp >> 2;   // lane quarter, column group
         const uint32_t lane_q = (uint32_t)(q4 * 32) << 16;
         const int c_own = q4 * 32 + lane;     // dk column of the state this thread holds
         const bool owns = c_own < DK;
@@ -236,14 +240,14 @@ __global__ void __launch_bounds__(kScanPairThreads, 1)
         float S[MH];
 #pragma unroll
         for (int i = 0; i < MH; ++i)
-            S[i] = (state_in && owns) ? state_in[(((size_t)n * H + h) * DV + r0 + hf * MH + i) * DK + c_own] : 0.f;
+            S[i] = (state_in && owns) ? state_in[(((size_t)n * H + h) * DV + r0 + hq * MH + i) * DK + c_own] : 0.f;
         bool aborted = false;
         if (npair > 0) {
             // S_-1 -> three bf16 parts, the B operand of the first MMA_a
-            if (owns) put_parts<MS, MH>(sbase + L::oBS, L::kLboS, c_own, hf, S);
+            if (owns) put_parts<MS, MH>(sbase + L::oBS, L::kLboS, c_own, hq, S);
             fence_async_smem();
             tc_fence_before();
-            named_bar(1, 256);
+            named_bar(1, 32 * NCW);
         }
         for (int j = 0; j < npair; ++j) {
             const int s = j & 1;
@@ -281,15 +285,15 @@ __global__ void __launch_bounds__(kScanPairThreads, 1)
             const float* gate = reinterpret_cast<const float*>(stp + L::oOp + kPairGate);
             const float Gam = gate[tok];
             float za[MH];
-            tmem_sum3<MS, MH>(tD1 + lane_q + hf * MH, za);
+            tmem_sum3<MS, MH>(tD1 + lane_q + hq * MH, za);
             if (xrow) {
                 // Y = V - diag(Gamma) X (zero past the sequence end) -> bf16 parts of MMA_b's B
                 float y[MH];
                 const uint8_t* vrow = stp + L::oV + tok * 64;
 #pragma unroll
                 for (int q8 = 0; q8 < MH / 8; ++q8) {
-                    // 16-byte chunk (hf * MH / 8 + q8) of row `tok` at its 64-byte-swizzled place
-                    const int jc = (hf * (MH / 8) + q8) ^ ((tok >> 1) & 3);
+                    // 16-byte chunk (hq * MH / 8 + q8) of row `tok` at its 64-byte-swizzled place
+                    const int jc = (hq * (MH / 8) + q8) ^ ((tok >> 1) & 3);
                     const uint4 u = *reinterpret_cast<const uint4*>(vrow + jc * 16);
                     const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
@@ -302,11 +306,11 @@ __global__ void __launch_bounds__(kScanPairThreads, 1)
                 const bool live = tok < Lr;
 #pragma unroll
                 for (int i = 0; i < MH; ++i) y[i] = live ? fmaf(-Gam, za[i], y[i]) : 0.f;
-                put_parts<MS, MH>(sbase + L::oBY, L::kLboY, tok, hf, y);   // N = part * MS + i, K = token
+                put_parts<MS, MH>(sbase + L::oBY, L::kLboY, tok, hq, y);   // N = part * MS + i, K = token
                 fence_async_smem();
             }
             tc_fence_before();
-            if (named_bar_any(1, 256, *abort_flag)) { aborted = true; break; }
+            if (named_bar_any(1, 32 * NCW, *abort_flag)) { aborted = true; break; }
             GDN_SCAN_TRACE(j, 2);
             // ---- MMA_b: [U; P U] = [T''; P T''] Y
             if (tid == 0) {
@@ -327,16 +331,16 @@ __global__ void __launch_bounds__(kScanPairThreads, 1)
             tc_fence_after();
             {
                 float u[MH];
-                tmem_sum3<MS, MH>(tD2 + lane_q + hf * MH, u);
+                tmem_sum3<MS, MH>(tD2 + lane_q + hq * MH, u);
                 if (xrow) {
                     // U~ = diag(delta) U -> bf16 parts, B operand of MMA_c (Y has been read)
                     const float del = gate[64 + tok];
 #pragma unroll
                     for (int i = 0; i < MH; ++i) u[i] *= del;
-                    put_parts<MS, MH>(sbase + L::oBY, L::kLboY, tok, hf, u);
+                    put_parts<MS, MH>(sbase + L::oBY, L::kLboY, tok, hq, u);
                     fence_async_smem();
                     tc_fence_before();
-                    named_bar(2, 128);
+                    named_bar(2, 16 * NCW);
                     GDN_SCAN_TRACE(j, 4);
                     // ---- MMA_c: (dS)^T = K^T U~
                     if (tid == 0 && !*abort_flag) {
@@ -352,7 +356,7 @@ __global__ void __launch_bounds__(kScanPairThreads, 1)
                     float o[MH];
 #pragma unroll
                     for (int i = 0; i < MH; ++i) o[i] = scale * fmaf(Gam, za[i], u[i]);
-                    store_row<MH>(out + ((size_t)(t0 + tok) * H + h) * DV + r0 + hf * MH, o);
+                    store_row<MH>(out + ((size_t)(t0 + tok) * H + h) * DV + r0 + hq * MH, o);
                 }
             }
             // ---- state: S_j = Gamma_C S_{j-1} + dS  (row c_own of (dS)^T, this thread's MH rows)
@@ -362,7 +366,7 @@ __global__ void __launch_bounds__(kScanPairThreads, 1)
             tc_fence_after();
             if (warp_owns) {
                 float d[MH];
-                tmem_sum3<MS, MH>(tD3 + lane_q + hf * MH, d);
+                tmem_sum3<MS, MH>(tD3 + lane_q + hq * MH, d);
                 const float GamC = gate[kPair - 1];
 #pragma unroll
                 for (int i = 0; i < MH; ++i) S[i] = fmaf(GamC, S[i], d[i]);
@@ -370,17 +374,17 @@ __global__ void __launch_bounds__(kScanPairThreads, 1)
                 if (CUTS && ok && snap >= 0 && snaps != nullptr && owns) {
 #pragma unroll
                     for (int i = 0; i < MH; ++i)
-                        snaps[(((size_t)snap * H + h) * DV + r0 + hf * MH + i) * DK + c_own] = S[i];
+                        snaps[(((size_t)snap * H + h) * DV + r0 + hq * MH + i) * DK + c_own] = S[i];
                 }
             }
             if (j + 1 == npair) {
                 aborted = *abort_flag != 0;
                 break;
             }
-            if (owns) put_parts<MS, MH>(sbase + L::oBS, L::kLboS, c_own, hf, S);
+            if (owns) put_parts<MS, MH>(sbase + L::oBS, L::kLboS, c_own, hq, S);
             fence_async_smem();
             tc_fence_before();
-            if (named_bar_any(1, 256, *abort_flag)) { aborted = true; break; }
+            if (named_bar_any(1, 32 * NCW, *abort_flag)) { aborted = true; break; }
             // stage s has no reader left: its products are complete and its tiles read
             if (tid == 0) mbar_arrive(&empty[s]);
             GDN_SCAN_TRACE(j, 6);
@@ -388,7 +392,7 @@ __global__ void __launch_bounds__(kScanPairThreads, 1)
         if (state_out && owns && !aborted) {
 #pragma unroll
             for (int i = 0; i < MH; ++i)
-                state_out[(((size_t)n * H + h) * DV + r0 + hf * MH + i) * DK + c_own] = S[i];
+                state_out[(((size_t)n * H + h) * DV + r0 + hq * MH + i) * DK + c_own] = S[i];
         }
     }
     tc_fence_before();
