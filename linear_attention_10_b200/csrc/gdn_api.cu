@@ -295,7 +295,7 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         const unsigned grid = (unsigned)(items < cap ? items : cap);
         ProfScope prof("gdn_prep_pair_kernel", st);
         if (launch_dependent(k1, dim3(grid), dim3(kPrepPairThreads), PL::kBytes, st, tq, tk, g, beta,
-                             (const int*)meta, (const int4*)chunk_tab, reinterpret_cast<uint8_t*>(op), H,
+                             meta, (const int4*)chunk_tab, reinterpret_cast<uint8_t*>(op), H,
                              status) != cudaSuccess)
             return GDN_ERR_LAUNCH;
       }

@@ -23,7 +23,7 @@ namespace gdn {
 struct PrefillLayout {
     int64_t nc_max;       // upper bound on the number of 32-row chunks: floor(T / 32) + NS
     int64_t np_max;       // upper bound on the number of 64-row pairs: floor(T / 64) + NS
-    size_t off_meta;      // int32[8]: [0] chunk (or pair) count, [1] error flag
+    size_t off_meta;      // int32[8]: [0] chunk (or pair) count, [1] error flag, [2] prep item counter
     size_t off_chunk_off; // int32[NS + 1]: first global chunk (or pair) of each sequence
     size_t off_chunk_tab; // int4[nc_max]: (sequence, first token, rows, snapshot index or -1)
     size_t off_seg;       // int32[6 NS + 1]: segment start, sequence, cut, end, snapshot, chunk offset
@@ -165,6 +165,7 @@ __global__ void __launch_bounds__(1024) gdn_plan_kernel(const int32_t* __restric
             chunk_off[N] = nc;
             meta[0] = s_err ? 0 : nc;
             meta[1] = s_err;
+            meta[2] = 0;                  // the bf16 prep's item counter
             if (s_err) report(status, GDN_ERR_BAD_SEQLENS);
         }
         if (s_err) return;
@@ -268,6 +269,7 @@ __global__ void __launch_bounds__(1024) gdn_plan_kernel(const int32_t* __restric
         chunk_off[N] = nc;
         meta[0] = nc;
         meta[1] = 0;
+        meta[2] = 0;
     }
     __syncthreads();
     // global chunk -> (sequence, first token, rows, snapshot index)

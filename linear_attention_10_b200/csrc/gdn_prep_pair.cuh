@@ -62,7 +62,8 @@ struct PrepPairSmem {
     static constexpr uint32_t oAlph = oBet + 256;                    // [64] exp(g), 4 spare
     static constexpr uint32_t oBar = oAlph + 272;                    // tile_full, gram, pt, drain
     static constexpr uint32_t oTmem = oBar + 32;
-    static constexpr uint32_t oAbort = oTmem + 4;
+    static constexpr uint32_t oClaim = oTmem + 8;                   // the item claimed two ahead
+    static constexpr uint32_t oAbort = oClaim + 4;
     static constexpr uint32_t kTotal = oAbort + 4;
     static constexpr uint32_t kBytes = kTotal + 1024;
     static_assert(oA % 1024 == 0 && oPp % 1024 == 0, "operand tiles on 1024-byte boundaries");
@@ -76,7 +77,7 @@ static_assert(kPrepPairCtasPerSm * (PrepPairSmem<128>::kBytes + 1024) <= 233472,
 template <int DK>
 __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
     gdn_prep_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                         const float* __restrict__ g, const float* __restrict__ beta, const int* __restrict__ meta,
+                         const float* __restrict__ g, const float* __restrict__ beta, int* __restrict__ meta,
                          const int4* __restrict__ chunk_tab, uint8_t* __restrict__ op, int H, int* status)
 {
     using namespace sm100;
@@ -101,15 +102,21 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
     uint64_t* drain = tile_full + 3;
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::oTmem);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::oAbort);
+    volatile int* s_claim = reinterpret_cast<volatile int*>(sm + L::oClaim);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nitems = meta[0] * H;
+    // Items: each CTA starts with item blockIdx.x, then takes the next unclaimed one from a counter
+    // (zeroed by the plan kernel), so that CTAs that finish early take more items.  The item after
+    // the current one is claimed an iteration ahead, so its rows and gates can be fetched early.
+    auto claim = [&]() { return (int)gridDim.x + atomicAdd(meta + 2, 1); };
     if (tid == 0) {
         mbar_init(tile_full, 1);
         mbar_init(mma_bar, 1);
         mbar_init(pt_bar, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
+        *s_claim = ((int)blockIdx.x < nitems) ? claim() : nitems;
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -120,6 +127,7 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
+    int next = *s_claim;
 
     // copies the [K; Q] rows of one item into the tile buffer (one thread; issued once the previous
     // item's product has read the buffer).  Panel p: K rows 0..63, then Q rows 0..63.
@@ -157,13 +165,16 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
     constexpr uint32_t idG = idesc_bf16(128, 64);
     constexpr float kLog2e = 1.4426950408889634f;
     uint32_t iter = 0;
-    for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++iter) {
+    for (int item = blockIdx.x; item < nitems; ++iter) {
         GDN_PREP_TRACE(iter, 0);
         const int gc = item / H, h = item % H;
-        const int next = item + (int)gridDim.x;
-        // first token of the next item, read now so that its copy can be issued without waiting
+        // first token of the next item, read now so that its copy can be issued without waiting;
+        // and the item after it, published by the barrier below
         int next_t0 = 0;
-        if (tid == 64 && next < nitems) next_t0 = chunk_tab[next / H].y;
+        if (tid == 64 && next < nitems) {
+            next_t0 = chunk_tab[next / H].y;
+            *s_claim = claim();
+        }
 
         // Gram products D[r][n] = [K; Q]_r . K_n, n < 64, on the tensor cores (thread 0)
         if (tid == 0) {
@@ -216,6 +227,7 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
         }
         __syncthreads();
         GDN_PREP_TRACE(iter, 1);
+        const int after_next = (next < nitems) ? *s_claim : nitems;
         if (*abort_flag) break;
         tc_fence_after();
         {
@@ -462,6 +474,8 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
         tc_fence_before();
         __syncthreads();
         GDN_PREP_TRACE(iter, 5);
+        item = next;
+        next = after_next;
     }
     tc_fence_before();
     __syncthreads();
