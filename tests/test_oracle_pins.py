@@ -359,6 +359,38 @@ def test_chunk_operator_reconstructs_the_recurrence(L, gate):
     assert rel(O, o2[:, 0]) < 1e-12 and rel(S1, s2[0, 0]) < 1e-12
 
 
+@pytest.mark.parametrize("L", [33, 63, 64])
+@pytest.mark.parametrize("gate", [(-0.5, 0.0), (-4.0, -1.0)])
+def test_pair_operator_reconstructs_the_recurrence(L, gate):
+    """The same over 64 rows (two chunks of 32 carried as one step): the operator over a pair of
+    chunks gives the recurrence's outputs and state, the last pair of a sequence being short."""
+    d = 16
+    q, k, v, g, b = _one_head(L, d, 70 + L, gate)
+    S0 = 0.05 * np.random.default_rng(71).standard_normal((d, d))
+    op = oracle.chunk_operator(q, k, g, b, chunk=64)
+    O, S1 = oracle.chunk_step(op, q, k, v, S0, chunk=64)
+    o2, s2 = oracle.recurrence(q[:, None], k[:, None], v[:, None], g[:, None], b[:, None], state_in=S0[None, None])
+    assert rel(O, o2[:, 0]) < 1e-12 and rel(S1, s2[0, 0]) < 1e-12
+
+
+@pytest.mark.parametrize("gate", [(-0.5, 0.0), (-4.0, -1.0)])
+def test_pair_inverse_is_the_block_combination_of_the_chunk_inverses(gate):
+    """(I + A)^-1 over 64 rows equals [[T_a, 0], [-T_b A_ba T_a, T_b]] with T_a, T_b the two 32-row
+    chunks' own inverses and A_ba the pair's A between them: the pair operator is built from the
+    chunks' 32 x 32 solves."""
+    d = 16
+    q, k, v, g, b = _one_head(64, d, 72, gate)
+    pair = oracle.chunk_operator(q, k, g, b, chunk=64)
+    ta = oracle.chunk_operator(q[:32], k[:32], g[:32], b[:32])["T"]
+    tb = oracle.chunk_operator(q[32:], k[32:], g[32:], b[32:])["T"]
+    a_ba = pair["A"][32:, :32]
+    blocks = np.block([[ta, np.zeros((32, 32))], [-tb @ a_ba @ ta, tb]])
+    assert rel(blocks, pair["T"]) < 1e-12
+    # a plausible slip: T_ba with the wrong sign or the factors swapped
+    wrong = np.block([[ta, np.zeros((32, 32))], [-ta @ a_ba @ tb, tb]])
+    assert rel(wrong, pair["T"]) > 1e-6
+
+
 def test_cross_chunk_gram_gives_the_lookahead_identity():
     """[X_c; Z_c] from the exact state equals Gamma_C(c-1) [K;Q]_c S_{c-2}^T + G'_c U~_{c-1}: the
     identity that lets the state-dependent product of a chunk run one chunk early."""
