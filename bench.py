@@ -72,6 +72,8 @@ KERNELS = {
 # and verify figures undercount writes: ncu starts each replay from a clean L2, and 56-58 MB of the
 # written states are still resident (dirty) in L2 when the launch ends.
 TRAFFIC = {
+    "gdn_scan_pair_kernel": 202.41e6 + 23.95e6,
+    "gdn_prep_pair_kernel": 68.99e6 + 48.17e6,
     "gdn_l2norm_kernel": 67.12e6 + 21.02e6,
     "gdn_decode_step_kernel": 135.83e6 + 77.84e6,
     "gdn_decode_verify_kernel": 140.59e6 + 479.75e6,
@@ -337,14 +339,16 @@ def run_reference(args, rank, world):
 WORKLOAD_DESCS = {
     "varlen_resume": "4 packed sequences of 8192/3000/517/13000 tokens (24,709), H=32, dk=dv=128, bf16 q/k/v, "
                      "initial states ~N(0,0.05^2) per sequence, C=32, final states written",
-    "long_128k": "B=1, T=131072, H=32, dk=dv=128, bf16 q/k/v, zero initial state, C=32 (4096 sequential chunks)",
+    "long_128k": "B=1, T=131072, H=32, dk=dv=128, bf16 q/k/v, zero initial state, C=32 (4096 chunks, scanned in "
+                 "2048 sequential steps of two)",
     "tiny_fp32": "B=1, T=128 (4 chunks), H=2, dk=dv=64, fp32 q/k/v, g~U[-0.5,0), zero initial state",
 }
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel for these workloads
 # (None until captured, reset whenever the kernel changes).  long_128k: captured on its first 32,768
-# tokens (1,025 chunks; the full launch holds too much memory for a multi-pass capture) and scaled by
-# the chunk count 4,097 / 1,025, the traffic per chunk-row being the same at every length.
+# tokens (512 pairs of chunks; the full launch holds too much memory for a multi-pass capture) and
+# scaled by the pair count 2,048 / 512, the traffic per pair-row being the same at every length.
 TRAFFIC_BY_WORKLOAD = {
+    ("long_128k", "gdn_scan_pair_kernel"): (1619.04e6 + 258.44e6) * 2048 / 512,
 }
 
 

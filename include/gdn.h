@@ -95,7 +95,8 @@ int gdn_version(void);
 
 /*
  * Bytes of device workspace that gdn_chunk_prefill needs for this problem size.  Depends only on
- * total_tokens, num_seqs, H and dk (chunk tables, the per-chunk WY/UT operator and gate data).
+ * total_tokens, num_seqs, H and dk (chunk tables, the WY/UT operator and gate data per chunk or
+ * pair of chunks), and covers both dtypes.
  * Returns 0 for arguments that gdn_chunk_prefill would reject.
  */
 size_t gdn_chunk_prefill_workspace_bytes(int64_t total_tokens, int num_seqs, int H, int dk, int dv);
@@ -111,7 +112,9 @@ size_t gdn_chunk_prefill_workspace_bytes_ex(int64_t total_tokens, int num_segmen
 /*
  * Chunked prefill (Ferrite project page, Design section 03): runs the gated delta rule over every
  * token of N packed sequences, chunk size C = 32 with chunk boundaries relative to each sequence's
- * start, and writes every output o_t and each sequence's final state.
+ * start, and writes every output o_t and each sequence's final state.  With bf16 q/k/v the state is
+ * carried once per pair of chunks (64 rows; the pair's operator is built from the two chunks'
+ * 32 x 32 inverses); with fp32 q/k/v once per chunk.
  *
  *   q, k, v       device, layouts above, dtype `dtype`
  *   g, beta       device fp32 [T_total, H]
