@@ -178,6 +178,7 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
 
         // Gram products D[r][n] = [K; Q]_r . K_n, n < 64, on the tensor cores (thread 0)
         if (tid == 0) {
+            bulk_wait_read();   // the last item's record stores have read the P parts' place
             if (!mbar_wait(tile_full, iter & 1u, abort_flag)) {
                 tc_abort(status, abort_flag);
             } else {
@@ -284,31 +285,38 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
         __syncthreads();
         GDN_PREP_TRACE(iter, 2);
 
-        if (warp < 2) {
-            // the four 16 x 16 diagonal blocks of T by forward substitution: lane -> block
-            // 2 warp + lane / 16, column j
-            const int blk = 2 * warp + (lane >> 4), j = lane & 15, o = blk * 16;
-            float t[16];
+        {
+            // the four 16 x 16 diagonal blocks of T by forward substitution, four threads per column:
+            // thread (blk = tid / 64, column j, row quarter rq) holds rows 4 rq .. 4 rq + 3 of column j;
+            // the row that is final at step i comes from its owner by a shuffle
+            const int blk = tid >> 6, j = (tid >> 2) & 15, rq = tid & 3, o = blk * 16;
+            float t[4];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) t[r] = (r == j) ? 1.f : 0.f;
+            for (int e = 0; e < 4; ++e) t[e] = (4 * rq + e == j) ? 1.f : 0.f;
 #pragma unroll
             for (int i = 0; i < 15; ++i) {
+                const float ti = __shfl_sync(0xffffffffu, t[i & 3], (lane & ~3) | (i >> 2));
 #pragma unroll
-                for (int r = i + 1; r < 16; ++r) t[r] = fmaf(-A[(o + r) * LD + o + i], t[i], t[r]);
+                for (int e = 0; e < 4; ++e) {
+                    const int r = 4 * rq + e;
+                    if (r > i) t[e] = fmaf(-A[(o + r) * LD + o + i], ti, t[e]);
+                }
             }
-            __syncwarp();      // every lane has read this block of A before T is written over it
+            // every thread of this block's two warps has read the block of A before T is written over it
+            switch (blk) {      // named barriers 1..4, one per block (compile-time ids)
+            case 0: named_bar(1, 64); break;
+            case 1: named_bar(2, 64); break;
+            case 2: named_bar(3, 64); break;
+            default: named_bar(4, 64); break;
+            }
 #pragma unroll
-            for (int r = 0; r < 16; ++r) Tm[(o + r) * LD + o + j] = t[r];
+            for (int e = 0; e < 4; ++e) Tm[(o + 4 * rq + e) * LD + o + j] = t[e];
             if ((blk & 1) == 0) {
 #pragma unroll
-                for (int r = 0; r < 16; ++r) Tm[(o + r) * LD + o + 16 + j] = 0.f;   // upper right of a chunk
+                for (int e = 0; e < 4; ++e) Tm[(o + 4 * rq + e) * LD + o + 16 + j] = 0.f;   // upper right of a chunk
             }
-        } else {
             // T is zero above the chunk blocks: rows 0..31, columns 32..63
-            for (int e = tid - 64; e < 32 * 8; e += 192) {
-                const int r = e >> 3, c4 = e & 7;
-                *reinterpret_cast<float4*>(Tm + r * LD + 32 + 4 * c4) = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+            *reinterpret_cast<float4*>(Tm + (tid >> 3) * LD + 32 + 4 * (tid & 7)) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         __syncthreads();
         {
@@ -391,8 +399,9 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
         GDN_PREP_TRACE(iter, 4);
 
         // T'' = T diag(beta): thread -> row m = tid / 4, columns 16 (tid % 4) .. + 15, as three bf16
-        // parts in the 128-byte-swizzled layout of 64 rows x 64 columns.  The same packets are the
-        // record's rows 0..63 and the B operand of P T'' (K = row m, N = column, N-major).
+        // parts in the 128-byte-swizzled layout of 64 rows x 64 columns.  These 8 KB images are the
+        // B operand of P T'' (K = row m, N = column, N-major) and, copied by bulk stores, the record's
+        // rows 0..63.
         uint8_t* dst = op + ((size_t)gc * H + h) * kPairRecordBytes;
         {
             const int m = tid >> 2, c0 = (tid & 3) * 16;
@@ -410,11 +419,9 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
                 bf16x2_split3(t1.z * b1.z, t1.w * b1.w, w[0][3], w[1][3], w[2][3]);
                 const uint32_t o = sw128_off_h(m, c, 64);
 #pragma unroll
-                for (int pp = 0; pp < 3; ++pp) {
+                for (int pp = 0; pp < 3; ++pp)
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::oTpp + pp * 8192 + o),
                                  "r"(w[pp][0]), "r"(w[pp][1]), "r"(w[pp][2]), "r"(w[pp][3]));
-                    stg128(dst + pp * kPairPart + o, w[pp]);
-                }
             }
         }
         fence_async_smem();
@@ -437,7 +444,18 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
                              ks > 0 || u > 0);
             }
             mma_commit(pt_bar);
+            // record rows 0..63: the T'' images, while the product reads them too
+#pragma unroll
+            for (int pp = 0; pp < 3; ++pp) bulk_store(dst + pp * kPairPart, sbase + L::oTpp + pp * 8192, 8192);
+            bulk_commit();
             if (!mbar_wait(pt_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
+            bulk_wait_read();   // the tile region is refilled after the next barrier
+        } else if (tid >= 128) {
+            // gates, while P T'' runs: Gamma_i (i < 64), then delta_i = Gamma_63 / Gamma_i as exp2 of
+            // the difference
+            float* gt = reinterpret_cast<float*>(dst + kPairGate);
+            const int e = tid - 128;
+            gt[e] = (e < 64) ? exp2f(gam[e]) : exp2f(gam[63] - gam[e - 64]);
         }
         __syncthreads();
         GDN_PREP_TRACE(iter, 7);
@@ -445,8 +463,9 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
         // the tile region is free (P T'' has read T''): fetch the next item's rows
         if (tid == 64 && next < nitems && !*abort_flag) issue_tile(next, next_t0);
         {
-            // P T'' rows -> record rows 64..127: warp (q, hf) lanes 0..15 hold row 16 q + lane, columns
-            // 32 hf .. 32 hf + 31 (lanes 16..31 of an M = 64 product carry no row)
+            // P T'' rows -> record rows 64..127, staged as three 8 KB images in the P parts' place (the
+            // product has read them) and copied by bulk stores: warp (q, hf) lanes 0..15 hold row
+            // 16 q + lane, columns 32 hf .. 32 hf + 31 (lanes 16..31 of an M = 64 product carry no row)
             const int q = warp & 3, hf = warp >> 2;
             float d[32];
             tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 32 * hf, d);
@@ -459,24 +478,29 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         bf16x2_split3(d[8 * g8 + 2 * e], d[8 * g8 + 2 * e + 1], w[0][e], w[1][e], w[2][e]);
-                    const uint32_t o = sw128_off_h(64 + i, 32 * hf + 8 * g8, 128);
+                    const uint32_t o = sw128_off_h(i, 32 * hf + 8 * g8, 64);
 #pragma unroll
-                    for (int pp = 0; pp < 3; ++pp) stg128(dst + pp * kPairPart + o, w[pp]);
+                    for (int pp = 0; pp < 3; ++pp)
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::oPp + pp * 8192 + o),
+                                     "r"(w[pp][0]), "r"(w[pp][1]), "r"(w[pp][2]), "r"(w[pp][3]));
                 }
             }
         }
-        if (tid >= 128) {
-            // gates: Gamma_i (i < 64), then delta_i = Gamma_63 / Gamma_i as exp2 of the difference
-            float* gt = reinterpret_cast<float*>(dst + kPairGate);
-            const int e = tid - 128;
-            gt[e] = (e < 64) ? exp2f(gam[e]) : exp2f(gam[63] - gam[e - 64]);
-        }
+        fence_async_smem();
         tc_fence_before();
         __syncthreads();
         GDN_PREP_TRACE(iter, 5);
+        if (tid == 0) {
+            // record rows 64..127; the P parts' place is rewritten after the next item's first barrier
+#pragma unroll
+            for (int pp = 0; pp < 3; ++pp)
+                bulk_store(dst + pp * kPairPart + 8192, sbase + L::oPp + pp * 8192, 8192);
+            bulk_commit();
+        }
         item = next;
         next = after_next;
     }
+    if (tid == 0) bulk_wait_all();   // the record stores are complete before the CTA exits
     tc_fence_before();
     __syncthreads();
     if (tid == 0 && *abort_flag) {
