@@ -207,19 +207,20 @@ static EncodeTiledFn encode_tiled()
     return fn;
 }
 
-// [rows, inner] bf16 matrix with row stride `row_elems`, tiles of box_rows x box_inner elements;
-// rows past the end read as zeros.
+// [rows, inner] matrix of 2-byte (bf16) or 4-byte (fp32) elements with row stride `row_elems`,
+// tiles of box_rows x box_inner elements; rows past the end read as zeros.
 // swizzle: 128 or 64 (bytes of the swizzle span), 0 for none
-static bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_elems,
-                           uint32_t box_inner, uint32_t box_rows, int swizzle)
+static bool make_tmap(CUtensorMap* m, bool f32, const void* base, uint64_t inner, uint64_t rows, uint64_t row_elems,
+                      uint32_t box_inner, uint32_t box_rows, int swizzle)
 {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     cuuint64_t dims[2] = {inner, rows};
-    cuuint64_t strides[1] = {row_elems * 2};
+    cuuint64_t strides[1] = {row_elems * (f32 ? 4 : 2)};
     cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+    return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+              dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE,
               swizzle == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                              : (swizzle == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE),
@@ -276,12 +277,18 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
     }
     if (!cuda_ok(cudaPeekAtLastError(), "gdn_plan_kernel launch")) return GDN_ERR_LAUNCH;
 
+    // Tensor maps of q, k, v: 32-row boxes.  bf16: 64 features (128 bytes) per box row of q/k, 128-byte
+    // swizzle; 32 v columns, 64-byte swizzle.  fp32: 32 features (128 bytes) of q/k, 128-byte
+    // swizzle; the scan's MS v columns unswizzled.
+    constexpr int MSF = GDN_SCAN_MS;
     CUtensorMap tq{}, tk{}, tv{};
-    if constexpr (kBf16) {
+    {
         const uint64_t Tn = (uint64_t)(T_total > 0 ? T_total : 1);
-        if (!make_tmap_bf16(&tq, q, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, 128) ||
-            !make_tmap_bf16(&tk, k, (uint64_t)H * DK, Tn, (uint64_t)H * DK, 64, 32, 128) ||
-            !make_tmap_bf16(&tv, v, (uint64_t)H * DV, Tn, (uint64_t)H * DV, 32, 32, 64))
+        const bool f32 = !kBf16;
+        const uint32_t kbox = kBf16 ? 64 : 32, vbox = kBf16 ? 32 : MSF;
+        if (!make_tmap(&tq, f32, q, (uint64_t)H * DK, Tn, (uint64_t)H * DK, kbox, 32, 128) ||
+            !make_tmap(&tk, f32, k, (uint64_t)H * DK, Tn, (uint64_t)H * DK, kbox, 32, 128) ||
+            !make_tmap(&tv, f32, v, (uint64_t)H * DV, Tn, (uint64_t)H * DV, vbox, 32, kBf16 ? 64 : 0))
             return GDN_ERR_CUDA;
     }
     if constexpr (kBf16) {
@@ -308,9 +315,8 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         const int64_t cap = (int64_t)g_num_sms * 4;
         const unsigned grid = (unsigned)(items < cap ? items : cap);
         ProfScope prof("gdn_prep_kernel", st);
-        if (launch_dependent(k1, dim3(grid), dim3(128), PL::kBytes, st, static_cast<const T*>(q),
-                             static_cast<const T*>(k), g, beta, (const int*)meta, (const int4*)chunk_tab, op, H,
-                             status) != cudaSuccess)
+        if (launch_dependent(k1, dim3(grid), dim3(128), PL::kBytes, st, tq, tk, g, beta, (const int*)meta,
+                             (const int4*)chunk_tab, op, H, status) != cudaSuccess)
             return GDN_ERR_LAUNCH;
     }
     if constexpr (kBf16) {
@@ -334,24 +340,25 @@ static int launch_prefill(const PrefillLayout& lay, char* ws, const void* q, con
         }
         return GDN_OK;
     }
-    // state rows per CTA and CTAs per SM of the scan (compile-time tuning knobs)
-    constexpr int MS = GDN_SCAN_MS;
-    using S1 = ScanSmem<T, DK, MS, 1>;
-    using S2 = ScanSmem<T, DK, MS, 2>;
-    constexpr int MINB = ((S1::kBytes + 1024) * GDN_SCAN_MINB <= 228 * 1024) ? GDN_SCAN_MINB : 1;
-    constexpr int STAGES = ((S2::kBytes + 1024) * MINB <= 228 * 1024) ? 2 : 1;
-    using SL = ScanSmem<T, DK, MS, STAGES>;
-    static_assert((SL::kBytes + 1024) * MINB <= 228 * 1024, "scan kernel shared memory");
-    auto k2 = gdn_scan_tc_kernel<T, DK, DV, MS, STAGES, MINB>;
-    if (!set_dyn_smem(k2, SL::kBytes, "cudaFuncSetAttribute(max dynamic shared memory)"))
-        return GDN_ERR_LAUNCH;
-    {
-        ProfScope prof("gdn_scan_tc_kernel", st);
-        if (launch_dependent(k2, dim3((unsigned)N, H, DV / MS), dim3(256), SL::kBytes, st, static_cast<const T*>(q),
-                             static_cast<const T*>(k), static_cast<const T*>(v), (const int*)meta,
-                             (const int*)chunk_off, (const int4*)chunk_tab, (const float*)op, state_in,
-                             static_cast<T*>(out), state_out, cuts.snaps, H, status) != cudaSuccess)
+    if constexpr (!kBf16) {
+        // state rows per CTA and CTAs per SM of the scan (compile-time tuning knobs)
+        constexpr int MS = GDN_SCAN_MS;
+        using S1 = ScanSmem<T, DK, MS, 1>;
+        using S2 = ScanSmem<T, DK, MS, 2>;
+        constexpr int MINB = ((S1::kBytes + 1024) * GDN_SCAN_MINB <= 228 * 1024) ? GDN_SCAN_MINB : 1;
+        constexpr int STAGES = ((S2::kBytes + 1024) * MINB <= 228 * 1024) ? 2 : 1;
+        using SL = ScanSmem<T, DK, MS, STAGES>;
+        static_assert((SL::kBytes + 1024) * MINB <= 228 * 1024, "scan kernel shared memory");
+        auto k2 = gdn_scan_tc_kernel<T, DK, DV, MS, STAGES, MINB>;
+        if (!set_dyn_smem(k2, SL::kBytes, "cudaFuncSetAttribute(max dynamic shared memory)"))
             return GDN_ERR_LAUNCH;
+        {
+            ProfScope prof("gdn_scan_tc_kernel", st);
+            if (launch_dependent(k2, dim3((unsigned)N, H, DV / MS), dim3(256), SL::kBytes, st, tq, tk, tv, (const int*)meta,
+                                 (const int*)chunk_off, (const int4*)chunk_tab, (const float*)op, state_in,
+                                 static_cast<T*>(out), state_out, cuts.snaps, H, status) != cudaSuccess)
+                return GDN_ERR_LAUNCH;
+        }
     }
     return GDN_OK;
 }

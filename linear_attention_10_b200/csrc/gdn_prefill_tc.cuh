@@ -225,15 +225,16 @@ struct PrepSmem {
     static constexpr uint32_t kT = kP + 32 * LD * 4;                  // [32][33] T''
     static constexpr uint32_t kGam = kT + 32 * LD * 4;                // [32] gamma
     static constexpr uint32_t kBet = kGam + 128;                      // [32] beta
-    static constexpr uint32_t kBar = kBet + 128;                      // mbarriers: MMA, drain
-    static constexpr uint32_t kTmem = kBar + 16;                      // tmem base (4 B)
+    static constexpr uint32_t kBar = kBet + 128;                      // mbarriers: MMA, drain, tile
+    static constexpr uint32_t kTmem = kBar + 24;                      // tmem base (4 B)
     static constexpr uint32_t kAbort = kTmem + 4;                     // abort flag (4 B)
     static constexpr uint32_t kTotal = kAbort + 4;
     static constexpr uint32_t kBytes = kTotal + 1024;                 // + alignment slack
 };
 
 template <typename T, int DK>
-__global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                       const __grid_constant__ CUtensorMap tm_k,
                                                        const float* __restrict__ g, const float* __restrict__ beta,
                                                        const int* __restrict__ meta,
                                                        const int4* __restrict__ chunk_tab, float* __restrict__ op,
@@ -242,6 +243,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const T* __restrict__ 
     using namespace sm100;
     using L = PrepSmem<T, DK>;
     constexpr bool EXACT = L::EXACT;
+    static_assert(!EXACT, "fp32 inputs (bf16 inputs take the pair kernels)");
     constexpr int C = kChunk;
     // launched as a dependent of the plan kernel: its chunk table is read below
     grid_dep_wait();
@@ -255,6 +257,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const T* __restrict__ 
     float* gam = reinterpret_cast<float*>(sm + L::kGam);
     float* bet = reinterpret_cast<float*>(sm + L::kBet);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBar);
+    uint64_t* tile_full = bar + 2;            // the item's [K; Q] rows have landed
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::kTmem);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kAbort);
 
@@ -262,6 +265,7 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const T* __restrict__ 
     if (tid == 0) {
         mbar_init(bar, 1);
         mbar_init(bar + 1, 1);
+        mbar_init(tile_full, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -277,11 +281,21 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const T* __restrict__ 
     constexpr uint32_t idesc = idesc_tf32(64, 32);
     uint32_t iter = 0;
 
-    // The next item's global loads are issued before the current item is processed, so their
-    // latency overlaps the tensor-core product and the triangular solve.
-    constexpr int NG = 64 * (DK / 8) / 128;          // 8-element groups of [K; Q] per thread
+    // The item's [K; Q] rows arrive by the tensor-memory-access engine, in fp32, straight into the
+    // hi tile's 128-byte-swizzled layout (32 features x 32 rows per box: K rows 0..31, Q rows 32..63
+    // of each 8 KB panel); the copy of the next item is issued once the Gram product has read the
+    // tile, so it overlaps the triangular solve and the record.  Its gates are loaded a step ahead.
+    auto issue_tile = [&](int item) {
+        const int gc = item / H, h = item % H;
+        const int t0 = chunk_tab[gc].y;
+        mbar_arrive_expect_tx(tile_full, 64 * DK * 4);
+#pragma unroll
+        for (int p = 0; p < DK / 32; ++p) {
+            tma_load_2d(sbase + L::kTileHi + p * 8192, &tm_k, h * DK + 32 * p, t0, tile_full);
+            tma_load_2d(sbase + L::kTileHi + p * 8192 + 4096, &tm_q, h * DK + 32 * p, t0, tile_full);
+        }
+    };
     struct Pre {
-        Raw8<T> x[NG];
         float gv, bv;
         int gc, h, Lr;
     };
@@ -291,34 +305,41 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const T* __restrict__ 
         const int4 ct = chunk_tab[p.gc];
         const int64_t t0 = ct.y;
         p.Lr = ct.z;
-#pragma unroll
-        for (int u = 0; u < NG; ++u) {
-            const int idx = tid + 128 * u;
-            const int r = idx / (DK / 8), kg = idx % (DK / 8);
-            const int row = r & 31;
-            if (row < p.Lr) p.x[u].load((r < 32 ? k : q) + ((size_t)(t0 + row) * H + p.h) * DK + kg * 8);
-            else p.x[u].zero();
-        }
         const bool ok = tid < p.Lr;
         p.gv = ok ? __ldg(g + (size_t)(t0 + tid) * H + p.h) : 0.f;
         p.bv = ok ? __ldg(beta + (size_t)(t0 + tid) * H + p.h) : 0.f;
     };
     Pre cur, nxt;
-    if ((int)blockIdx.x < nitems) load_item(cur, blockIdx.x);
+    if ((int)blockIdx.x < nitems) {
+        load_item(cur, blockIdx.x);
+        if (tid == 0) issue_tile(blockIdx.x);
+    }
 
     for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++iter) {
         GDN_PREP_TRACE(iter, 0);
         if (item + (int)gridDim.x < nitems) load_item(nxt, item + gridDim.x);
         const int gc = cur.gc, h = cur.h;
 
-        // [K; Q] tile as fp32 (split for fp32 inputs), 64 rows x DK
-#pragma unroll
-        for (int u = 0; u < NG; ++u) {
+        // TF32 parts of the [K; Q] tile, in place: hi = x with its 13 low mantissa bits cleared, lo =
+        // x - hi; rows past the chunk's end (the next tokens, or zeros past the tensor) become zero
+        if (!mbar_wait(tile_full, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
+#pragma unroll 4
+        for (int u = 0; u < 64 * DK / 4 / 128; ++u) {
             const int idx = tid + 128 * u;
-            const int r = idx / (DK / 8), kg = idx % (DK / 8);
-            float x[8];
-            cur.x[u].get(x);
-            put8<!EXACT>(sbase + L::kTileHi, sbase + L::kTileLo, r, kg * 8, 64, x);
+            const int r = idx / (DK / 4), k0 = (idx % (DK / 4)) * 4;
+            const uint32_t o = sw128_off(r, k0, 64);
+            float4 x;
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w)
+                         : "r"(sbase + L::kTileHi + o));
+            if ((r & 31) >= cur.Lr) x = make_float4(0.f, 0.f, 0.f, 0.f);
+            float hi[4], lo[4];
+            tf32_split(x.x, hi[0], lo[0]);
+            tf32_split(x.y, hi[1], lo[1]);
+            tf32_split(x.z, hi[2], lo[2]);
+            tf32_split(x.w, hi[3], lo[3]);
+            sts4(sbase + L::kTileHi, o, hi[0], hi[1], hi[2], hi[3]);
+            sts4(sbase + L::kTileLo, o, lo[0], lo[1], lo[2], lo[3]);
         }
         if (tid < 32) {
             float gv = cur.gv;
@@ -349,6 +370,8 @@ __global__ void __launch_bounds__(128, 4) gdn_prep_kernel(const T* __restrict__ 
             }
             mma_commit(bar);
             if (!mbar_wait(bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
+            // the tile has been read: the next item's rows may land in it
+            else if (item + (int)gridDim.x < nitems) issue_tile(item + gridDim.x);
         }
         __syncthreads();
         GDN_PREP_TRACE(iter, 2);
@@ -477,16 +500,21 @@ struct ScanSmem {
     static constexpr uint32_t oBS = STAGES * kStage;                  // S: 2MS x DK
     static constexpr uint32_t oBY = oBS + 2 * MS * DK * 4;            // Y: 2MS x 32
     static constexpr uint32_t oBU = oBY + kB32;                       // U~: 2MS x 32
-    static constexpr uint32_t oBar = oBU + kB32;                      // full[S], empty[S], a, b, c
-    static constexpr uint32_t oTmem = oBar + 8 * (2 * STAGES + 4);   // + drain barrier
+    // the next chunk's rows as copied by the tensor-memory-access engine, before they are split:
+    // [K; Q] fp32 in the 128-byte-swizzled layout of the [K; Q] tile, V rows 0..31 x MS unswizzled
+    static constexpr uint32_t oRawKQ = ((oBU + kB32) + 1023) & ~1023u;
+    static constexpr uint32_t oRawV = oRawKQ + kAKQ;
+    static constexpr uint32_t oBar = oRawV + 32 * MS * 4;             // full[S], empty[S], a, b, c, drain, raw
+    static constexpr uint32_t oTmem = oBar + 8 * (2 * STAGES + 5);
     static constexpr uint32_t oAbort = oTmem + 4;
     static constexpr uint32_t kTotal = oAbort + 4;
     static constexpr uint32_t kBytes = kTotal + 1024;
 };
 
 template <typename T, int DK, int DV, int MS, int STAGES, int MINB>
-__global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                                                             const T* __restrict__ v,
+__global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                             const __grid_constant__ CUtensorMap tm_k,
+                                                             const __grid_constant__ CUtensorMap tm_v,
                                                              const int* __restrict__ meta,
                                                              const int* __restrict__ chunk_off,
                                                              const int4* __restrict__ chunk_tab,
@@ -498,6 +526,7 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
     using namespace sm100;
     using L = ScanSmem<T, DK, MS, STAGES>;
     constexpr bool EXACT = L::EXACT;
+    static_assert(!EXACT, "fp32 inputs (bf16 inputs take the pair kernels)");
     // launched as a dependent of the prep kernel: its records (and the plan's table) are read below
     grid_dep_wait();
     static_assert(MS == 16 || MS == 32, "MS");
@@ -512,6 +541,7 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
     uint64_t* bar_b = bar_a + 1;
     uint64_t* bar_c = bar_a + 2;
     uint64_t* bar_drain = bar_a + 3;
+    uint64_t* raw_full = bar_a + 4;           // the next chunk's raw rows have landed
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::oTmem);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::oAbort);
 
@@ -530,6 +560,7 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
         mbar_init(bar_b, 1);
         mbar_init(bar_c, 1);
         mbar_init(bar_drain, 1);
+        mbar_init(raw_full, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -545,41 +576,36 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
 
     if (warp >= 4) {
         // ------------------------------------------------------------------ producers
-        // Per chunk and thread: DK/64 blocks of 4 tokens x 8 features of K or Q and one 8-element
-        // group of the V slice; the [T''; P T''] image and the gates come by one bulk copy.
+        // The tensor-memory-access engine copies chunk cl + 1's [K; Q] rows (fp32, 32 features x 32
+        // rows per box, in the [K; Q] tile's 128-byte-swizzled layout) and its V rows (MS columns)
+        // into one raw buffer while chunk cl is converted; the [T''; P T''] image and the gates come
+        // by one bulk copy per stage.  Per chunk and thread: DK/64 blocks of 4 tokens x 8 features of
+        // K or Q and one 8-element group of the V slice, read back from the raw buffer, split into
+        // TF32 hi and lo parts and stored as the MMA operands (K also transposed).  Rows past the
+        // chunk's end (the next tokens, or zeros past the tensor) become zero.
         const int ptid = tid - 128;
         constexpr int NB = DK / 64;
         constexpr int NVG = 4 * MS;                    // 8-element groups in the V slice
-        struct Pre {
-            Raw8<T> kq[NB][4];
-            Raw8<T> vv;
-        };
-        auto load_chunk = [&](Pre& p, int cl) {
-            const int gc = c_begin + cl;
-            const int4 ctab = chunk_tab[gc];
-            const int64_t t0 = ctab.y;
-            const int Lr = ctab.z;
+        auto chunk_t0 = [&](int cl) { return chunk_tab[c_begin + cl].y; };
+        auto issue_raw = [&](int cl) {
+            const int t0 = chunk_t0(cl);
+            mbar_arrive_expect_tx(raw_full, L::kAKQ + 32 * MS * 4);
 #pragma unroll
-            for (int u = 0; u < NB; ++u) {
-                const int b = ptid + 128 * u;
-                const bool isq = b >= DK;
-                const int bb = isq ? b - DK : b;
-                const int jg = bb & 7, kg = bb >> 3;
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int j = 4 * jg + r;
-                    if (j < Lr) p.kq[u][r].load((isq ? q : k) + ((size_t)(t0 + j) * H + h) * DK + kg * 8);
-                    else p.kq[u][r].zero();
-                }
+            for (int p = 0; p < DK / 32; ++p) {
+                tma_load_2d(sbase + L::oRawKQ + p * 8192, &tm_k, h * DK + 32 * p, t0, raw_full);
+                tma_load_2d(sbase + L::oRawKQ + p * 8192 + 4096, &tm_q, h * DK + 32 * p, t0, raw_full);
             }
-            (void)gc;
-            if (ptid < NVG) {
-                const int j = ptid / (MS / 8), cg = ptid % (MS / 8);
-                if (j < Lr) p.vv.load(v + ((size_t)(t0 + j) * H + h) * DV + r0 + cg * 8);
-                else p.vv.zero();
-            }
+            tma_load_2d(sbase + L::oRawV, &tm_v, h * DV + r0, t0, raw_full);
         };
-        auto store_chunk = [&](const Pre& p, int s) {
+        // elements k0 .. k0 + 7 of a raw [K; Q] row: two 16-byte chunks, each at its swizzled place
+        auto raw8 = [&](int row, int k0, float (&x)[8]) {
+            const uint32_t o0 = sw128_off(row, k0, 64), o1 = sw128_off(row, k0 + 4, 64);
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3]) : "r"(sbase + L::oRawKQ + o0));
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(x[4]), "=f"(x[5]), "=f"(x[6]), "=f"(x[7]) : "r"(sbase + L::oRawKQ + o1));
+        };
+        auto store_chunk = [&](int Lr, int s) {
             const uint32_t st = sbase + s * L::kStage;
             float* stf = reinterpret_cast<float*>(sm + s * L::kStage);
 #pragma unroll
@@ -591,48 +617,50 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                 float x[4][8];
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
-                    p.kq[u][r].get(x[r]);
-                    put8<!EXACT>(st + L::oAKQh, st + L::oAKQl, (isq ? 32 : 0) + 4 * jg + r, kg * 8, 64, x[r]);
+                    const int j = 4 * jg + r;
+                    raw8((isq ? 32 : 0) + j, kg * 8, x[r]);
+                    if (j >= Lr) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) x[r][e] = 0.f;
+                    }
+                    put8<true>(st + L::oAKQh, st + L::oAKQl, (isq ? 32 : 0) + j, kg * 8, 64, x[r]);
                 }
                 if (!isq) {
                     // K^T: feature rows, 4 consecutive tokens per 16-byte store
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const uint32_t o = sw128_off(kg * 8 + e, 4 * jg, DK);
-                        if constexpr (EXACT) {
-                            sts4(st + L::oAKTh, o, x[0][e], x[1][e], x[2][e], x[3][e]);
-                        } else {
-                            float hi[4], lo[4];
+                        float hi[4], lo[4];
 #pragma unroll
-                            for (int r = 0; r < 4; ++r) tf32_split(x[r][e], hi[r], lo[r]);
-                            sts4(st + L::oAKTh, o, hi[0], hi[1], hi[2], hi[3]);
-                            sts4(st + L::oAKTl, o, lo[0], lo[1], lo[2], lo[3]);
-                        }
+                        for (int r = 0; r < 4; ++r) tf32_split(x[r][e], hi[r], lo[r]);
+                        sts4(st + L::oAKTh, o, hi[0], hi[1], hi[2], hi[3]);
+                        sts4(st + L::oAKTl, o, lo[0], lo[1], lo[2], lo[3]);
                     }
                 }
             }
             if (ptid < NVG) {
                 const int j = ptid / (MS / 8), cg = ptid % (MS / 8);
                 float x[8];
-                p.vv.get(x);
+                const float* vr = reinterpret_cast<const float*>(sm + L::oRawV) + j * MS + cg * 8;
+                const float4 v0 = *reinterpret_cast<const float4*>(vr);
+                const float4 v1 = *reinterpret_cast<const float4*>(vr + 4);
+                x[0] = v0.x; x[1] = v0.y; x[2] = v0.z; x[3] = v0.w; x[4] = v1.x; x[5] = v1.y; x[6] = v1.z; x[7] = v1.w;
                 float* Vt = stf + L::oV / 4;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) Vt[(cg * 8 + e) * 33 + j] = x[e];
+                for (int e = 0; e < 8; ++e) Vt[(cg * 8 + e) * 33 + j] = (j < Lr) ? x[e] : 0.f;
             }
         };
 
-        Pre cur, nxt;
-        if (nch > 0) load_chunk(cur, 0);
+        if (nch > 0 && ptid == 0) issue_raw(0);
+        int issued = nch > 0 ? 1 : 0;
         for (int cl = 0; cl < nch; ++cl) {
             const int s = cl % STAGES;
-            if (cl + 1 < nch) load_chunk(nxt, cl + 1);     // in flight while chunk cl is stored
             GDN_SCAN_TRACE(cl, 10);
-            if (cl >= STAGES) {
-                if (ptid == 0 && !mbar_wait(&empty[s], (uint32_t)((cl / STAGES) - 1) & 1u, abort_flag))
-                    tc_abort(status, abort_flag);
-                named_bar(1, 128);
-                if (*abort_flag) break;
-            }
+            bool ok = mbar_wait(raw_full, (uint32_t)cl & 1u, abort_flag);
+            if (ptid == 0 && ok && cl >= STAGES)
+                ok = mbar_wait(&empty[s], (uint32_t)((cl / STAGES) - 1) & 1u, abort_flag);
+            if (!ok) tc_abort(status, abort_flag);
+            if (named_bar_any(1, 128, *abort_flag)) break;
             GDN_SCAN_TRACE(cl, 11);
             if (ptid == 0) {
                 // operator image and gates: one bulk copy, counted by the same barrier
@@ -641,11 +669,21 @@ __global__ void __launch_bounds__(256, MINB) gdn_scan_tc_kernel(const T* __restr
                           reinterpret_cast<const uint8_t*>(op) + ((size_t)(c_begin + cl) * H + h) * kOpBytes,
                           kOpCopyBytes, &full[s]);
             }
-            store_chunk(cur, s);
+            store_chunk(chunk_tab[c_begin + cl].z, s);
             fence_async_smem();
             mbar_arrive(&full[s]);
+            // every producer has read the raw buffer: the next chunk's rows may land in it
+            named_bar(1, 128);
+            if (ptid == 0 && cl + 1 < nch) {
+                issue_raw(cl + 1);
+            }
+            if (cl + 1 < nch) issued = cl + 2;
             GDN_SCAN_TRACE(cl, 12);
-            cur = nxt;
+        }
+        // after an abort, a copy still in flight lands before the CTA exits (bounded)
+        if (ptid == 0 && issued > 0 && *abort_flag) {
+            volatile int never = 0;
+            mbar_wait(raw_full, (uint32_t)(issued - 1) & 1u, &never, 100000000ull);
         }
     } else {
         // ------------------------------------------------------------------ consumers
