@@ -31,9 +31,10 @@
 //   MMA_c  (dS)^T      = K^T (diag(delta) U)    M=dk, N=MS, K=32
 //
 // with the elementwise steps between them done by the epilogue warps on tensor-memory rows.  Every
-// product uses the 3xTF32 split (hi*hi + hi*lo + lo*hi); the lo terms of an operand that is
-// exactly representable in TF32 (bf16 q/k) are zero and are skipped.  Producer warps stage the
-// next chunk's operands into a second buffer while the current chunk runs.
+// product uses the 3xTF32 split (hi*hi + hi*lo + lo*hi).  These kernels serve fp32 q/k/v (bf16
+// inputs take gdn_prep_pair.cuh / gdn_scan_pair.cuh).  The tensor-memory-access engine copies the
+// chunks' fp32 q/k/v rows into shared memory and the producer warps split them into the operands
+// while the current chunk runs.
 #pragma once
 
 #include "gdn_common.cuh"
@@ -54,29 +55,6 @@ template <typename T>
 struct ExactTF32 { static constexpr bool value = false; };
 template <>
 struct ExactTF32<__nv_bfloat16> { static constexpr bool value = true; };
-
-// Loads 8 consecutive elements as fp32 (16-byte aligned for bf16, two 16-byte loads for fp32).
-template <typename T>
-__device__ __forceinline__ void load8(const T* p, float (&x)[8]);
-template <>
-__device__ __forceinline__ void load8<float>(const float* p, float (&x)[8])
-{
-    float4 a = __ldg(reinterpret_cast<const float4*>(p));
-    float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&x)[8])
-{
-    uint4 raw = __ldg(reinterpret_cast<const uint4*>(p));
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float2 f = __bfloat1622float2(h[i]);
-        x[2 * i] = f.x;
-        x[2 * i + 1] = f.y;
-    }
-}
 
 // Shared-memory stores by 32-bit shared address.  No memory clobber: the compiler may move other
 // loads and stores across them (none of the kernels' threads reads back what it stores before a
@@ -127,42 +105,6 @@ __device__ __forceinline__ void put8(uint32_t hi, uint32_t lo, int r, int k0, in
         sts4(hi, o1, x[4], x[5], x[6], x[7]);
     }
 }
-
-// Eight consecutive elements as loaded from global memory, not yet converted.  Producers keep the
-// next chunk's data in this form while they convert and store the current chunk, so the global
-// load latency of chunk c+1 overlaps the shared-memory work of chunk c.
-template <typename T>
-struct Raw8;
-template <>
-struct Raw8<__nv_bfloat16> {
-    uint4 u;
-    __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
-    __device__ __forceinline__ void zero() { u = make_uint4(0u, 0u, 0u, 0u); }
-    __device__ __forceinline__ void get(float (&x)[8]) const
-    {
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(h[i]);
-            x[2 * i] = f.x;
-            x[2 * i + 1] = f.y;
-        }
-    }
-};
-template <>
-struct Raw8<float> {
-    float4 a, b;
-    __device__ __forceinline__ void load(const float* p)
-    {
-        a = __ldg(reinterpret_cast<const float4*>(p));
-        b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-    }
-    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
-    __device__ __forceinline__ void get(float (&x)[8]) const
-    {
-        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-    }
-};
 
 // Stores N consecutive outputs with 16-byte stores (dst 16-byte aligned, N % 8 == 0).
 template <typename T, int N>
