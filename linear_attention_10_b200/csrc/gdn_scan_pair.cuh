@@ -310,7 +310,9 @@ __global__ void __launch_bounds__(scan_pair_threads(NQ), 1)
                 fence_async_smem();
             }
             tc_fence_before();
-            if (named_bar_any(1, 32 * NCW, *abort_flag)) { aborted = true; break; }
+            // MMA_b reads only the Y parts: the warps of the Z rows do not hold its issue back (the
+            // loop's abort decision is taken at the state barrier below)
+            if (xrow) named_bar(3, 16 * NCW);
             GDN_SCAN_TRACE(j, 2);
             // ---- MMA_b: [U; P U] = [T''; P T''] Y
             if (tid == 0) {
