@@ -72,7 +72,7 @@ KERNELS = {
 # and verify figures undercount writes: ncu starts each replay from a clean L2, and 56-58 MB of the
 # written states are still resident (dirty) in L2 when the launch ends.
 TRAFFIC = {
-    "gdn_scan_pair_kernel": 202.41e6 + 23.95e6,
+    "gdn_scan_pair_kernel": 202.50e6 + 24.83e6,
     "gdn_prep_pair_kernel": 68.22e6 + 46.22e6,
     "gdn_l2norm_kernel": 67.12e6 + 21.02e6,
     "gdn_decode_step_kernel": 135.83e6 + 77.84e6,
@@ -348,7 +348,7 @@ WORKLOAD_DESCS = {
 # tokens (512 pairs of chunks; the full launch holds too much memory for a multi-pass capture) and
 # scaled by the pair count 2,048 / 512, the traffic per pair-row being the same at every length.
 TRAFFIC_BY_WORKLOAD = {
-    ("long_128k", "gdn_scan_pair_kernel"): (1619.04e6 + 258.44e6) * 2048 / 512,
+    ("long_128k", "gdn_scan_pair_kernel"): (1619.12e6 + 258.24e6) * 2048 / 512,
 }
 
 
