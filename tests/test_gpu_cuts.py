@@ -70,10 +70,11 @@ def test_cuts_equal_resumed_calls_bitwise(dtype):
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 def test_cuts_at_chunk_boundaries_leave_the_prefill_unchanged(dtype):
-    """Cuts on multiples of 32 move no chunk boundary.  fp32 path: outputs and final states are those
-    of the call without cuts, bit for bit.  bf16 path: the chunk after a cut takes its products from
-    the exact state at the cut instead of the one-chunk lookahead form, so the two agree to rounding
-    (fp32-level states, at most one bf16 step on outputs)."""
+    """Cuts on multiples of 32 move no chunk boundary.  fp32 path (state carried per chunk): outputs
+    and final states are those of the call without cuts, bit for bit.  bf16 path (state carried per
+    pair of chunks): the cut at an odd multiple of 32 (288 = 256 + 32) moves the boundaries of the
+    pairs after it, so the two agree to rounding (fp32-level states, at most one bf16 step on
+    outputs)."""
     inp = make_prefill_inputs([256, 96], 2, 128, 128, dtype, "softplus", seed=42, state_std=0.05, device=DEV)
     o0, s0 = run(inp)
     out, st, sn = run_cuts(inp, [64, 128, 288])
