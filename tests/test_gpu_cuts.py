@@ -86,6 +86,22 @@ def test_cuts_at_chunk_boundaries_leave_the_prefill_unchanged(dtype):
         assert rel_err(f64(st), f64(s0)) <= 1e-5
 
 
+def test_cuts_at_pair_boundaries_leave_the_bf16_prefill_unchanged():
+    """Cuts on multiples of 64 from their sequence's start move no boundary of a pair of chunks, the
+    unit the bf16 path carries the state by: outputs and final states are those of the call without
+    cuts, bit for bit, and each snapshot is the state the recurrence reaches there."""
+    inp = make_prefill_inputs([256, 200], 2, 128, 128, "bf16", "softplus", seed=44, state_std=0.05, device=DEV)
+    o0, s0 = run(inp)
+    cuts = [64, 192, 256 + 128]
+    out, st, sn = run_cuts(inp, cuts)
+    torch.cuda.synchronize()
+    assert gdn.gdn_get_device_status() == 0
+    assert torch.equal(out, o0) and torch.equal(st, s0)
+    _, _, ref = oracle.states_at(*(f64(inp[x]) for x in ("q", "k", "v", "g", "beta")), cuts,
+                                 cu_seqlens=inp["cu_seqlens"].cpu().numpy(), state_in=f64(inp["state_in"]))
+    assert rel_err(f64(sn), ref) <= 1e-5
+
+
 @pytest.mark.parametrize("cuts", [[50, 40], [0], [100], [100, 100], [130, 400]])
 def test_bad_cuts_are_rejected_on_the_device(cuts):
     """Not increasing, at a sequence start, at a sequence end, repeated, or past the batch: the
