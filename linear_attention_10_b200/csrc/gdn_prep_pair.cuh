@@ -444,12 +444,13 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
                              ks > 0 || u > 0);
             }
             mma_commit(pt_bar);
-            // record rows 0..63: the T'' images, while the product reads them too
+            if (!mbar_wait(pt_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
+        } else if (tid == 64) {
+            // record rows 0..63: the T'' images, while the product reads them too (this thread also
+            // refills the tile region, after its stores have read it)
 #pragma unroll
             for (int pp = 0; pp < 3; ++pp) bulk_store(dst + pp * kPairPart, sbase + L::oTpp + pp * 8192, 8192);
             bulk_commit();
-            if (!mbar_wait(pt_bar, iter & 1u, abort_flag)) tc_abort(status, abort_flag);
-            bulk_wait_read();   // the tile region is refilled after the next barrier
         } else if (tid >= 128) {
             // gates, while P T'' runs: Gamma_i (i < 64), then delta_i = Gamma_63 / Gamma_i as exp2 of
             // the difference
@@ -460,8 +461,12 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
         __syncthreads();
         GDN_PREP_TRACE(iter, 7);
         tc_fence_after();
-        // the tile region is free (P T'' has read T''): fetch the next item's rows
-        if (tid == 64 && next < nitems && !*abort_flag) issue_tile(next, next_t0);
+        // the tile region is free once P T'' (completed) and the record stores (waited for here) have
+        // read T'': fetch the next item's rows
+        if (tid == 64) {
+            bulk_wait_read();
+            if (next < nitems && !*abort_flag) issue_tile(next, next_t0);
+        }
         {
             // P T'' rows -> record rows 64..127, staged as three 8 KB images in the P parts' place (the
             // product has read them) and copied by bulk stores: warp (q, hf) lanes 0..15 hold row
@@ -500,7 +505,7 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
         item = next;
         next = after_next;
     }
-    if (tid == 0) bulk_wait_all();   // the record stores are complete before the CTA exits
+    if (tid == 0 || tid == 64) bulk_wait_all();   // the record stores are complete before the CTA exits
     tc_fence_before();
     __syncthreads();
     if (tid == 0 && *abort_flag) {
