@@ -285,38 +285,31 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
         __syncthreads();
         GDN_PREP_TRACE(iter, 2);
 
-        {
-            // the four 16 x 16 diagonal blocks of T by forward substitution, four threads per column:
-            // thread (blk = tid / 64, column j, row quarter rq) holds rows 4 rq .. 4 rq + 3 of column j;
-            // the row that is final at step i comes from its owner by a shuffle
-            const int blk = tid >> 6, j = (tid >> 2) & 15, rq = tid & 3, o = blk * 16;
-            float t[4];
+        if (warp < 2) {
+            // the four 16 x 16 diagonal blocks of T by forward substitution: lane -> block
+            // 2 warp + lane / 16, column j
+            const int blk = 2 * warp + (lane >> 4), j = lane & 15, o = blk * 16;
+            float t[16];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) t[e] = (4 * rq + e == j) ? 1.f : 0.f;
+            for (int r = 0; r < 16; ++r) t[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
             for (int i = 0; i < 15; ++i) {
-                const float ti = __shfl_sync(0xffffffffu, t[i & 3], (lane & ~3) | (i >> 2));
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = 4 * rq + e;
-                    if (r > i) t[e] = fmaf(-A[(o + r) * LD + o + i], ti, t[e]);
-                }
+                for (int r = i + 1; r < 16; ++r) t[r] = fmaf(-A[(o + r) * LD + o + i], t[i], t[r]);
             }
-            // every thread of this block's two warps has read the block of A before T is written over it
-            switch (blk) {      // named barriers 1..4, one per block (compile-time ids)
-            case 0: named_bar(1, 64); break;
-            case 1: named_bar(2, 64); break;
-            case 2: named_bar(3, 64); break;
-            default: named_bar(4, 64); break;
-            }
+            __syncwarp();      // every lane has read this block of A before T is written over it
 #pragma unroll
-            for (int e = 0; e < 4; ++e) Tm[(o + 4 * rq + e) * LD + o + j] = t[e];
+            for (int r = 0; r < 16; ++r) Tm[(o + r) * LD + o + j] = t[r];
             if ((blk & 1) == 0) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) Tm[(o + 4 * rq + e) * LD + o + 16 + j] = 0.f;   // upper right of a chunk
+                for (int r = 0; r < 16; ++r) Tm[(o + r) * LD + o + 16 + j] = 0.f;   // upper right of a chunk
             }
+        } else {
             // T is zero above the chunk blocks: rows 0..31, columns 32..63
-            *reinterpret_cast<float4*>(Tm + (tid >> 3) * LD + 32 + 4 * (tid & 7)) = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int e = tid - 64; e < 32 * 8; e += 192) {
+                const int r = e >> 3, c4 = e & 7;
+                *reinterpret_cast<float4*>(Tm + r * LD + 32 + 4 * c4) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
         }
         __syncthreads();
         {
