@@ -351,6 +351,20 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
         }
         __syncthreads();
         GDN_PREP_TRACE(iter, 3);
+        // four consecutive columns of a row of T'' = T diag(beta) as three bf16 parts (8 bytes each) in
+        // the 128-byte-swizzled layout of 64 rows x 64 columns: the B operand of P T'' (K = row, N =
+        // column, N-major) and, copied by bulk stores, the record's rows 0..63
+        auto put_tpp4 = [&](int row, int col, float4 t) {
+            const float4 b = *reinterpret_cast<const float4*>(bet + col);
+            uint32_t w[3][2];
+            bf16x2_split3(t.x * b.x, t.y * b.y, w[0][0], w[1][0], w[2][0]);
+            bf16x2_split3(t.z * b.z, t.w * b.w, w[0][1], w[1][1], w[2][1]);
+            const uint32_t o = sw128_off_h(row, col, 64);
+#pragma unroll
+            for (int pp = 0; pp < 3; ++pp)
+                asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(sbase + L::oTpp + pp * 8192 + o), "r"(w[pp][0]),
+                             "r"(w[pp][1]));
+        };
         {
             // M32 = A_ba T_a (32 x 32; T_a lower triangular): thread -> row r, columns c0 .. c0 + 3
             const int r = tid >> 3, c0 = (tid & 7) * 4;
@@ -368,6 +382,10 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
                 }
             }
             *reinterpret_cast<float4*>(M + r * LM + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            // the blocks of T'' that are final already: T_a (rows 0..31), zero above it, T_b
+            put_tpp4(r, c0, *reinterpret_cast<const float4*>(Tm + r * LD + c0));
+            put_tpp4(r, 32 + c0, make_float4(0.f, 0.f, 0.f, 0.f));
+            put_tpp4(32 + r, 32 + c0, *reinterpret_cast<const float4*>(Tm + (32 + r) * LD + 32 + c0));
         }
         __syncthreads();
         {
@@ -386,40 +404,16 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
                     acc[3] = fmaf(tb[e], mv.w, acc[3]);
                 }
             }
-            *reinterpret_cast<float4*>(Tm + (32 + r) * LD + c0) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
-        }
-        __syncthreads();
-        GDN_PREP_TRACE(iter, 4);
-
-        // T'' = T diag(beta): thread -> row m = tid / 4, columns 16 (tid % 4) .. + 15, as three bf16
-        // parts in the 128-byte-swizzled layout of 64 rows x 64 columns.  These 8 KB images are the
-        // B operand of P T'' (K = row m, N = column, N-major) and, copied by bulk stores, the record's
-        // rows 0..63.
-        uint8_t* dst = op + ((size_t)gc * H + h) * kPairRecordBytes;
-        {
-            const int m = tid >> 2, c0 = (tid & 3) * 16;
-#pragma unroll
-            for (int g8 = 0; g8 < 2; ++g8) {
-                const int c = c0 + 8 * g8;
-                const float4 t0 = *reinterpret_cast<const float4*>(Tm + m * LD + c);
-                const float4 t1 = *reinterpret_cast<const float4*>(Tm + m * LD + c + 4);
-                const float4 b0 = *reinterpret_cast<const float4*>(bet + c);
-                const float4 b1 = *reinterpret_cast<const float4*>(bet + c + 4);
-                uint32_t w[3][4];
-                bf16x2_split3(t0.x * b0.x, t0.y * b0.y, w[0][0], w[1][0], w[2][0]);
-                bf16x2_split3(t0.z * b0.z, t0.w * b0.w, w[0][1], w[1][1], w[2][1]);
-                bf16x2_split3(t1.x * b1.x, t1.y * b1.y, w[0][2], w[1][2], w[2][2]);
-                bf16x2_split3(t1.z * b1.z, t1.w * b1.w, w[0][3], w[1][3], w[2][3]);
-                const uint32_t o = sw128_off_h(m, c, 64);
-#pragma unroll
-                for (int pp = 0; pp < 3; ++pp)
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::oTpp + pp * 8192 + o),
-                                 "r"(w[pp][0]), "r"(w[pp][1]), "r"(w[pp][2]), "r"(w[pp][3]));
-            }
+            const float4 tba = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+            *reinterpret_cast<float4*>(Tm + (32 + r) * LD + c0) = tba;
+            put_tpp4(32 + r, c0, tba);
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
+        GDN_PREP_TRACE(iter, 4);
+
+        uint8_t* dst = op + ((size_t)gc * H + h) * kPairRecordBytes;
         GDN_PREP_TRACE(iter, 6);
         // P T'' on the tensor cores (thread 0): M = 64 (row r in lane 32 (r / 16) + r % 16), N = 64,
         // K = 64; part products a_p t_q with p + q <= 4 into one fp32 accumulator (the Gram's columns)
