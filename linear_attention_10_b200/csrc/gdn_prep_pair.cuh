@@ -456,21 +456,24 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
         }
         {
             // P T'' rows -> record rows 64..127, staged as three 8 KB images in the P parts' place (the
-            // product has read them) and copied by bulk stores: warp (q, hf) lanes 0..15 hold row
-            // 16 q + lane, columns 32 hf .. 32 hf + 31 (lanes 16..31 of an M = 64 product carry no row)
+            // product has read them) and copied by bulk stores.  Rows 16 q .. 16 q + 15 of an M = 64
+            // product sit in lanes 0..15 of lane quarter q; warp (q, hf) reads columns 32 hf .. + 31 of
+            // them, one half of the columns per half-warp
             const int q = warp & 3, hf = warp >> 2;
-            float d[32];
-            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 32 * hf, d);
+            float d[16];
+            // lanes 0..15 of the quarter, twice: threads 0..15 columns 32 hf .. + 15, threads 16..31
+            // columns 32 hf + 16 .. + 31 of the same rows
+            tmem_ld16x2(tmem + ((uint32_t)(q * 32) << 16) + 32 * hf, d);
             tmem_ld_wait();
-            if (lane < 16) {
-                const int i = 16 * q + lane;
+            {
+                const int i = 16 * q + (lane & 15), cb = 32 * hf + 16 * (lane >> 4);
 #pragma unroll
-                for (int g8 = 0; g8 < 4; ++g8) {
+                for (int g8 = 0; g8 < 2; ++g8) {
                     uint32_t w[3][4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         bf16x2_split3(d[8 * g8 + 2 * e], d[8 * g8 + 2 * e + 1], w[0][e], w[1][e], w[2][e]);
-                    const uint32_t o = sw128_off_h(i, 32 * hf + 8 * g8, 64);
+                    const uint32_t o = sw128_off_h(i, cb + 8 * g8, 64);
 #pragma unroll
                     for (int pp = 0; pp < 3; ++pp)
                         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::oPp + pp * 8192 + o),

@@ -233,6 +233,18 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&r)[8])
                  : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
                  : "r"(taddr));
 }
+// 16 lanes x 32 bits, 16 consecutive columns, twice: thread i < 16 receives lane (quarter base + i),
+// columns [col, col + 16); thread i >= 16 lane (quarter base + i - 16), columns [col + 16, col + 32).
+__device__ __forceinline__ void tmem_ld16x2(uint32_t taddr, float (&r)[16])
+{
+    uint32_t* u = reinterpret_cast<uint32_t*>(r);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 16;"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+          "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
+        : "r"(taddr));
+}
+
 template <int N>
 __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&r)[N])
 {
