@@ -247,11 +247,14 @@ __global__ void __launch_bounds__(kPrepPairThreads, kPrepPairCtasPerSm)
             const uint32_t dst = sbase + L::oA + (uint32_t)(i * LD * 4 + hf * 128);
             // two halves of 16 columns, high half first (the running product goes down the row).
             // A rows: fp32 for the inverse; P rows: three bf16 parts, the A operand of P T''.
+            // both halves' tensor-memory loads in flight before one wait
+            float dd[2][16];
+            tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + 32 * hf + 16, dd[1]);
+            tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + 32 * hf, dd[0]);
+            tmem_ld_wait();
 #pragma unroll
             for (int half = 1; half >= 0; --half) {
-                float d[16];
-                tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + 32 * hf + 16 * half, d);
-                tmem_ld_wait();
+                const float (&d)[16] = dd[half];
                 float vals[16];
 #pragma unroll
                 for (int jj = 15; jj >= 0; --jj) {
