@@ -73,7 +73,7 @@ KERNELS = {
 # written states are still resident (dirty) in L2 when the launch ends.
 TRAFFIC = {
     "gdn_scan_pair_kernel": 202.50e6 + 24.83e6,
-    "gdn_prep_pair_kernel": 68.67e6 + 46.98e6,
+    "gdn_prep_pair_kernel": 68.21e6 + 45.12e6,
     "gdn_l2norm_kernel": 67.12e6 + 21.02e6,
     "gdn_decode_step_kernel": 135.83e6 + 77.84e6,
     "gdn_decode_verify_kernel": 140.59e6 + 479.75e6,
