@@ -20,8 +20,8 @@
 // Gram rows come out of tensor memory.  P T'' is a second tensor-core product (M = 64, N = 64,
 // K = 64): P and T'' as three bf16 parts each, the six part products with p + q <= 4 accumulated in
 // fp32, which keeps every term above 2^-24 relative (fp32-accurate).  T'' is staged in exactly the
-// byte layout of the record's rows 0..63, so the same 16-byte packets go to shared memory (the
-// product's B operand) and to the record.
+// byte layout of the record's rows 0..63 (the product's B operand), and P T'' the same way for rows
+// 64..127; both leave for the record by bulk stores from shared memory.
 //
 // Rows past a sequence's end (the pair's last rows may hold the next sequence's tokens) get g = 0
 // and beta = 0: their rows of A and columns of T'' are zero, so they never reach the scan's state.
