@@ -70,6 +70,18 @@ def test_strong_gates():
     check_full(inp, "strong-gates")
 
 
+def test_strong_gates_bf16_pairs():
+    """The bf16 path takes the cumulative gate over a pair of chunks (64 rows): with g down to -8 per
+    token it reaches -512, so Gamma_i and Gamma_C underflow to zero in fp32 inside a pair while the
+    decay ratios between nearby rows (running products) stay exact; outputs and states still match
+    the oracle, states at fp32 level."""
+    inp = make_prefill_inputs([200, 64, 31], 2, 128, 128, "bf16", "uniform", seed=9, state_std=0.05, device=DEV)
+    inp["g"] = inp["g"] * 16.0
+    out, st = check_full(inp, "strong-gates-bf16")
+    o_ref, s_ref = oracle_full(inp)
+    assert rel_err(f64(st), s_ref) <= STATE_TOL_BF16_FP32LEVEL
+
+
 def test_null_state_in_equals_zeros():
     inp = make_prefill_inputs([100], 2, 128, 128, "bf16", "softplus", seed=8, device=DEV)
     o1, s1 = run(inp)
