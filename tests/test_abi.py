@@ -58,6 +58,36 @@ def test_workspace_bytes(L):
     assert w(4096, 1, 32, 128, 128) % 256 == 0
 
 
+def _restated_workspace(T, NS, H):
+    """The prefill workspace as the header describes it: 256-byte aligned regions (meta int32[8],
+    table offsets int32[NS+1], the table int4[T/32 + NS], segments int32[6 NS + 1], the scan order
+    int32[NS]) and the operator records, [T/32 + NS][H] x 16,896 B (fp32 path) or [T/64 + NS][H] x
+    49,664 B (bf16 path), whichever is larger."""
+    al = lambda x: (x + 255) & ~255
+    nc, npair = T // 32 + NS, T // 64 + NS
+    regions = [8 * 4, (NS + 1) * 4, nc * 16, (6 * NS + 1) * 4, NS * 4, max(nc * H * 16896, npair * H * 49664)]
+    return sum(al(r) for r in regions)
+
+
+def test_workspace_bytes_match_the_documented_layout(L):
+    for T, NS, H, dk, dv in [(4096, 1, 32, 128, 128), (24709, 4, 32, 128, 128), (100, 3, 4, 64, 64),
+                             (0, 1, 2, 64, 128), (131072, 1, 32, 128, 128), (63, 7, 1, 128, 64)]:
+        assert gdn.workspace_bytes(T, NS, H, dk, dv) == _restated_workspace(T, NS, H), (T, NS, H, dk, dv)
+
+
+def test_scratch_limit_stated_in_the_header(L):
+    """The allocation-free entry point's 64 MiB scratch holds one bf16 sequence of about 2,680 tokens at
+    H = 32, d = 128 (include/gdn.h): the largest length whose workspace fits."""
+    lo, hi = 1, 1 << 20
+    while lo < hi:
+        mid = (lo + hi + 1) // 2
+        if gdn.workspace_bytes(mid, 1, 32, 128, 128) <= 64 << 20:
+            lo = mid
+        else:
+            hi = mid - 1
+    assert 2600 <= lo <= 2700, lo
+
+
 FAKE = 1 << 20   # 16-byte aligned non-null address; never dereferenced on these paths
 
 
